@@ -1,0 +1,413 @@
+/*
+ * nf4_oracle.c -- plain, slow CPU oracle for the QLoRA linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or constant with the
+ * CUDA path.  All floating point is done in fp64 unless a step's definition
+ * fixes a narrower rounding (noted where it happens).
+ *
+ * Sources (web pages; cited below by the short tag in brackets):
+ *   [CSDN]  "大模型量化从0到1（十）：bitsandbytes——一行配置就量化的最省心方案"
+ *           (aicoding.csdn.net) -- sections 5.2, 6.2, 7.1-7.2, 8.6, 12.2, 12.4
+ *   [AIQZ]  "QLoRA：用4比特行李箱装下整个大模型，单卡微调不再是梦"
+ *           (aiqz.cc) -- chapter 3 (NF4 by quantiles), chapter 4 (double quant)
+ *   [BLOG]  "从 LoRA 到 QLoRA、QA-LoRA：低秩更新如何进入量化模型"
+ *           (ludovicoyin.github.io) -- sections 1-5
+ *   [CARD]  airsota "Science Depth" card on LoRA/QLoRA -- section 3
+ *
+ * Conventions (the plainest reading where the pages leave a step open):
+ *   - x:[M,Din], A:[Din,r], B:[r,Dout], y:[M,Dout] with row-vector
+ *     activations ([BLOG] section 1 shapes; [CSDN] 12.2 Y = XW + sXAB).
+ *   - The frozen weight is stored transposed, Wt:[Dout,Din] row-major
+ *     (nn.Linear layout); flattening it row-major and cutting it into blocks
+ *     of 64 ([CSDN] 5.1) makes every block run along Din.
+ *   - Two 4-bit indices per byte ([CSDN] 5.2, last paragraph): element 2i
+ *     goes to the HIGH nibble of byte i, element 2i+1 to the low nibble.
+ *   - Activations, adapters and the dequantized weight are bf16 values; the
+ *     oracle reads them exactly as doubles and returns fp64 results.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_STATUS_NONFINITE 1
+
+/* ------------------------------------------------------------------------ */
+/* bf16 <-> fp32 helpers (storage format of the inputs and of dequant out)  */
+/* ------------------------------------------------------------------------ */
+
+static double bf16_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round an fp32 value to bf16, round-to-nearest-even on the bit pattern. */
+static uint16_t float_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) {
+        return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+    }
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Standard normal CDF and its inverse                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Phi(x) = P(Z <= x) for Z ~ N(0,1), written through the complementary
+ * error function: Phi(x) = erfc(-x/sqrt(2)) / 2. */
+double orc_normal_cdf(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
+
+/* Phi^{-1}(p): the x with Phi(x) = p.  Found from the definition alone:
+ * bisection on the monotone Phi over [-40, 40] until the bracket stops
+ * shrinking, then two Newton steps x -= (Phi(x) - p) / phi(x) to polish the
+ * last bits.  p must lie in (0, 1).  For p > 1/2 the symmetry
+ * Phi^{-1}(p) = -Phi^{-1}(1-p) is used (1-p is exact there), so the search
+ * always runs in the lower tail, where erfc keeps full relative precision. */
+double orc_normal_ppf(double p) {
+    if (!(p > 0.0 && p < 1.0)) return NAN;
+    if (p > 0.5) return -orc_normal_ppf(1.0 - p);
+    double lo = -40.0, hi = 40.0;
+    for (int it = 0; it < 200; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if (mid == lo || mid == hi) break;
+        if (orc_normal_cdf(mid) < p) lo = mid; else hi = mid;
+    }
+    double x = 0.5 * (lo + hi);
+    for (int it = 0; it < 2; ++it) {
+        double pdf = exp(-0.5 * x * x) / sqrt(2.0 * M_PI);
+        if (pdf <= 0.0) break;
+        double step = (orc_normal_cdf(x) - p) / pdf;
+        if (!isfinite(step)) break;
+        x -= step;
+    }
+    return x;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The NF4 codebook                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* [AIQZ] ch.3: levels are taken from standard-normal quantiles (Phi^{-1})
+ * of equal-probability pieces of the CDF, 16 levels.  [CSDN] 6.2: the
+ * levels are fixed (not per block), normalised to [-1,1], and the positive
+ * and negative halves are built asymmetrically so that 0 is an exact level.
+ *
+ * Reading (the formula itself is missing from the pages): 8 positive and 7
+ * negative levels plus an exact 0.  Positive side: Phi^{-1} of 9 probabilities
+ * equally spaced from `delta` down to 1/2, the last (1/2 -> 0) dropped.
+ * Negative side: the same with 8 probabilities, mirrored.  All values are
+ * divided by Phi^{-1}(delta) so the extremes are exactly -1 and +1, then
+ * rounded to fp32 and sorted ascending.  `delta` < 1 because Phi^{-1}(1) is
+ * infinite; the library default is 1 - (1/32 + 1/30)/2, the mean of the
+ * outermost interval-midpoint probabilities for 16 and for 15 equal pieces. */
+void orc_nf4_codebook(double delta, float out[16]) {
+    double v[16];
+    int n = 0;
+    double zmax = orc_normal_ppf(delta);
+    for (int i = 0; i < 8; ++i) { /* linspace(delta, 1/2, 9), last dropped */
+        double p = delta + (0.5 - delta) * (double)i / 8.0;
+        v[n++] = orc_normal_ppf(p) / zmax;
+    }
+    for (int i = 0; i < 7; ++i) { /* linspace(delta, 1/2, 8), last dropped */
+        double p = delta + (0.5 - delta) * (double)i / 7.0;
+        v[n++] = -orc_normal_ppf(p) / zmax;
+    }
+    v[n++] = 0.0;
+    /* insertion sort, ascending */
+    for (int i = 1; i < 16; ++i) {
+        double t = v[i];
+        int j = i - 1;
+        while (j >= 0 && v[j] > t) { v[j + 1] = v[j]; --j; }
+        v[j + 1] = t;
+    }
+    for (int i = 0; i < 16; ++i) out[i] = (float)v[i];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Blockwise quantization ([CSDN] 5.2) and double quantization ([CSDN] 7.2) */
+/* ------------------------------------------------------------------------ */
+
+static int zero_level_index(const float cb[16]) {
+    for (int j = 0; j < 16; ++j)
+        if (cb[j] == 0.0f) return j;
+    return -1;
+}
+
+/* Knuth's TwoSum: s = fl(x + y) and e such that s + e == x + y exactly. */
+static void two_sum(double x, double y, double *s, double *e) {
+    double ss = x + y;
+    double yy = ss - x;
+    *e = (x - (ss - yy)) + (y - yy);
+    *s = ss;
+}
+
+/* |w - p| held exactly as hi + lo (hi = fl(|w - p|)). */
+static void abs_diff_exact(double w, double p, double *hi, double *lo) {
+    double s, e;
+    two_sum(w, -p, &s, &e);
+    if (s < 0.0 || (s == 0.0 && e < 0.0)) { s = -s; e = -e; }
+    *hi = s;
+    *lo = e;
+}
+
+/* Nearest level of w in a block with absmax a: q = argmin_j |w/a - c_j|,
+ * the first minimum on ties ([CSDN] 5.2).  Multiplying through by a > 0 the
+ * rule is argmin_j |w - c_j a|, evaluated in exact real arithmetic: c_j a is
+ * an exact fp64 product of two fp32 values, and w - c_j a is kept as an
+ * unevaluated sum hi + lo of two doubles, so comparing (hi, lo) pairs
+ * lexicographically compares the exact distances.  a == 0 (an all-zero
+ * block) leaves u = w/a undefined; every weight then maps to the exact-zero
+ * level, the only level that reproduces it. */
+static int nearest_level(float w, float a, const float cb[16], int zero_idx) {
+    if (a == 0.0f) return zero_idx;
+    int best = 0;
+    double bh, bl;
+    abs_diff_exact((double)w, (double)cb[0] * (double)a, &bh, &bl);
+    for (int j = 1; j < 16; ++j) {
+        double h, l;
+        abs_diff_exact((double)w, (double)cb[j] * (double)a, &h, &l);
+        if (h < bh || (h == bh && l < bl)) { bh = h; bl = l; best = j; }
+    }
+    return best;
+}
+
+/* Quantize Wt:[rows, cols] (fp32, row-major; rows*cols a multiple of 64).
+ *   packed  [rows*cols/2]        two indices per byte, high nibble first
+ *   absmax  [nb]                 fp32 block absmax (used when dq == 0)
+ *   codes   [nb], steps [ceil(nb/dq_group)]   (used when dq != 0)
+ * Returns a status word: ORC_STATUS_NONFINITE if any weight is NaN/Inf
+ * (the pages are silent; such a block's outputs are unspecified).
+ *
+ * Double quantization reading ([CSDN] 7.2; [AIQZ] ch.4): the first-level
+ * fp32 absmax values are quantized to 8 bits and each run of dq_group (256)
+ * consecutive first-level scales shares one fp32 second-level constant.  The
+ * pages give no 8-bit code; the only 8-bit quantizer they define is absmax
+ * with rounding ([CSDN] 4.1).  Absmax values are >= 0, so the code is
+ * unsigned with 255 as the top: the stored constant is the step
+ * f = RN32(max_b a_b / 255) and code_b = round-half-even(a_b / f) in
+ * [0,255] (f = 0 gives code 0).  The weights themselves are encoded once,
+ * with the true a_b ([CSDN] 7: the second pass quantizes the scales, not
+ * the weights). */
+int orc_quantize(const float *W, int64_t rows, int64_t cols, const float cb[16],
+                 int dq, int dq_group, uint8_t *packed, float *absmax,
+                 uint8_t *codes, float *steps) {
+    const int64_t n = rows * cols;
+    const int64_t nb = n / 64;
+    const int zero_idx = zero_level_index(cb);
+    int status = 0;
+    float *a_all = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int64_t b = 0; b < nb; ++b) {
+        const float *wb = W + b * 64;
+        double a = 0.0;
+        for (int i = 0; i < 64; ++i) {
+            if (!isfinite(wb[i])) status |= ORC_STATUS_NONFINITE;
+            double m = fabs((double)wb[i]);
+            if (m > a) a = m;
+        }
+        float af = (float)a; /* exact: a is the magnitude of an fp32 value */
+        a_all[b] = af;
+        for (int i = 0; i < 64; i += 2) {
+            int q0 = nearest_level(wb[i], af, cb, zero_idx);
+            int q1 = nearest_level(wb[i + 1], af, cb, zero_idx);
+            packed[(b * 64 + i) / 2] = (uint8_t)((q0 << 4) | q1);
+        }
+        if (!dq) absmax[b] = af;
+    }
+    if (dq) {
+        int64_t ng = (nb + dq_group - 1) / dq_group;
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t b0 = g * dq_group;
+            int64_t b1 = b0 + dq_group < nb ? b0 + dq_group : nb;
+            float mx = 0.0f;
+            for (int64_t b = b0; b < b1; ++b)
+                if (a_all[b] > mx) mx = a_all[b];
+            /* RN32(mx/255): fp64 division then one rounding to fp32 is the
+             * correctly rounded fp32 quotient (53 >= 2*24+2). */
+            float f = (float)((double)mx / 255.0);
+            steps[g] = f;
+            for (int64_t b = b0; b < b1; ++b) {
+                int code = 0;
+                if (f > 0.0f) {
+                    /* a/f is a ratio of two fp32 values below 256: when it is
+                     * not a half-integer it sits at least 2^-33 (relative)
+                     * away from one, far above fp64 rounding, so rint of the
+                     * fp64 quotient is round-half-even of the exact ratio. */
+                    double qd = rint((double)a_all[b] / (double)f);
+                    if (qd < 0.0) qd = 0.0;
+                    if (qd > 255.0) qd = 255.0;
+                    code = (int)qd;
+                }
+                codes[b] = (uint8_t)code;
+            }
+        }
+    }
+    free(a_all);
+    return status;
+}
+
+/* Decoded first-level scale of block b: a_b itself, or with double
+ * quantization RN32(code_b * f_g) -- the product is exact in fp64 and is
+ * rounded once to fp32. */
+static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
+                         const uint8_t *codes, const float *steps) {
+    if (!dq) return absmax[b];
+    return (float)((double)codes[b] * (double)steps[b / dq_group]);
+}
+
+/* Dequantize ([CSDN] 5.2 w_hat = a * c_q; 8.6 the result is in the compute
+ * dtype, bf16 here): w_hat = RN_bf16(RN_fp32(a_hat * c_q)).  Output is bf16
+ * bit patterns, [rows, cols]. */
+void orc_dequantize(int64_t rows, int64_t cols, const float cb[16], int dq,
+                    int dq_group, const uint8_t *packed, const float *absmax,
+                    const uint8_t *codes, const float *steps, uint16_t *out) {
+    const int64_t n = rows * cols;
+    for (int64_t e = 0; e < n; ++e) {
+        int64_t b = e / 64;
+        uint8_t byte = packed[e / 2];
+        int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
+        float ah = block_scale(b, dq, dq_group, absmax, codes, steps);
+        float w = (float)((double)ah * (double)cb[q]);
+        out[e] = float_to_bf16_rne(w);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The layer: forward and backward in fp64                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Adapter input: x itself, or with pooling ([BLOG] sections 3-4) the mean of
+ * each run of g consecutive input features: p[m,k'] = (1/g) sum_i x[m,k'g+i]. */
+static double adapter_in(const uint16_t *X, int64_t Din, int64_t m, int64_t kp,
+                         int g) {
+    if (g == 1) return bf16_to_double(X[m * Din + kp]);
+    double s = 0.0;
+    for (int i = 0; i < g; ++i) s += bf16_to_double(X[m * Din + kp * g + i]);
+    return s / (double)g;
+}
+
+/* T = adapter_in(x) . A   ->  T:[M, r]   ([BLOG] section 2; [CSDN] 12.2) */
+void orc_adapter_down(const uint16_t *X, int64_t M, int64_t Din,
+                      const uint16_t *A, int r, int g, double *T) {
+    const int64_t Da = Din / g;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t k = 0; k < Da; ++k)
+                s += adapter_in(X, Din, m, k, g) * bf16_to_double(A[k * r + j]);
+            T[m * r + j] = s;
+        }
+}
+
+/* Forward ([BLOG] section 2 W_eff = dequant(W4) + (alpha/r) A B;
+ * [CSDN] 12.4 Y = X W_hat + s X A B with s = lora_alpha / r):
+ *   y[m,n] = sum_k x[m,k] Wt[n,k] + s * sum_j T[m,j] B[j,n].
+ * Wt is the dequantized weight (bf16 bits, [Dout, Din]).  T may be NULL. */
+void orc_forward(const uint16_t *X, int64_t M, int64_t Din, int64_t Dout,
+                 const uint16_t *Wt, const uint16_t *A, const uint16_t *B,
+                 int r, double alpha, int g, double *Y, double *T_out) {
+    const double s = alpha / (double)r;
+    double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
+    orc_adapter_down(X, M, Din, A, r, g, T);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < Dout; ++n) {
+            double base = 0.0;
+            for (int64_t k = 0; k < Din; ++k)
+                base += bf16_to_double(X[m * Din + k]) * bf16_to_double(Wt[n * Din + k]);
+            double ad = 0.0;
+            for (int j = 0; j < r; ++j) ad += T[m * r + j] * bf16_to_double(B[(int64_t)j * Dout + n]);
+            Y[m * Dout + n] = base + s * ad;
+        }
+    if (T_out) memcpy(T_out, T, sizeof(double) * (size_t)(M * r));
+    free(T);
+}
+
+/* G = dY . B^T  ->  G:[M, r] */
+void orc_grad_G(const uint16_t *dY, int64_t M, int64_t Dout, const uint16_t *B,
+                int r, double *G) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t n = 0; n < Dout; ++n)
+                s += bf16_to_double(dY[m * Dout + n]) * bf16_to_double(B[(int64_t)j * Dout + n]);
+            G[m * r + j] = s;
+        }
+}
+
+/* Backward input gradient ([CSDN] 12.4: the chain rule runs through the
+ * frozen base; W gets no gradient).  With y = x W + s adapter_in(x) A B:
+ *   dX[m,k] = sum_n dY[m,n] Wt[n,k] + (s/g) sum_j G[m,j] A[k/g, j]. */
+void orc_backward_dx(const uint16_t *dY, int64_t M, int64_t Din, int64_t Dout,
+                     const uint16_t *Wt, const uint16_t *A, const uint16_t *B,
+                     int r, double alpha, int g, double *dX) {
+    const double s = alpha / (double)r;
+    double *G = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
+    orc_grad_G(dY, M, Dout, B, r, G);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < Din; ++k) {
+            double base = 0.0;
+            for (int64_t n = 0; n < Dout; ++n)
+                base += bf16_to_double(dY[m * Dout + n]) * bf16_to_double(Wt[n * Din + k]);
+            double ad = 0.0;
+            for (int j = 0; j < r; ++j)
+                ad += G[m * r + j] * bf16_to_double(A[(k / g) * r + j]);
+            dX[m * Din + k] = base + s * ad / (double)g;
+        }
+    free(G);
+}
+
+/* Backward adapter gradients:
+ *   dA[k',j] = s sum_m adapter_in(x)[m,k'] G[m,j]      (dA:[Din/g, r])
+ *   dB[j,n]  = s sum_m T[m,j] dY[m,n]                  (dB:[r, Dout]) */
+void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
+                       int64_t Din, int64_t Dout, const uint16_t *A,
+                       const uint16_t *B, int r, double alpha, int g,
+                       double *dA, double *dB) {
+    const double s = alpha / (double)r;
+    const int64_t Da = Din / g;
+    double *G = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
+    double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
+    orc_grad_G(dY, M, Dout, B, r, G);
+    orc_adapter_down(X, M, Din, A, r, g, T);
+    if (dA) {
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < Da; ++k)
+            for (int j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m) acc += adapter_in(X, Din, m, k, g) * G[m * r + j];
+                dA[k * r + j] = s * acc;
+            }
+    }
+    if (dB) {
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < Dout; ++n)
+            for (int j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m) acc += T[m * r + j] * bf16_to_double(dY[m * Dout + n]);
+                dB[(int64_t)j * Dout + n] = s * acc;
+            }
+    }
+    free(G);
+    free(T);
+}
+
+/* Threads the OpenMP runtime will use for the parallel loops above. */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,307 @@
+"""Pins for the oracle's blockwise NF4 quantization, double quantization and
+dequantization.
+
+The rule pinned here is the one the bitsandbytes article (CSDN) gives in
+section 5.2: a = max|w| over a block of 64, u = w / a, q = argmin_j |u - c_j|,
+w_hat = a * c_q; section 7.2 for double quantization.  Every expected value is
+computed in exact rational arithmetic (``fractions``) by brute force over all
+16 levels / all 256 codes, independently of the oracle's C code.
+"""
+from fractions import Fraction as Fr
+
+import numpy as np
+import pytest
+
+from conftest import floats, read_golden
+
+BLOCK = 64
+
+
+# ---------------------------------------------------------------- helpers
+
+def unpack(packed, n):
+    out = np.empty(n, dtype=np.int64)
+    out[0::2] = packed >> 4        # element 2i -> high nibble
+    out[1::2] = packed & 0x0F
+    return out
+
+
+def exact_argmin(w, a, cb):
+    if a == 0:
+        return int(np.flatnonzero(cb == 0)[0])
+    wf, af = Fr(float(w)), Fr(float(a))
+    best, bd = None, None
+    for j, c in enumerate(cb):
+        d = abs(wf - Fr(float(c)) * af)
+        if bd is None or d < bd:
+            best, bd = j, d
+    return best
+
+
+def rn32(fr):
+    """Round an exact rational to the nearest fp32, ties to even."""
+    x = np.float32(float(fr))
+    cands = [x, np.nextafter(x, np.float32(np.inf)), np.nextafter(x, np.float32(-np.inf))]
+    return min(cands, key=lambda c: (abs(Fr(float(c)) - fr), int(c.view(np.uint32)) & 1))
+
+
+def bf16_of_f32(x):
+    """RNE fp32 -> bf16 bits, for finite x."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def blocks_to_W(blocks):
+    flat = np.concatenate([np.asarray(b, dtype=np.float32) for b in blocks])
+    return flat.reshape(len(blocks), BLOCK)
+
+
+# ---------------------------------------------------------------- NF4 indices
+
+def test_random_blocks_bruteforce(orc):
+    rng = np.random.default_rng(1)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_normal((12, 128)) * 0.02).astype(np.float32)
+    W[3, :64] *= 1e-30          # a block of tiny (subnormal-adjacent) values
+    W[5, 64:] = rng.standard_t(3, 64).astype(np.float32)
+    q = orc.quantize(W, cb, double_quant=False)
+    assert q.status == 0
+    flat = W.reshape(-1)
+    idx = unpack(q.packed, flat.size)
+    for b in range(flat.size // BLOCK):
+        blk = flat[b * BLOCK:(b + 1) * BLOCK]
+        a = np.float32(np.max(np.abs(blk)))
+        assert q.absmax[b] == a
+        for i in range(BLOCK):
+            assert idx[b * BLOCK + i] == exact_argmin(blk[i], a, cb), (b, i)
+
+
+def _adversarial_blocks(cb, a):
+    """Blocks holding values at and within a few ulps of every decision
+    threshold (c_j + c_{j+1})/2 * a, plus +-a to fix the absmax."""
+    vals = []
+    af = Fr(float(a))
+    for j in range(15):
+        t = (Fr(float(cb[j])) + Fr(float(cb[j + 1]))) / 2 * af
+        x = rn32(t)
+        for k in range(-3, 4):
+            y = x
+            step = np.float32(np.inf) if k > 0 else np.float32(-np.inf)
+            for _ in range(abs(k)):
+                y = np.nextafter(y, step)
+            vals.append(y)
+    vals = np.array(vals, dtype=np.float32)
+    blocks = []
+    for s in range(0, len(vals), BLOCK - 2):
+        chunk = list(vals[s:s + BLOCK - 2])
+        chunk += [np.float32(0.0)] * (BLOCK - 2 - len(chunk))
+        blocks.append([a, -a] + chunk)
+    return blocks
+
+
+@pytest.mark.parametrize("a", [np.float32(1.0), np.float32(0.0371), np.float32(3.1e-3),
+                               np.float32(2.0 ** -120), np.float32(1.7e30)])
+def test_near_threshold_bruteforce(orc, a):
+    cb = orc.nf4_codebook()
+    W = blocks_to_W(_adversarial_blocks(cb, a))
+    q = orc.quantize(W, cb, double_quant=False)
+    idx = unpack(q.packed, W.size)
+    flat = W.reshape(-1)
+    for e in range(flat.size):
+        blk = flat[(e // BLOCK) * BLOCK:(e // BLOCK + 1) * BLOCK]
+        am = np.float32(np.max(np.abs(blk)))
+        assert idx[e] == exact_argmin(flat[e], am, cb), e
+
+
+def test_ties_go_to_lower_index(orc):
+    """With a codebook whose midpoints are exact fp32 values, a weight exactly
+    on a midpoint is equidistant from two levels: argmin takes the first."""
+    cb = np.array([-1, -.75, -.5, -.375, -.25, -.125, -.0625, 0,
+                   .0625, .125, .25, .375, .5, .625, .75, 1], dtype=np.float32)
+    a = np.float32(2.0)
+    mids = [(cb[j] + cb[j + 1]) / 2 * a for j in range(15)]
+    blk = [a] + mids + [np.float32(0)] * (BLOCK - 16)
+    q = orc.quantize(blocks_to_W([blk]), cb, double_quant=False)
+    idx = unpack(q.packed, BLOCK)
+    assert list(idx[1:16]) == list(range(15))
+
+
+def test_exact_where_naive_fp64_would_tie(orc):
+    """A level of -2^-60 next to -0.5: for w = -a/4 the distance to -2^-60*a
+    is smaller by 2^-60 a, below fp64 resolution of |w - c a|.  The exact rule
+    picks the tiny level."""
+    cb = np.array([-1, -.9, -.8, -.7, -.6, -.5, -2.0 ** -60, 0,
+                   .5, .6, .7, .75, .8, .85, .9, 1], dtype=np.float32)
+    a = np.float32(1.0)
+    blk = [a, np.float32(-0.25)] + [np.float32(0)] * (BLOCK - 2)
+    q = orc.quantize(blocks_to_W([blk]), cb, double_quant=False)
+    idx = unpack(q.packed, BLOCK)
+    assert idx[1] == exact_argmin(np.float32(-0.25), a, cb) == 6
+
+
+def test_codebook_round_trip(orc):
+    """A block whose entries are c_j * a with a a power of two maps back to
+    index j, and dequantizes to RN_bf16(c_j * a)."""
+    cb = orc.nf4_codebook()
+    for a in (np.float32(1.0), np.float32(2.0 ** -7), np.float32(64.0)):
+        vals = (cb * a).astype(np.float32)
+        blk = np.tile(vals, 4)
+        q = orc.quantize(blk.reshape(1, BLOCK), cb, double_quant=False)
+        idx = unpack(q.packed, BLOCK)
+        assert list(idx) == list(range(16)) * 4
+        assert q.absmax[0] == a
+        deq = orc.dequantize(q, cb)
+        assert np.array_equal(deq.reshape(-1), bf16_of_f32(blk))
+
+
+def test_special_blocks(orc):
+    cb = orc.nf4_codebook()
+    zero = [np.float32(0)] * BLOCK
+    negzero = [np.float32(-0.0)] * BLOCK
+    pm = [np.float32(0.5), np.float32(-0.5)] + [np.float32(0.01)] * (BLOCK - 2)
+    q = orc.quantize(blocks_to_W([zero, negzero, pm]), cb, double_quant=False)
+    idx = unpack(q.packed, 3 * BLOCK)
+    assert np.all(idx[:2 * BLOCK] == 7) and q.absmax[0] == 0 and q.absmax[1] == 0
+    assert idx[2 * BLOCK] == 15 and idx[2 * BLOCK + 1] == 0
+    # nibble order: element 0 (-> 15) is the high nibble of byte 0
+    assert q.packed[BLOCK] == 0xF0
+
+
+def test_nonfinite_flagged(orc):
+    cb = orc.nf4_codebook()
+    W = np.zeros((2, BLOCK), dtype=np.float32)
+    W[1, 3] = np.nan
+    assert orc.quantize(W, cb, double_quant=False).status == orc.STATUS_NONFINITE
+    W[1, 3] = np.inf
+    assert orc.quantize(W, cb, double_quant=True).status == orc.STATUS_NONFINITE
+    W[1, 3] = 1.0
+    assert orc.quantize(W, cb, double_quant=True).status == 0
+
+
+def test_dequant_error_bound(orc):
+    """Dequantization does not recover the weight (information is lost,
+    bitsandbytes article, misconception 19) but the fp32 reconstruction is
+    within half the widest codebook gap times the absmax."""
+    rng = np.random.default_rng(7)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_normal((8, 256)) * 0.02).astype(np.float32)
+    q = orc.quantize(W, cb, double_quant=False)
+    idx = unpack(q.packed, W.size)
+    a = np.repeat(q.absmax.astype(np.float64), BLOCK)
+    rec = a * cb.astype(np.float64)[idx]
+    gap = np.max(np.diff(cb.astype(np.float64))) / 2
+    assert np.all(np.abs(rec - W.reshape(-1)) <= a * gap * (1 + 1e-6))
+    assert not np.array_equal(rec.astype(np.float32), W.reshape(-1))
+
+
+# ---------------------------------------------------------------- double quant
+
+def _dq_blocks(absmaxes):
+    return blocks_to_W([[np.float32(a)] + [np.float32(0)] * (BLOCK - 1) for a in absmaxes])
+
+
+def _expected_dq(absmaxes, group=256):
+    codes, steps = [], []
+    for g0 in range(0, len(absmaxes), group):
+        grp = absmaxes[g0:g0 + group]
+        mx = max(Fr(float(x)) for x in grp)
+        f = rn32(mx / 255)
+        steps.append(f)
+        for x in grp:
+            if f == 0:
+                codes.append(0)
+                continue
+            xf, ff = Fr(float(x)), Fr(float(f))
+            # brute force over all 256 codes; ties to the even code
+            codes.append(min(range(256), key=lambda c: (abs(c * ff - xf), c & 1)))
+    return np.array(codes, dtype=np.uint8), np.array(steps, dtype=np.float32)
+
+
+def test_double_quant_bruteforce(orc):
+    rng = np.random.default_rng(3)
+    cb = orc.nf4_codebook()
+    am = np.abs(rng.standard_normal(256 + 37) * 0.05).astype(np.float32)   # partial last group
+    am[5] = 0.0
+    am[293 - 7] = np.float32(np.max(am[256:]) * 0.5 + 1e-7)
+    q = orc.quantize(_dq_blocks(am), cb, double_quant=True)
+    codes, steps = _expected_dq(list(am))
+    assert np.array_equal(q.steps, steps)
+    assert np.array_equal(q.codes, codes)
+
+
+def test_double_quant_half_way_codes(orc):
+    """absmax values that sit exactly half-way between two codes round to the
+    even code (round-half-even of the exact ratio)."""
+    f = np.float32(2.0 ** -10)
+    am = [np.float32(255 * f)] + [np.float32((k + 0.5) * f) for k in range(0, 254, 9)]
+    q = orc.quantize(_dq_blocks(am), orc.nf4_codebook(), double_quant=True)
+    assert q.steps[0] == f
+    for a, c in zip(am[1:], q.codes[1:]):
+        k = int(a / f - 0.5)
+        assert c == (k if k % 2 == 0 else k + 1)
+
+
+def test_double_quant_properties(orc):
+    rng = np.random.default_rng(4)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_t(5, (64, 1024)) * 0.02).astype(np.float32)
+    q = orc.quantize(W, cb, double_quant=True)
+    q0 = orc.quantize(W, cb, double_quant=False)
+    a = q0.absmax
+    ng = len(q.steps)
+    assert ng == (a.size + 255) // 256
+    for g in range(ng):
+        sl = slice(g * 256, (g + 1) * 256)
+        f = np.float64(q.steps[g])
+        ahat = (q.codes[sl].astype(np.float64) * f).astype(np.float32).astype(np.float64)
+        assert np.all(np.abs(ahat - a[sl]) <= f / 2 * (1 + 1e-6) + np.spacing(a[sl]))
+        assert q.codes[sl][np.argmax(a[sl])] == 255, "the group max maps to the top code"
+    # the weights are encoded once, with the true absmax: indices do not change
+    assert np.array_equal(q.packed, q0.packed)
+
+
+def test_double_quant_exact_round_trip(orc):
+    """If every absmax is an integer multiple of 2^k and the group max is
+    255 * 2^k, the step is exactly 2^k and every scale decodes exactly."""
+    k = -12
+    am = np.array([255 * 2.0 ** k] + [m * 2.0 ** k for m in range(0, 255)], dtype=np.float32)
+    cb = orc.nf4_codebook()
+    q = orc.quantize(_dq_blocks(am), cb, double_quant=True)
+    assert q.steps[0] == np.float32(2.0 ** k)
+    dec = (q.codes.astype(np.float64) * float(q.steps[0])).astype(np.float32)
+    assert np.array_equal(dec, am)
+    # and the dequantized weights equal those of the non-DQ path
+    q0 = orc.quantize(_dq_blocks(am), cb, double_quant=False)
+    assert np.array_equal(orc.dequantize(q, cb), orc.dequantize(q0, cb))
+
+
+# ---------------------------------------------------------------- bits per parameter
+
+def test_bits_per_parameter_closed_forms(orc):
+    g = read_golden("double_quant_overhead.txt")
+    rng = np.random.default_rng(5)
+    cb = orc.nf4_codebook()
+    rows, cols = 256, 4096        # N = 64 * 256 * 64: whole DQ groups
+    W = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    n = rows * cols
+    q0 = orc.quantize(W, cb, double_quant=False)
+    q1 = orc.quantize(W, cb, double_quant=True)
+    bits0 = 8 * q0.nbytes / n
+    bits1 = 8 * q1.nbytes / n
+    assert bits0 == 4 + float(g["overhead_no_dq_bits"]) == 4.5
+    assert bits1 - 4 == 8 / 64 + 32 / (64 * 256) == 0.126953125
+    assert round(bits1 - 4, 3) == float(g["overhead_dq_bits"])
+    saving = bits0 - bits1
+    assert saving == 0.373046875 and round(saving, 3) == float(g["saving_bits"])
+    for item in g["saving_GB"].split():
+        params, gb = item.split(":")
+        assert round(float(params) * saving / 8 / 1e9, 2) == float(gb)
+
+
+def test_dq_overhead_partial_group(orc):
+    """A weight whose block count is not a multiple of 256 stores one extra
+    (partial-group) fp32 constant."""
+    cb = orc.nf4_codebook()
+    W = np.ones((3, 64 * 100), dtype=np.float32)       # nb = 300
+    q = orc.quantize(W, cb, double_quant=True)
+    assert q.codes.size == 300 and q.steps.size == 2
