@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA linear layer (NF4 + double quant + LoRA) on B200.
+
+One step = the whole hot path on one batch: nf4_quantize of the frozen
+weight (fp32 -> NF4 + double-quantized absmax), qlora_forward and
+qlora_backward (dX, dA, dB), on the training-shaped 7B up-projection
+workload (Din=4096, Dout=11008, M=4096 tokens, r=64, alpha=128, W ~ t5*0.02).
+With N > 1 ranks each rank runs its own batch (weak scaling) and the adapter
+gradients dA, dB are summed over ranks with NCCL (the data-parallel exchange).
+
+Prints ONE JSON line on rank 0.  `--impl reference` times the CPU oracle
+(the only reference there is) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_nf4_quantized_22_b200 import synth  # noqa: E402
+
+CFG = 3
+WORKLOAD = "7B up-projection Din=4096 Dout=11008 M=4096 r=64 alpha=128 NF4+DQ (quantize+fwd+bwd)"
+METRIC = "QLoRA linear fwd+bwd TFLOP/s (quantize+fwd+bwd step)"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def layer_flops(M, Din, Dout, r):
+    """Algorithmic flops of forward + backward (no dW)."""
+    fwd = 2 * M * Din * Dout + 2 * M * r * (Din + Dout)
+    bwd = 2 * M * Din * Dout + 4 * M * r * (Din + Dout)
+    return fwd + bwd
+
+
+def weight_bytes(Din, Dout, dq=True):
+    n = Din * Dout
+    nb = n // 64
+    return n // 2 + (nb + 4 * ((nb + 255) // 256) if dq else 4 * nb)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return (d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured")
+    return (6650.0, 1590.0, 1400.0, "fallback")
+
+
+def stored_traffic(kernel_file, summary):
+    """dram bytes per launch recorded in a profiles/ summary, if the kernel
+    source is unchanged since that capture (sha256 line), else None."""
+    path = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "bit_nf4_quantized_22_b200", "csrc", kernel_file)
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    vals = {}
+    for line in open(path):
+        if line.startswith("bench:"):
+            k, v = line[len("bench:"):].split("=", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], None, set()
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import oracle
+    spec = synth.CONFIGS[CFG]["linears"][0]
+    M = synth.CONFIGS[CFG]["M"][0]
+    a = synth.draw(spec, M, CFG)
+    cb = oracle.nf4_codebook()
+    S = args.ref_rows
+    flops = layer_flops(S, spec.Din, spec.Dout, spec.r)
+
+    def step(i):
+        rows = (np.arange(S) * 131 + i * 17) % M
+        qw = oracle.quantize(a["W"], cb, True)
+        Wt = oracle.dequantize(qw, cb)
+        oracle.forward(a["x"][rows], Wt, a["A"], a["B"], spec.r, spec.alpha)
+        oracle.backward(a["x"][rows], a["dY"][rows], Wt, a["A"], a["B"], spec.r, spec.alpha)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = flops / dt / 1e12
+    sample = (f"{S} of {M} token rows per step (forward, dX, dA, dB on those rows) "
+              f"+ full-weight quantize/dequantize")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def cpu_baseline(rows=256):
+    """The oracle as it stands on a bounded sample of the workload."""
+    import oracle
+    spec = synth.CONFIGS[CFG]["linears"][0]
+    M = synth.CONFIGS[CFG]["M"][0]
+    a = synth.draw(spec, M, CFG)
+    cb = oracle.nf4_codebook()
+    sel = np.arange(rows)
+    t0 = time.perf_counter()
+    qw = oracle.quantize(a["W"], cb, True)
+    Wt = oracle.dequantize(qw, cb)
+    oracle.forward(a["x"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
+    oracle.backward(a["x"][sel], a["dY"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
+    dt = time.perf_counter() - t0
+    return {"value": layer_flops(rows, spec.Din, spec.Dout, spec.r) / dt / 1e12, "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows} of {M} token rows (forward, dX, dA, dB) + full-weight quantize; "
+                      f"{dt:.1f} s"}
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import bit_nf4_quantized_22_b200 as q
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    lib = q.load()
+    hbm, tf_burst, tf_sus, peak_src = peaks()
+    spec = synth.CONFIGS[CFG]["linears"][0]
+    M = synth.CONFIGS[CFG]["M"][0]
+    Din, Dout, r, alpha = spec.Din, spec.Dout, spec.r, spec.alpha
+
+    base = synth.draw(spec, M, CFG, 0, which=("W", "A", "B"))
+    batch = synth.draw(spec, M, CFG, rank, which=("x", "dY"))
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    W_h = torch.from_numpy(base["W"]).pin_memory()
+    x_h, A_h, B_h, dy_h = (bf(batch["x"]).pin_memory(), bf(base["A"]).pin_memory(),
+                           bf(base["B"]).pin_memory(), bf(batch["dY"]).pin_memory())
+    W, x, A, B, dy = (W_h.to(dev), x_h.to(dev), A_h.to(dev), B_h.to(dev), dy_h.to(dev))
+    w = q.NF4Weight.empty(Dout, Din, True, dev)
+    ws_f = torch.empty(q.workspace_size(M, w, r, 1, 0), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.workspace_size(M, w, r, 1, 1), dtype=torch.uint8, device=dev)
+    y = torch.empty(M, Dout, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        q.quantize(W, double_quant=True, out=w)
+        _, T = q.forward(x, w, A, B, alpha, out=y, workspace=ws_f)
+        dX, dA, dB = q.backward(x, dy, w, A, B, alpha, T=T, workspace=ws_b)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+        return dX, dA, dB
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---------------- timed region: K steps, L2 flushed between steps
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    lib.qlora_profile_reset()
+    lib.qlora_profile_enable(1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    lib.qlora_profile_enable(0)
+    launches = lib.qlora_launch_count()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    import ctypes
+    umma_n, umma_ms = ctypes.c_int64(), ctypes.c_double()
+    quant_n, quant_ms = ctypes.c_int64(), ctypes.c_double()
+    lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
+    lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    flops_step = layer_flops(M, Din, Dout, r)
+    value = world * args.steps * flops_step / (total_ms / 1e3) / 1e12
+
+    # dominant kernel: the tcgen05 GEMM (forward and dX launches)
+    umma_flops = args.steps * (2 * M * Din * Dout + 2 * M * Dout * r      # forward + adapter ext
+                               + 2 * M * Dout * Din + 2 * M * Din * r)    # dX + adapter ext
+    umma_tf = umma_flops / (umma_ms.value / 1e3) / 1e12 if umma_ms.value > 0 else None
+    traffic = stored_traffic("umma_gemm.cu", "k_umma_qgemm_up_proj_4096x11008_M4096.md")
+    roof = {"bound": "tensor", "kernel": "k_umma_qgemm", "achieved": umma_tf, "peak": tf_sus,
+            "unit": "TFLOP/s", "frac": (umma_tf / tf_sus) if umma_tf else None,
+            "traffic": traffic, "peak_kind": f"bf16 dense, sustained ({peak_src})",
+            "launches": int(umma_n.value),
+            "share_of_step": umma_ms.value / sum(step_ms) if step_ms else None}
+    qbytes = Din * Dout * 4 + weight_bytes(Din, Dout)
+    quant = {"kernel": "k_nf4_quantize", "bound": "hbm",
+             "achieved": qbytes / (quant_ms.value / quant_n.value / 1e3) / 1e9 if quant_n.value else None,
+             "peak": hbm, "unit": "GB/s"}
+    if quant["achieved"]:
+        quant["frac"] = quant["achieved"] / hbm
+
+    # ---------------- end to end through the public API, host buffers
+    y_h = torch.empty(M, Dout, dtype=torch.bfloat16).pin_memory()
+    dX_h = torch.empty(M, Din, dtype=torch.bfloat16).pin_memory()
+    dA_h = torch.empty(Din, r, dtype=torch.float32).pin_memory()
+    dB_h = torch.empty(r, Dout, dtype=torch.float32).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    es.record()
+    for _ in range(e2e_steps):
+        W.copy_(W_h, non_blocking=True)
+        x.copy_(x_h, non_blocking=True)
+        A.copy_(A_h, non_blocking=True)
+        B.copy_(B_h, non_blocking=True)
+        dy.copy_(dy_h, non_blocking=True)
+        dX, dA, dB = step()
+        y_h.copy_(y, non_blocking=True)
+        dX_h.copy_(dX, non_blocking=True)
+        dA_h.copy_(dA, non_blocking=True)
+        dB_h.copy_(dB, non_blocking=True)
+    ee.record()
+    torch.cuda.synchronize()
+    e2e_ms = es.elapsed_time(ee)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (W_h, x_h, A_h, B_h, dy_h))
+    d2h = sum(t.numel() * t.element_size() for t in (y_h, dX_h, dA_h, dB_h))
+    e2e = {"value": world * e2e_steps * flops_step / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    # ---------------- decode-shaped GEMV lines (M = 1, 16; forward only)
+    extras = {}
+    if not args.no_extras:
+        extras = decode_lines(args, q, lib, torch, dev, hbm, flush)
+
+    if rank != 0:
+        return
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy PCG64; W~t5*0.02, x,dY~N(0,1), A~N(0,1/r), B~N(0,1e-4))",
+        "config": {"workload": WORKLOAD, "M": M, "Din": Din, "Dout": Dout, "r": r, "alpha": alpha,
+                   "double_quant": True, "parallelism": f"dp{world}",
+                   "l2": "flushed between timed steps (256 MB write, outside the step events)"},
+        "roofline": roof,
+        "quantize_roofline": quant,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
+        "decode": extras,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+    print(json.dumps(out), flush=True)
+
+
+def decode_lines(args, q, lib, torch, dev, hbm, flush):
+    """Forward-only decode steps (the GEMV path): weight GB/s and the GEMV
+    kernel's HBM roofline fraction, L2 flushed before every launch."""
+    import ctypes
+    res = {}
+    for cfg, lin in ((2, 0), (5, 0)):
+        spec = synth.CONFIGS[cfg]["linears"][lin]
+        base = synth.draw(spec, 16, cfg, lin, which=("W", "A", "B"))
+        W = torch.from_numpy(base["W"]).to(dev)
+        w = q.quantize(W, double_quant=True)
+        del W
+
+        def bf(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        A, B = bf(base["A"]), bf(base["B"])
+        for M in (1, 16):
+            x = bf(synth.draw(spec, M, cfg, lin, which=("x",))["x"])
+            ws = torch.empty(max(1, q.workspace_size(M, w, spec.r, 1, 0)), dtype=torch.uint8, device=dev)
+            y = torch.empty(M, spec.Dout, dtype=torch.bfloat16, device=dev)
+            for _ in range(5):
+                q.forward(x, w, A, B, spec.alpha, out=y, workspace=ws, save_T=False)
+            reps = 30
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(reps)]
+            torch.cuda.synchronize()
+            lib.qlora_profile_reset()
+            lib.qlora_profile_enable(1)
+            for s, e in ev:
+                flush.zero_()
+                s.record()
+                q.forward(x, w, A, B, spec.alpha, out=y, workspace=ws, save_T=False)
+                e.record()
+            torch.cuda.synchronize()
+            lib.qlora_profile_enable(0)
+            n, ms = ctypes.c_int64(), ctypes.c_double()
+            lib.qlora_profile_read(1, ctypes.byref(n), ctypes.byref(ms))
+            step = statistics.median(s.elapsed_time(e) for s, e in ev)
+            wb = weight_bytes(spec.Din, spec.Dout)
+            alg = wb + 2 * M * spec.Din + 2 * M * spec.Dout + 2 * spec.r * (spec.Din + spec.Dout) + 4 * M * spec.r
+            kern_ms = ms.value / max(1, n.value)
+            res[f"{spec.Din}x{spec.Dout}_M{M}"] = {
+                "forward_ms": step, "weight_GBps": wb / (step / 1e3) / 1e9,
+                "kernel": "k_gemv_fwd", "kernel_ms": kern_ms,
+                "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
+                "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None,
+                "tflops": (2 * M * spec.Din * spec.Dout + 2 * M * spec.r * (spec.Din + spec.Dout)) / (step / 1e3) / 1e12,
+            }
+        del w
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

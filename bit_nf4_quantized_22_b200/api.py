@@ -1,0 +1,191 @@
+"""Python binding of the QLoRA layer library.
+
+Argument marshalling only: every function hands device pointers, sizes and
+the current CUDA stream to the C ABI (include/qlora.h) and every step of the
+computation runs in the library's CUDA kernels.  PyTorch provides device
+memory (tensors, the workspace) and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from .codebook import nf4_codebook
+
+BLOCK = 64
+DQ_GROUP = 256
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cb_host(codebook: torch.Tensor | None) -> ctypes.Array:
+    cb = nf4_codebook() if codebook is None else codebook.detach().to("cpu", torch.float32)
+    arr = (ctypes.c_float * 16)(*cb.tolist())
+    return arr
+
+
+def _need(t: torch.Tensor, dtype, name: str, dims: int):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != dims:
+        raise TypeError(f"{name}: expected a {dims}-D {dtype} tensor")
+    if not t.is_cuda:
+        raise TypeError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise TypeError(f"{name}: must be contiguous")
+
+
+@dataclass
+class NF4Weight:
+    """A quantized frozen weight Wt:[rows = Dout, cols = Din] (device buffers)."""
+    rows: int
+    cols: int
+    double_quant: bool
+    packed: torch.Tensor                   # uint8 [rows*cols/2]
+    absmax: torch.Tensor | None = None     # fp32 [nb]
+    codes: torch.Tensor | None = None      # uint8 [nb]
+    steps: torch.Tensor | None = None      # fp32 [ceil(nb/256)]
+
+    @staticmethod
+    def empty(rows: int, cols: int, double_quant: bool, device="cuda") -> "NF4Weight":
+        nb = rows * cols // BLOCK
+        packed = torch.empty(rows * cols // 2, dtype=torch.uint8, device=device)
+        if double_quant:
+            ng = (nb + DQ_GROUP - 1) // DQ_GROUP
+            return NF4Weight(rows, cols, True, packed,
+                             codes=torch.empty(nb, dtype=torch.uint8, device=device),
+                             steps=torch.empty(ng, dtype=torch.float32, device=device))
+        return NF4Weight(rows, cols, False, packed,
+                         absmax=torch.empty(nb, dtype=torch.float32, device=device))
+
+    def c_struct(self) -> _lib.NF4WeightC:
+        return _lib.NF4WeightC(
+            self.rows, self.cols, BLOCK, int(self.double_quant), DQ_GROUP, 0,
+            self.packed.data_ptr(),
+            self.absmax.data_ptr() if self.absmax is not None else None,
+            self.codes.data_ptr() if self.codes is not None else None,
+            self.steps.data_ptr() if self.steps is not None else None)
+
+    @property
+    def nbytes(self) -> int:
+        n = self.packed.numel()
+        for t in (self.absmax, self.codes, self.steps):
+            if t is not None:
+                n += t.numel() * t.element_size()
+        return n
+
+
+def load():
+    """Load libqlora.so; raises if it is missing (no fallback exists)."""
+    return _lib.load()
+
+
+def check_codebook(codebook: torch.Tensor) -> int:
+    return load().qlora_check_codebook(_cb_host(codebook))
+
+
+def quantize(W: torch.Tensor, double_quant: bool = True, codebook: torch.Tensor | None = None,
+             status: torch.Tensor | None = None, out: NF4Weight | None = None) -> NF4Weight:
+    """nf4_quantize on W (fp32 [Dout, Din], CUDA)."""
+    _need(W, torch.float32, "W", 2)
+    rows, cols = W.shape
+    q = out if out is not None else NF4Weight.empty(rows, cols, double_quant, W.device)
+    qc = q.c_struct()
+    rc = load().nf4_quantize(_ptr(W), ctypes.byref(qc), _cb_host(codebook), _ptr(status), _stream())
+    _lib.check(rc, "nf4_quantize")
+    return q
+
+
+def dequantize(q: NF4Weight, codebook: torch.Tensor | None = None,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=torch.bfloat16,
+                                                  device=q.packed.device)
+    qc = q.c_struct()
+    rc = load().nf4_dequantize(ctypes.byref(qc), _cb_host(codebook), _ptr(out), _stream())
+    _lib.check(rc, "nf4_dequantize")
+    return out
+
+
+def workspace_size(M: int, q: NF4Weight, r: int, pool_group: int = 1, which: int = 0) -> int:
+    qc = q.c_struct()
+    return int(load().qlora_workspace_size(M, ctypes.byref(qc), r, pool_group, which))
+
+
+def _workspace(nbytes: int, device, ws: torch.Tensor | None):
+    if nbytes == 0:
+        return None, 0
+    if ws is not None and ws.numel() >= nbytes:
+        return ws, ws.numel()
+    return torch.empty(nbytes, dtype=torch.uint8, device=device), nbytes
+
+
+def forward(x: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+            pool_group: int = 1, codebook: torch.Tensor | None = None, save_T: bool = True,
+            workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+            out: torch.Tensor | None = None):
+    """y = x dequant(W4) + (alpha/r) (u A) B.  Returns (y bf16 [M, Dout], T fp32 [M, r] or None)."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(A, torch.bfloat16, "A", 2)
+    _need(B, torch.bfloat16, "B", 2)
+    M = x.shape[0]
+    r = A.shape[1]
+    y = out if out is not None else torch.empty(M, q.rows, dtype=torch.bfloat16, device=x.device)
+    T = torch.empty(M, r, dtype=torch.float32, device=x.device) if save_T else None
+    ws, nbytes = _workspace(workspace_size(M, q, r, pool_group, 0), x.device, workspace)
+    qc = q.c_struct()
+    rc = load().qlora_forward(_ptr(x), M, ctypes.byref(qc), _cb_host(codebook), _ptr(A), _ptr(B),
+                              r, float(alpha), pool_group, _ptr(y), _ptr(T), _ptr(ws), nbytes,
+                              _ptr(status), _stream())
+    _lib.check(rc, "qlora_forward")
+    return y, T
+
+
+def backward(x: torch.Tensor | None, dy: torch.Tensor, q: NF4Weight, A: torch.Tensor,
+             B: torch.Tensor, alpha: float, pool_group: int = 1, T: torch.Tensor | None = None,
+             need_dx: bool = True, need_dA: bool = True, need_dB: bool = True,
+             codebook: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+             status: torch.Tensor | None = None):
+    """Returns (dX bf16 [M, Din] | None, dA fp32 | None, dB fp32 | None); W4 gets none."""
+    _need(dy, torch.bfloat16, "dy", 2)
+    _need(A, torch.bfloat16, "A", 2)
+    _need(B, torch.bfloat16, "B", 2)
+    M = dy.shape[0]
+    r = A.shape[1]
+    dev = dy.device
+    dX = torch.empty(M, q.cols, dtype=torch.bfloat16, device=dev) if need_dx else None
+    dA = torch.empty(A.shape[0], r, dtype=torch.float32, device=dev) if need_dA else None
+    dB = torch.empty(r, q.rows, dtype=torch.float32, device=dev) if need_dB else None
+    ws, nbytes = _workspace(workspace_size(M, q, r, pool_group, 1), dev, workspace)
+    qc = q.c_struct()
+    rc = load().qlora_backward(_ptr(x), _ptr(dy), M, ctypes.byref(qc), _cb_host(codebook),
+                               _ptr(A), _ptr(B), r, float(alpha), pool_group, _ptr(T), _ptr(dX),
+                               _ptr(dA), _ptr(dB), _ptr(ws), nbytes, _ptr(status), _stream())
+    _lib.check(rc, "qlora_backward")
+    return dX, dA, dB
+
+
+class QLoRALinearFn(torch.autograd.Function):
+    """Autograd wrapper: gradients for x, A and B; none for the frozen W4."""
+
+    @staticmethod
+    def forward(ctx, x, A, B, q: NF4Weight, alpha: float, pool_group: int):
+        y, T = forward(x, q, A, B, alpha, pool_group)
+        ctx.save_for_backward(x, A, B, T)
+        ctx.q, ctx.alpha, ctx.pool = q, alpha, pool_group
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, A, B, T = ctx.saved_tensors
+        dX, dA, dB = backward(x, dy.contiguous(), ctx.q, A, B, ctx.alpha, ctx.pool, T=T,
+                              need_dx=ctx.needs_input_grad[0], need_dA=ctx.needs_input_grad[1],
+                              need_dB=ctx.needs_input_grad[2])
+        return (dX, None if dA is None else dA.to(A.dtype), None if dB is None else dB.to(B.dtype),
+                None, None, None)

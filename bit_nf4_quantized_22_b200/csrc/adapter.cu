@@ -1,0 +1,196 @@
+// adapter.cu -- the rank-r adapter products and their helpers.
+//
+//   T  = u . A        u = x, or pool(x) = mean over runs of 64 inputs
+//   G  = dY . B^T
+//   dA = s u^T G      dB = s T^T dY
+//
+// (LoRA/QLoRA/QA-LoRA blog sections 2-5; bitsandbytes article (CSDN) 12.2.)
+// All four are skinny GEMMs run on the warp-MMA tiled GEMM.  fp32 operands
+// (T, G, pool(x)) are carried as two bf16 terms hi + lo, hi = RN_bf16(v),
+// lo = RN_bf16(v - hi), which keeps ~16 mantissa bits; the GEMM multiplies
+// both terms and the reduce kernel adds the two halves in fp32.
+#include "mma_gemm.cuh"
+
+namespace qlora {
+namespace {
+
+__device__ __forceinline__ uint16_t to_bf16(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+__device__ __forceinline__ float from_bf16(uint16_t v) {
+    return __bfloat162float(__ushort_as_bfloat16(v));
+}
+
+// dst[i][j] = j < r ? src[(i / rep)][j] * mul : 0     (dst: [rows][rp])
+__global__ void k_pad_rows(const uint16_t *__restrict__ src, int64_t rows, int r, int rp, int rep,
+                           float mul, uint16_t *__restrict__ dst) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * rp) return;
+    const int64_t row = i / rp;
+    const int j = (int)(i % rp);
+    dst[i] = j < r ? to_bf16(from_bf16(src[(row / rep) * r + j]) * mul) : (uint16_t)0;
+}
+
+// pool(x)[m][k'] = (1/g) sum_i x[m][k' g + i], emitted as hi/lo bf16 terms
+// into [M][ld] buffers (columns k' >= Din/g are zero).
+__global__ void k_pool_split(const uint16_t *__restrict__ X, int64_t M, int64_t Din, int g,
+                             int64_t ld, uint16_t *__restrict__ hi, uint16_t *__restrict__ lo) {
+    const int64_t Da = Din / g;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= M * ld) return;
+    const int64_t m = i / ld, k = i % ld;
+    if (k >= Da) {
+        hi[i] = 0;
+        lo[i] = 0;
+        return;
+    }
+    const uint16_t *p = X + m * Din + k * g;
+    float sum = 0.f;
+    for (int e = 0; e < g; ++e) sum += from_bf16(p[e]);
+    const float v = sum / (float)g;
+    const uint16_t h = to_bf16(v);
+    hi[i] = h;
+    lo[i] = to_bf16(v - from_bf16(h));
+}
+
+// fp32 [rows][r] -> bf16 [rows][2 rp] = [hi | lo] with zero padding
+__global__ void k_split_f32(const float *__restrict__ src, int64_t rows, int r, int rp,
+                            uint16_t *__restrict__ dst) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * rp) return;
+    const int64_t row = i / rp;
+    const int j = (int)(i % rp);
+    uint16_t h = 0, l = 0;
+    if (j < r) {
+        const float v = src[row * r + j];
+        h = to_bf16(v);
+        l = to_bf16(v - from_bf16(h));
+    }
+    dst[row * 2 * rp + j] = h;
+    dst[row * 2 * rp + rp + j] = l;
+}
+
+// Deterministic split-K reduce (fixed summation order) with the adapter
+// epilogues.  v(p,q) = sum_z partial[z][p][q] (+ partial[z][p][q+H] when H>0),
+// for q < Qv:
+//   out_f32[p*fsp + q*fsq]  = f32_scale * v
+//   out_bf16[p*bsp + q]     = RN_bf16(bf_scale * v)          (row stride bsp)
+//   out_split[p*2*sp + q], [p*2*sp + sp + q] = hi/lo of v    (row stride 2 sp)
+struct ReduceArgs {
+    const float *partial;
+    int splits;
+    int64_t P, Qp;        // partial layout [splits][P][Qp]
+    int H;                // 0, or the offset of the second half to add
+    int Qv;               // valid output columns
+    float f32_scale; float *out_f32; int64_t fsp, fsq;
+    float bf_scale; uint16_t *out_bf16; int64_t bsp;
+    uint16_t *out_split; int64_t sp;
+};
+
+__global__ void k_reduce(ReduceArgs a) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.P * a.Qv) return;
+    const int64_t p = i / a.Qv;
+    const int q = (int)(i % a.Qv);
+    float v = 0.f;
+    for (int z = 0; z < a.splits; ++z) {
+        const float *base = a.partial + ((int64_t)z * a.P + p) * a.Qp;
+        v += base[q];
+        if (a.H) v += base[q + a.H];
+    }
+    if (a.out_f32) a.out_f32[p * a.fsp + q * a.fsq] = a.f32_scale * v;
+    if (a.out_bf16) a.out_bf16[p * a.bsp + q] = to_bf16(a.bf_scale * v);
+    if (a.out_split) {
+        const uint16_t h = to_bf16(v);
+        a.out_split[p * 2 * a.sp + q] = h;
+        a.out_split[p * 2 * a.sp + a.sp + q] = to_bf16(v - from_bf16(h));
+    }
+}
+
+inline unsigned blocks_for(int64_t n, int t = 256) { return (unsigned)((n + t - 1) / t); }
+
+}  // namespace
+
+int launch_pad_rows(const uint16_t *src, int64_t rows, int r, int rp, int rep, float mul,
+                    uint16_t *dst, cudaStream_t st) {
+    const int64_t n = rows * rp;
+    if (n == 0) return QLORA_OK;
+    k_pad_rows<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, rep, mul, dst);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+int launch_pool_split(const uint16_t *X, int64_t M, int64_t Din, int g, int64_t ld, uint16_t *hi,
+                      uint16_t *lo, cudaStream_t st) {
+    const int64_t n = M * ld;
+    if (n == 0) return QLORA_OK;
+    k_pool_split<<<blocks_for(n), 256, 0, st>>>(X, M, Din, g, ld, hi, lo);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st) {
+    const int64_t n = rows * rp;
+    if (n == 0) return QLORA_OK;
+    k_split_f32<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, dst);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H, int Qv,
+                  float f32_scale, float *out_f32, int64_t fsp, int64_t fsq, float bf_scale,
+                  uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp,
+                  cudaStream_t st) {
+    ReduceArgs a{partial, splits, P, Qp, H, Qv, f32_scale, out_f32, fsp, fsq,
+                 bf_scale, out_bf16, bsp, out_split, sp};
+    const int64_t n = P * Qv;
+    if (n == 0) return QLORA_OK;
+    k_reduce<<<blocks_for(n), 256, 0, st>>>(a);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+// ---------------------------------------------------------------- GEMM launcher
+
+static int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
+template <int BM, int BN>
+static int run_mma_gemm(MmaGemmArgs a, cudaStream_t st) {
+    using S = MmaSmem<BM, BN>;
+    cudaFuncSetAttribute(k_mma_gemm<BM, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)S::BYTES);
+    dim3 grid((unsigned)((a.Q + BN - 1) / BN), (unsigned)((a.P + BM - 1) / BM), (unsigned)a.splits);
+    k_mma_gemm<BM, BN><<<grid, kMmaThreads, S::BYTES, st>>>(a);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+// Number of k-splits that fills the machine for a (P, Q, R) problem, capped
+// so each split keeps >= 8 k-tiles.  The caller sizes `partial` with
+// mma_partial_floats().
+int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN) {
+    const int64_t tiles = ((P + 127) / 128) * ((Q + BN - 1) / BN);
+    const int64_t nkt = (Rtot + kMmaBK - 1) / kMmaBK;
+    int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+    const int64_t cap = nkt / 8 > 1 ? nkt / 8 : 1;
+    if (s > cap) s = cap;
+    if (s > 32) s = 32;
+    return (int)(s < 1 ? 1 : s);
+}
+
+int launch_mma_gemm(MmaGemmArgs a, int bn, cudaStream_t st) {
+    if (a.P <= 0 || a.Q <= 0) return QLORA_OK;
+    if (bn == 128) return run_mma_gemm<128, 128>(a, st);
+    return run_mma_gemm<128, 64>(a, st);
+}
+
+}  // namespace qlora

@@ -1,0 +1,440 @@
+// api.cu -- the extern "C" entry points declared in include/qlora.h:
+// argument validation, workspace layout and kernel dispatch.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "mma_gemm.cuh"
+
+namespace qlora {
+// quantize.cu
+int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
+                        uint32_t *d_status, cudaStream_t st);
+int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *out, cudaStream_t st);
+// gemv.cu
+size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout);
+size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout);
+int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
+                    const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
+                    float *partial, cudaStream_t st);
+int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Codebook &cb,
+                    const float *G, const uint16_t *Al, int r, int pool, float s, uint16_t *dX,
+                    float *partial, cudaStream_t st);
+// adapter.cu
+int launch_pad_rows(const uint16_t *src, int64_t rows, int r, int rp, int rep, float mul,
+                    uint16_t *dst, cudaStream_t st);
+int launch_pool_split(const uint16_t *X, int64_t M, int64_t Din, int g, int64_t ld, uint16_t *hi,
+                      uint16_t *lo, cudaStream_t st);
+int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st);
+int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H, int Qv,
+                  float f32_scale, float *out_f32, int64_t fsp, int64_t fsq, float bf_scale,
+                  uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp, cudaStream_t st);
+int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN);
+int launch_mma_gemm(MmaGemmArgs a, int bn, cudaStream_t st);
+// umma_gemm.cu
+int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t &q,
+                      const Codebook &cb, const uint16_t *sAct, int r, const uint16_t *adapter,
+                      uint16_t *Y, uint32_t *d_status, cudaStream_t st);
+
+namespace {
+
+constexpr int kGemvMaxM = 16;
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_codebook(const float *cb, int *zero_idx) {
+    if (!cb) return QLORA_EINVAL;
+    int zi = -1;
+    for (int j = 0; j < 16; ++j) {
+        if (!std::isfinite(cb[j]) || cb[j] < -1.f || cb[j] > 1.f) return QLORA_EINVAL;
+        if (j > 0 && !(cb[j] > cb[j - 1])) return QLORA_EINVAL;
+        if (cb[j] == 0.f) zi = j;
+    }
+    if (zi < 0) return QLORA_EINVAL;
+    if (zero_idx) *zero_idx = zi;
+    return QLORA_OK;
+}
+
+int check_weight(const nf4_weight_t *q, bool need_rows) {
+    if (!q) return QLORA_EINVAL;
+    if (q->rows < 0 || q->cols < 0) return QLORA_EINVAL;
+    if (need_rows && q->rows < 1) return QLORA_EINVAL;
+    if (q->cols % 64 != 0) return QLORA_EINVAL;
+    if (q->block != 64) return QLORA_EUNSUPPORTED;
+    if (q->double_quant != 0 && q->double_quant != 1) return QLORA_EINVAL;
+    if (q->rows * q->cols == 0) return QLORA_OK;
+    if (!q->packed || !aligned16(q->packed)) return QLORA_EINVAL;
+    if (q->double_quant) {
+        if (q->dq_group != 256) return QLORA_EUNSUPPORTED;
+        if (!q->absmax_code || !q->dq_step) return QLORA_EINVAL;
+    } else {
+        if (!q->absmax) return QLORA_EINVAL;
+    }
+    return QLORA_OK;
+}
+
+bool large_path_uses_mma() {
+    const char *e = std::getenv("QLORA_LARGE_M_PATH");
+    return e && std::strcmp(e, "mma") == 0;
+}
+
+// Bump allocator over the caller's workspace (256-byte aligned pieces).
+struct Bump {
+    uintptr_t base;
+    size_t off = 0;
+    explicit Bump(void *b) : base(reinterpret_cast<uintptr_t>(b)) {}
+    template <class T>
+    T *take(size_t count) {
+        off = (off + 255) & ~size_t(255);
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += count * sizeof(T);
+        return p;
+    }
+};
+
+struct Dims {
+    int64_t M, Din, Dout;
+    int r, rp, rp64, g;
+    int64_t Da, Dap;
+    bool small, mma_large;
+};
+
+Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
+    Dims d;
+    d.M = M;
+    d.Din = q->cols;
+    d.Dout = q->rows;
+    d.r = r;
+    d.rp = (int)round_up(r, 16);
+    d.rp64 = (int)round_up(r, 64);
+    d.g = g;
+    d.Da = d.Din / g;
+    d.Dap = round_up(d.Da, 8);
+    d.small = M <= kGemvMaxM;
+    d.mma_large = !d.small && large_path_uses_mma();
+    return d;
+}
+
+int t_splits(const Dims &d) { return mma_choose_splits(d.M, d.r, d.g > 1 ? 2 * d.Da : d.Din, 64); }
+int g_splits(const Dims &d) { return mma_choose_splits(d.M, d.r, d.Dout, 64); }
+int da_splits(const Dims &d) { return mma_choose_splits(d.Da, 2 * d.rp, (d.g > 1 ? 2 : 1) * d.M, 128); }
+int db_splits(const Dims &d) { return mma_choose_splits(d.Dout, 2 * d.rp, d.M, 128); }
+
+// Workspace pieces.  The same function sizes (base == nullptr) and carves.
+struct FwdWs {
+    uint16_t *Apad, *ph, *pl, *sT, *Wdeq;
+    float *T32, *Tpart, *gemv_part;
+};
+struct BwdWs {
+    uint16_t *Apad, *ph, *pl, *sG, *Gsplit, *Tsplit, *Aext, *Wdeq;
+    float *G32, *Gpart, *T32, *Tpart, *dApart, *dBpart, *gemv_part;
+};
+
+size_t layout_fwd(const Dims &d, bool have_tsave, void *base, FwdWs *w) {
+    Bump b(base);
+    FwdWs x{};
+    x.Apad = b.take<uint16_t>(d.Da * d.rp);
+    if (d.g > 1) {
+        x.ph = b.take<uint16_t>(d.M * d.Dap);
+        x.pl = b.take<uint16_t>(d.M * d.Dap);
+    }
+    if (!have_tsave) x.T32 = b.take<float>(d.M * d.r);
+    x.Tpart = b.take<float>((size_t)t_splits(d) * d.M * d.r);
+    if (d.small) {
+        x.gemv_part = b.take<float>(gemv_fwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
+    } else {
+        x.sT = b.take<uint16_t>(d.M * d.rp64);
+        if (d.mma_large) x.Wdeq = b.take<uint16_t>(d.Dout * d.Din);
+    }
+    if (w) *w = x;
+    return b.off;
+}
+
+size_t layout_bwd(const Dims &d, bool have_tsaved, bool want_dx, bool want_da, bool want_db,
+                  void *base, BwdWs *w) {
+    Bump b(base);
+    BwdWs x{};
+    x.G32 = b.take<float>(d.M * d.r);
+    x.Gpart = b.take<float>((size_t)g_splits(d) * d.M * d.r);
+    if (want_da) x.Gsplit = b.take<uint16_t>(d.M * 2 * d.rp);
+    if (d.g > 1 && (want_da || (want_db && !have_tsaved))) {
+        x.ph = b.take<uint16_t>(d.M * d.Dap);
+        x.pl = b.take<uint16_t>(d.M * d.Dap);
+    }
+    if (want_db) {
+        if (!have_tsaved) {
+            x.Apad = b.take<uint16_t>(d.Da * d.rp);
+            x.T32 = b.take<float>(d.M * d.r);
+            x.Tpart = b.take<float>((size_t)t_splits(d) * d.M * d.r);
+        }
+        x.Tsplit = b.take<uint16_t>(d.M * 2 * d.rp);
+        x.dBpart = b.take<float>((size_t)db_splits(d) * d.Dout * 2 * d.rp);
+    }
+    if (want_da) x.dApart = b.take<float>((size_t)da_splits(d) * d.Da * 2 * d.rp);
+    if (want_dx) {
+        if (d.small) {
+            x.gemv_part = b.take<float>(gemv_bwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
+        } else {
+            x.sG = b.take<uint16_t>(d.M * d.rp64);
+            if (d.mma_large) {
+                x.Aext = b.take<uint16_t>(d.Din * d.rp);
+                x.Wdeq = b.take<uint16_t>(d.Dout * d.Din);
+            } else {
+                x.Aext = b.take<uint16_t>(d.Din * d.rp64);
+            }
+        }
+    }
+    if (w) *w = x;
+    return b.off;
+}
+
+int check_layer_args(int64_t M, const nf4_weight_t *q, const float *cb, int r, float alpha, int g,
+                     int *zero_idx) {
+    if (M < 0 || M > (int64_t)0x7fffffff) return QLORA_EINVAL;
+    int rc = check_weight(q, true);
+    if (rc) return rc;
+    if (q->rows % 8 != 0) return QLORA_EUNSUPPORTED;
+    rc = check_codebook(cb, zero_idx);
+    if (rc) return rc;
+    if (r < 1 || r > QLORA_MAX_RANK) return QLORA_EINVAL;
+    if (!std::isfinite(alpha)) return QLORA_EINVAL;
+    if (g != 1 && g != 64) return QLORA_EINVAL;
+    return QLORA_OK;
+}
+
+Codebook to_cb(const float *c) {
+    Codebook cb;
+    for (int j = 0; j < 16; ++j) cb.c[j] = c[j];
+    return cb;
+}
+
+#define RC(x)                    \
+    do {                         \
+        int _rc = (x);           \
+        if (_rc) return _rc;     \
+    } while (0)
+
+// T = u . A  ->  T32 [M, r] (and s*T as bf16 into sT [M, rp64] if sT)
+int run_adapter_down(const Dims &d, const uint16_t *X, const uint16_t *A, uint16_t *Apad,
+                     const uint16_t *ph, const uint16_t *pl, float *Tpart, float *T32, float s,
+                     uint16_t *sT, cudaStream_t st) {
+    RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st));
+    MmaGemmArgs a{};
+    const MmaOperand Bop{Apad, d.rp, 0};
+    if (d.g == 1) {
+        a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 1}, Bop, d.Din};
+        a.nseg = 1;
+    } else {
+        a.seg[0] = MmaSeg{MmaOperand{ph, d.Dap, 1}, Bop, d.Da};
+        a.seg[1] = MmaSeg{MmaOperand{pl, d.Dap, 1}, Bop, d.Da};
+        a.nseg = 2;
+    }
+    a.P = d.M;
+    a.Q = d.r;
+    a.splits = t_splits(d);
+    a.partial = Tpart;
+    RC(launch_mma_gemm(a, 64, st));
+    if (sT && cudaMemsetAsync(sT, 0, d.M * d.rp64 * sizeof(uint16_t), st) != cudaSuccess)
+        return QLORA_ECUDA;
+    return launch_reduce(Tpart, a.splits, d.M, d.r, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
+                         nullptr, 0, st);
+}
+
+int run_pool(const Dims &d, const uint16_t *X, uint16_t *ph, uint16_t *pl, cudaStream_t st) {
+    return launch_pool_split(X, d.M, d.Din, d.g, d.Dap, ph, pl, st);
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char *qlora_strerror(int code) {
+    switch (code) {
+        case QLORA_OK: return "ok";
+        case QLORA_EINVAL: return "invalid argument";
+        case QLORA_EUNSUPPORTED: return "unsupported configuration";
+        case QLORA_ECUDA: return "CUDA launch failure";
+        case QLORA_EWORKSPACE: return "workspace too small";
+        default: return "unknown error";
+    }
+}
+
+int qlora_version(void) { return 100; }
+
+int qlora_check_codebook(const float codebook[16]) { return check_codebook(codebook, nullptr); }
+
+int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16],
+                 uint32_t *d_status, void *stream) {
+    int zi = 0;
+    RC(check_weight(q, false));
+    RC(check_codebook(codebook, &zi));
+    if (q->rows * q->cols == 0) return QLORA_OK;
+    if (!W || !aligned16(W)) return QLORA_EINVAL;
+    return launch_nf4_quantize(W, *q, to_cb(codebook), zi, d_status, (cudaStream_t)stream);
+}
+
+int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out, void *stream) {
+    RC(check_weight(q, false));
+    RC(check_codebook(codebook, nullptr));
+    if (q->rows * q->cols == 0) return QLORA_OK;
+    if (!W_out || !aligned16(W_out)) return QLORA_EINVAL;
+    return launch_nf4_dequantize(*q, to_cb(codebook), W_out, (cudaStream_t)stream);
+}
+
+size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t pool_group,
+                            int32_t which) {
+    static const float kCb[16] = {-1, -.875f, -.75f, -.625f, -.5f, -.375f, -.25f, 0,
+                                  .125f, .25f, .375f, .5f, .625f, .75f, .875f, 1};
+    if (check_layer_args(M, q, kCb, r, 0.f, pool_group, nullptr)) return 0;
+    if (M == 0) return 0;
+    const Dims d = make_dims(M, q, r, pool_group);
+    if (which == 0) return layout_fwd(d, false, nullptr, nullptr);
+    return layout_bwd(d, false, true, true, true, nullptr, nullptr);
+}
+
+int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const float codebook[16],
+                  const uint16_t *A, const uint16_t *B, int32_t r, float alpha, int32_t pool_group,
+                  uint16_t *Y, float *T_save, void *workspace, size_t ws_bytes, uint32_t *d_status,
+                  void *stream) {
+    RC(check_layer_args(M, q, codebook, r, alpha, pool_group, nullptr));
+    if (M == 0) return QLORA_OK;
+    if (!X || !A || !B || !Y) return QLORA_EINVAL;
+    if (!aligned16(X) || !aligned16(B) || !aligned16(Y)) return QLORA_EINVAL;
+    const Dims d = make_dims(M, q, r, pool_group);
+    const size_t need = layout_fwd(d, T_save != nullptr, nullptr, nullptr);
+    if (need > ws_bytes || (need > 0 && !workspace)) return QLORA_EWORKSPACE;
+    FwdWs w;
+    layout_fwd(d, T_save != nullptr, workspace, &w);
+    cudaStream_t st = (cudaStream_t)stream;
+    const Codebook cb = to_cb(codebook);
+    const float s = alpha / (float)r;
+    float *T32 = T_save ? T_save : w.T32;
+
+    if (d.g > 1) RC(run_pool(d, X, w.ph, w.pl, st));
+    RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT, st));
+    if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, st);
+    if (!d.mma_large) return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
+    // warp-MMA path: dequantize to a bf16 copy, then one two-segment GEMM
+    RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));
+    MmaGemmArgs a{};
+    a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 1}, MmaOperand{w.Wdeq, d.Din, 1}, d.Din};
+    a.seg[1] = MmaSeg{MmaOperand{w.sT, d.rp64, 1}, MmaOperand{B, d.Dout, 0}, (int64_t)r};
+    a.nseg = 2;
+    a.P = M;
+    a.Q = d.Dout;
+    a.out_scale = 1.f;
+    a.out_bf16 = Y;
+    a.bf_sp = d.Dout;
+    a.bf_sq = 1;
+    a.splits = 1;
+    return launch_mma_gemm(a, 128, st);
+}
+
+int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_weight_t *q,
+                   const float codebook[16], const uint16_t *A, const uint16_t *B, int32_t r,
+                   float alpha, int32_t pool_group, const float *T_saved, uint16_t *dX, float *dA,
+                   float *dB, void *workspace, size_t ws_bytes, uint32_t *d_status, void *stream) {
+    RC(check_layer_args(M, q, codebook, r, alpha, pool_group, nullptr));
+    if (M == 0) return QLORA_OK;
+    if (!dY || !A || !B) return QLORA_EINVAL;
+    const bool want_dx = dX != nullptr, want_da = dA != nullptr, want_db = dB != nullptr;
+    if ((want_da || (want_db && !T_saved)) && !X) return QLORA_EINVAL;
+    if (!aligned16(dY) || !aligned16(B) || (X && !aligned16(X)) || (dX && !aligned16(dX)))
+        return QLORA_EINVAL;
+    const Dims d = make_dims(M, q, r, pool_group);
+    const size_t need = layout_bwd(d, T_saved != nullptr, want_dx, want_da, want_db, nullptr, nullptr);
+    if (need > ws_bytes || (need > 0 && !workspace)) return QLORA_EWORKSPACE;
+    BwdWs w;
+    layout_bwd(d, T_saved != nullptr, want_dx, want_da, want_db, workspace, &w);
+    cudaStream_t st = (cudaStream_t)stream;
+    const Codebook cb = to_cb(codebook);
+    const float s = alpha / (float)r;
+
+    // G = dY . B^T  (fp32), s*G (bf16, large M), hi/lo split (for dA)
+    {
+        MmaGemmArgs a{};
+        a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 1}, MmaOperand{B, d.Dout, 1}, d.Dout};
+        a.nseg = 1;
+        a.P = M;
+        a.Q = r;
+        a.splits = g_splits(d);
+        a.partial = w.Gpart;
+        RC(launch_mma_gemm(a, 64, st));
+        uint16_t *sG = (want_dx && !d.small) ? w.sG : nullptr;
+        if (sG && cudaMemsetAsync(sG, 0, M * d.rp64 * 2, st) != cudaSuccess) return QLORA_ECUDA;
+        if (w.Gsplit && cudaMemsetAsync(w.Gsplit, 0, M * 2 * d.rp * 2, st) != cudaSuccess)
+            return QLORA_ECUDA;
+        RC(launch_reduce(w.Gpart, a.splits, M, r, 0, r, 1.f, w.G32, r, 1, s, sG, d.rp64, w.Gsplit,
+                         d.rp, st));
+    }
+    if (d.g > 1 && w.ph) RC(run_pool(d, X, w.ph, w.pl, st));
+
+    if (want_dx) {
+        if (d.small) {
+            RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st));
+        } else if (!d.mma_large) {
+            RC(launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st));
+            RC(launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, w.Aext, dX, d_status, st));
+        } else {
+            RC(launch_pad_rows(A, d.Din, r, d.rp, d.g, 1.f / d.g, w.Aext, st));
+            RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));
+            MmaGemmArgs a{};
+            a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 1}, MmaOperand{w.Wdeq, d.Din, 0}, d.Dout};
+            a.seg[1] = MmaSeg{MmaOperand{w.sG, d.rp64, 1}, MmaOperand{w.Aext, d.rp, 1}, (int64_t)r};
+            a.nseg = 2;
+            a.P = M;
+            a.Q = d.Din;
+            a.out_scale = 1.f;
+            a.out_bf16 = dX;
+            a.bf_sp = d.Din;
+            a.bf_sq = 1;
+            a.splits = 1;
+            RC(launch_mma_gemm(a, 128, st));
+        }
+    }
+    if (want_da) {
+        MmaGemmArgs a{};
+        const MmaOperand Gop{w.Gsplit, 2 * d.rp, 0};
+        if (d.g == 1) {
+            a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 0}, Gop, M};
+            a.nseg = 1;
+        } else {
+            a.seg[0] = MmaSeg{MmaOperand{w.ph, d.Dap, 0}, Gop, M};
+            a.seg[1] = MmaSeg{MmaOperand{w.pl, d.Dap, 0}, Gop, M};
+            a.nseg = 2;
+        }
+        a.P = d.Da;
+        a.Q = 2 * d.rp;
+        a.splits = da_splits(d);
+        a.partial = w.dApart;
+        RC(launch_mma_gemm(a, 128, st));
+        RC(launch_reduce(w.dApart, a.splits, d.Da, 2 * d.rp, d.rp, r, s, dA, r, 1, 0.f, nullptr, 0,
+                         nullptr, 0, st));
+    }
+    if (want_db) {
+        const float *T32 = T_saved;
+        if (!T32) {
+            RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, w.T32, s, nullptr, st));
+            T32 = w.T32;
+        }
+        RC(launch_split_f32(T32, M, r, d.rp, w.Tsplit, st));
+        MmaGemmArgs a{};
+        a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 0}, MmaOperand{w.Tsplit, 2 * d.rp, 0}, M};
+        a.nseg = 1;
+        a.P = d.Dout;
+        a.Q = 2 * d.rp;
+        a.splits = db_splits(d);
+        a.partial = w.dBpart;
+        RC(launch_mma_gemm(a, 128, st));
+        RC(launch_reduce(w.dBpart, a.splits, d.Dout, 2 * d.rp, d.rp, r, s, dB, 1, d.Dout, 0.f,
+                         nullptr, 0, nullptr, 0, st));
+    }
+    return QLORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// common.cuh -- device helpers shared by the QLoRA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qlora.h"
+
+namespace qlora {
+
+// The 16-level codebook, passed to kernels by value.
+struct Codebook {
+    float c[16];
+};
+
+// Decoded first-level scale of block b: the fp32 absmax, or with double
+// quantization RN32(code * step) (one rounding of an exact product).
+struct ScaleSrc {
+    const float *absmax;      // when !dq
+    const uint8_t *code;      // when dq
+    const float *step;        // when dq
+    int dq;
+};
+
+__device__ __forceinline__ float load_scale(const ScaleSrc &s, int64_t b) {
+    if (!s.dq) return __ldg(s.absmax + b);
+    float f = __ldg(s.step + (b >> 8));
+    return __fmul_rn((float)__ldg(s.code + b), f);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// ---------------------------------------------------------------------------
+// NF4 decode through a per-block product table.
+//
+// For one block with decoded scale a_hat, entry j of the table is the bf16
+// weight RN_bf16(RN32(a_hat * c_j)).  The 16 entries are held as two byte
+// planes (low and high byte of each bf16) of four registers each, so a
+// lookup of four 4-bit indices is two byte-permutes per plane plus a select
+// on the index's top bit: no shared memory, no local memory.
+// ---------------------------------------------------------------------------
+struct ProdTable {
+    uint32_t lo[4];   // lo[i] byte k = low byte of entry 4i+k
+    uint32_t hi[4];   // hi[i] byte k = high byte of entry 4i+k
+};
+
+__device__ __forceinline__ void build_table(float ah, const Codebook &cb, ProdTable &t) {
+    uint32_t p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        p[i] = bf16x2_bits(__fmul_rn(ah, cb.c[2 * i]), __fmul_rn(ah, cb.c[2 * i + 1]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        t.lo[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x6420);
+        t.hi[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x7531);
+    }
+}
+
+// Decode the 8 indices of one packed 32-bit word (bytes b0..b3 in memory
+// order; byte i holds element 2i in its high nibble and 2i+1 in its low
+// nibble) into four bf16x2 registers: out[k] = (element 2k, element 2k+1).
+__device__ __forceinline__ void decode8(uint32_t w, const ProdTable &t, uint32_t out[4]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t v = (h == 0) ? w : (w >> 16);
+        // selector nibbles, output byte n <- nibble n of v: [e1, e0, e3, e2]
+        const uint32_t sel = v & 0x7777u;
+        const uint32_t m = __byte_perm(0u, 0xffffffffu, (v >> 1) & 0x4444u);
+        const uint32_t l0 = __byte_perm(t.lo[0], t.lo[1], sel);
+        const uint32_t l1 = __byte_perm(t.lo[2], t.lo[3], sel);
+        const uint32_t h0 = __byte_perm(t.hi[0], t.hi[1], sel);
+        const uint32_t h1 = __byte_perm(t.hi[2], t.hi[3], sel);
+        const uint32_t L = (l0 & ~m) | (l1 & m);
+        const uint32_t H = (h0 & ~m) | (h1 & m);
+        out[2 * h + 0] = __byte_perm(L, H, 0x4051);   // (e0, e1)
+        out[2 * h + 1] = __byte_perm(L, H, 0x6273);   // (e2, e3)
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Legacy warp-level tensor-core helpers (m16n8k16, bf16 in, fp32 accumulate).
+// Used where the tensor unit is not the bottleneck (HBM-bound GEMV, skinny
+// adapter products).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t r[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred) {
+    const int n = pred ? 16 : 0;   // src-size 0 zero-fills the 16 bytes
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+                 "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+}  // namespace qlora
+
+namespace qlora {
+// Launch accounting and optional per-kernel event timing (profile.cu).
+enum ProfKind { kProfUmma = 0, kProfGemv = 1, kProfQuant = 2, kProfAdapter = 3, kProfKinds = 4 };
+void count_launch();
+void prof_begin(int kind, cudaStream_t st);
+void prof_end(int kind, cudaStream_t st);
+}  // namespace qlora
+
+// Host-side launch check used after every kernel launch.
+#define QLORA_LAUNCH_CHECK()                                              \
+    do {                                                                  \
+        ::qlora::count_launch();                                          \
+        if (cudaPeekAtLastError() != cudaSuccess) return QLORA_ECUDA;     \
+    } while (0)

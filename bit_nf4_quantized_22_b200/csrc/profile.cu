@@ -1,0 +1,79 @@
+// profile.cu -- launch counting and opt-in CUDA-event timing of the
+// library's main kernels, for benchmarks.  When enabled, an event pair is
+// recorded on the launch stream around each timed kernel; reading the totals
+// synchronizes on those events.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace qlora {
+namespace {
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_on{0};
+std::mutex g_mu;
+struct Pairs {
+    std::vector<cudaEvent_t> start, stop;
+    size_t used = 0;
+};
+Pairs g_pairs[kProfKinds];
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void prof_begin(int kind, cudaStream_t st) {
+    if (!g_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Pairs &p = g_pairs[kind];
+    if (p.used == p.start.size()) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return;
+        if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+        p.start.push_back(a);
+        p.stop.push_back(b);
+    }
+    cudaEventRecord(p.start[p.used], st);
+}
+
+void prof_end(int kind, cudaStream_t st) {
+    if (!g_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Pairs &p = g_pairs[kind];
+    if (p.used < p.start.size()) {
+        cudaEventRecord(p.stop[p.used], st);
+        ++p.used;
+    }
+}
+
+}  // namespace qlora
+
+extern "C" {
+
+void qlora_profile_enable(int on) { qlora::g_on.store(on ? 1 : 0); }
+
+void qlora_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(qlora::g_mu);
+    for (auto &p : qlora::g_pairs) p.used = 0;
+    qlora::g_launches.store(0);
+}
+
+int64_t qlora_launch_count(void) { return qlora::g_launches.load(); }
+
+int qlora_profile_read(int32_t kind, int64_t *launches, double *total_ms) {
+    if (kind < 0 || kind >= qlora::kProfKinds || !launches || !total_ms) return QLORA_EINVAL;
+    std::lock_guard<std::mutex> lk(qlora::g_mu);
+    auto &p = qlora::g_pairs[kind];
+    double t = 0.0;
+    for (size_t i = 0; i < p.used; ++i) {
+        if (cudaEventSynchronize(p.stop[i]) != cudaSuccess) return QLORA_ECUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, p.start[i], p.stop[i]) != cudaSuccess) return QLORA_ECUDA;
+        t += ms;
+    }
+    *launches = (int64_t)p.used;
+    *total_ms = t;
+    return QLORA_OK;
+}
+
+}  // extern "C"

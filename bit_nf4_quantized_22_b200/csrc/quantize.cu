@@ -1,0 +1,191 @@
+// quantize.cu -- blockwise NF4 quantization (+ double quantization) and
+// dequantization kernels.
+//
+// Rule (bitsandbytes article (CSDN) section 5.2): per block of 64 weights
+// a = max|w|; each weight takes the codebook index argmin_j |w/a - c_j|
+// (exact arithmetic, first index on ties); two indices per byte, element 2i
+// in the high nibble.  Double quantization (section 7.2): per 256 blocks,
+// step f = RN32(max a / 255), code = round-half-even(a / f) in [0, 255].
+#include "common.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kQuantThreads = 256;   // one thread per block, one CTA per DQ group
+
+__device__ __forceinline__ float next_up(float x) {
+    const uint32_t u = __float_as_uint(x);
+    if ((u & 0x7fffffffu) == 0u) return __uint_as_float(1u);   // +-0 -> smallest subnormal
+    return __uint_as_float(x > 0.f ? u + 1u : u - 1u);
+}
+
+// tau such that, for every fp32 w,  w >= tau  <=>  w > (c_lo + c_hi) * a / 2
+// exactly.  c*a is an exact fp64 product of two fp32 values; TwoSum gives the
+// midpoint sum as S + err exactly.  tau = smallest fp32 >= S/2, moved up one
+// ulp when S/2 is itself an fp32 value and err >= 0 (then the exact midpoint
+// is >= tau and w must exceed it).  In every other case the fp64 residue is
+// far below the fp32 spacing, so no fp32 value lies between the midpoint and
+// tau.
+__device__ __forceinline__ float exact_threshold(float c_lo, float c_hi, float a) {
+    const double p1 = __dmul_rn((double)c_lo, (double)a);
+    const double p2 = __dmul_rn((double)c_hi, (double)a);
+    const double s = __dadd_rn(p1, p2);
+    const double bb = __dsub_rn(s, p1);
+    const double err = __dadd_rn(__dsub_rn(p1, __dsub_rn(s, bb)), __dsub_rn(p2, bb));
+    const double half = s * 0.5;
+    float tau = __double2float_ru(half);
+    if ((double)tau == half && err >= 0.0) tau = next_up(tau);
+    return tau;
+}
+
+// Branch-free binary search over 15 sorted thresholds: the number of j with
+// w >= t[j], i.e. the index of the nearest level.
+__device__ __forceinline__ uint32_t level_index(float w, const float t[15]) {
+    const bool b3 = w >= t[7];
+    const float t2 = b3 ? t[11] : t[3];
+    const bool b2 = w >= t2;
+    const float t1 = b3 ? (b2 ? t[13] : t[9]) : (b2 ? t[5] : t[1]);
+    const bool b1 = w >= t1;
+    const float t0 = b3 ? (b2 ? (b1 ? t[14] : t[12]) : (b1 ? t[10] : t[8]))
+                        : (b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]));
+    const bool b0 = w >= t0;
+    return (uint32_t(b3) << 3) | (uint32_t(b2) << 2) | (uint32_t(b1) << 1) | uint32_t(b0);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+k_nf4_quantize(const float *__restrict__ W, int64_t nb, Codebook cb, int zero_idx, int dq,
+               uint8_t *__restrict__ packed, float *__restrict__ absmax,
+               uint8_t *__restrict__ codes, float *__restrict__ steps,
+               uint32_t *__restrict__ status) {
+    const int64_t b = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x;
+    const bool valid = b < nb;
+    float w[64];
+    if (valid) {
+        const float4 *src = reinterpret_cast<const float4 *>(W + b * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 v = __ldg(src + i);
+            w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) w[i] = 0.f;
+    }
+    float a = 0.f;
+    uint32_t bad = 0;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        a = fmaxf(a, fabsf(w[i]));
+        bad |= ((__float_as_uint(w[i]) & 0x7f800000u) == 0x7f800000u);
+    }
+    if (bad && status) atomicOr(status, QLORA_STATUS_NONFINITE);
+
+    if (valid) {
+        uint32_t out[8];
+        if (a == 0.f) {
+            const uint32_t z = (uint32_t)zero_idx * 0x11111111u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) out[i] = z;
+        } else {
+            float t[15];
+#pragma unroll
+            for (int j = 0; j < 15; ++j) t[j] = exact_threshold(cb.c[j], cb.c[j + 1], a);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t q0 = level_index(w[8 * i + 2 * k], t);
+                    const uint32_t q1 = level_index(w[8 * i + 2 * k + 1], t);
+                    word |= ((q0 << 4) | q1) << (8 * k);
+                }
+                out[i] = word;
+            }
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(packed + b * 32);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        if (!dq) absmax[b] = a;
+    }
+
+    if (dq) {
+        // group max over this CTA's 256 blocks (one double-quant group)
+        __shared__ float warp_max[kQuantThreads / 32];
+        float m = valid ? a : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+        __syncthreads();
+        float gm = warp_max[0];
+#pragma unroll
+        for (int i = 1; i < kQuantThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
+        const float f = __fdiv_rn(gm, 255.f);
+        if (threadIdx.x == 0) steps[blockIdx.x] = f;
+        if (valid) {
+            int code = 0;
+            if (f > 0.f) {
+                // a/f < 256 is a ratio of fp32 values: rint of the fp64
+                // quotient is round-half-even of the exact ratio.
+                double qd = rint(__ddiv_rn((double)a, (double)f));
+                qd = fmin(fmax(qd, 0.0), 255.0);
+                code = (int)qd;
+            }
+            codes[b] = (uint8_t)code;
+        }
+    }
+}
+
+// Dequantize: 4 threads per block; thread i of the 4 owns packed bytes
+// [4i, 4i+4) and [16+4i, 16+4i+4) of its block, i.e. output elements
+// [8i, 8i+8) and [32+8i, 32+8i+8), so each group of 4 threads reads 16
+// contiguous bytes and writes 64 contiguous bytes per instruction.
+__global__ void __launch_bounds__(256)
+k_nf4_dequantize(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t nb, Codebook cb,
+                 uint16_t *__restrict__ out) {
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t b = gt >> 2;
+    const int part = (int)(gt & 3);
+    if (b >= nb) return;
+    const float ah = load_scale(sc, b);
+    ProdTable tab;
+    build_table(ah, cb, tab);
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(packed + b * 32);
+    const uint32_t w0 = __ldg(src + part);
+    const uint32_t w1 = __ldg(src + 4 + part);
+    uint32_t o0[4], o1[4];
+    decode8(w0, tab, o0);
+    decode8(w1, tab, o1);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + b * 64);
+    dst[part] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    dst[4 + part] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+}
+
+}  // namespace
+
+int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
+                        uint32_t *d_status, cudaStream_t st) {
+    const int64_t nb = q.rows * q.cols / 64;
+    if (nb == 0) return QLORA_OK;
+    const int64_t grid = (nb + kQuantThreads - 1) / kQuantThreads;
+    prof_begin(kProfQuant, st);
+    k_nf4_quantize<<<(unsigned)grid, kQuantThreads, 0, st>>>(
+        W, nb, cb, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
+        d_status);
+    prof_end(kProfQuant, st);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *out,
+                          cudaStream_t st) {
+    const int64_t nb = q.rows * q.cols / 64;
+    if (nb == 0) return QLORA_OK;
+    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    const int64_t threads = nb * 4;
+    const int64_t grid = (threads + 255) / 256;
+    k_nf4_dequantize<<<(unsigned)grid, 256, 0, st>>>(q.packed, sc, nb, cb, out);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+}  // namespace qlora

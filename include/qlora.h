@@ -1,0 +1,167 @@
+/*
+ * qlora.h -- C ABI of the QLoRA linear-layer library (libqlora.so, sm_100a).
+ *
+ * The layer, in row-vector convention with x:[M,Din], A:[Din,r], B:[r,Dout]:
+ *
+ *     y  = x . dequant(W4) + s (x . A) . B,          s = alpha / r
+ *     dX = dY . dequant(W4)^T + s (dY . B^T) . A^T   (no gradient for W4)
+ *     dA = s x^T (dY . B^T),   dB = s (x . A)^T dY
+ *
+ * Sources: "从 LoRA 到 QLoRA、QA-LoRA：低秩更新如何进入量化模型" (ludovicoyin.github.io),
+ * section 2 (y = x dequant(W4) + xAB; W_eff = dequant(W4) + (alpha/r) AB) and
+ * sections 3-5 (pooled adapter input); "大模型量化从0到1（十）：bitsandbytes"
+ * (aicoding.csdn.net), section 5.2 (block absmax, nearest codebook level,
+ * two indices per byte), 7.2 (double quantization: 8-bit first-level scales,
+ * one fp32 constant per 256), 8.6 (dequantize fused into the matmul),
+ * 12.2/12.4 (s = lora_alpha / r; the gradient passes through the frozen
+ * base, which receives none).
+ *
+ * Conventions shared by every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller, except the
+ *     16-entry codebook, which is a HOST array read during the call.  The
+ *     library allocates nothing: scratch memory is the caller's `workspace`
+ *     buffer, sized by qlora_workspace_size().
+ *   - bf16 arrays are passed as uint16_t bit patterns; every 2-D array is
+ *     row-major and densely packed.
+ *   - The frozen weight is stored transposed, Wt:[Dout, Din] (the
+ *     nn.Linear layout).  Flattened row-major it is cut into blocks of 64
+ *     consecutive weights, each inside one row; Din must be a multiple of 64.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; no call synchronizes the host.
+ *   - Return value: QLORA_OK, or an error code.  Arguments are validated on
+ *     the host before anything is enqueued; a failed validation enqueues
+ *     nothing.  QLORA_ECUDA reports a launch failure (the CUDA error is left
+ *     for the caller to query).
+ *   - `d_status` (optional, may be NULL): a device uint32_t into which
+ *     kernels OR the QLORA_STATUS_* bits they detect.  The library never
+ *     clears it.  Device-side conditions never trap or abort the context.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QLORA_OK 0
+#define QLORA_EINVAL 1          /* bad pointer, size, rank, alpha or codebook   */
+#define QLORA_EUNSUPPORTED 2    /* valid request outside what this build does  */
+#define QLORA_ECUDA 3           /* a kernel launch failed                       */
+#define QLORA_EWORKSPACE 4      /* workspace missing or smaller than required  */
+
+#define QLORA_STATUS_NONFINITE 1u /* nf4_quantize met a NaN or Inf weight      */
+#define QLORA_STATUS_TIMEOUT 2u   /* a pipeline wait in a kernel gave up       */
+
+#define QLORA_BLOCK 64
+#define QLORA_DQ_GROUP 256
+#define QLORA_MAX_RANK 256
+
+/* One quantized weight Wt:[rows = Dout, cols = Din]; nb = rows*cols/64.
+ *   packed      [rows*cols/2] uint8   two 4-bit codebook indices per byte;
+ *                                     element 2i in the HIGH nibble of byte i
+ *   absmax      [nb] fp32             block absmax (double_quant == 0)
+ *   absmax_code [nb] uint8            8-bit scale codes (double_quant == 1)
+ *   dq_step     [ceil(nb/256)] fp32   one second-level step per 256 blocks
+ * With double quantization the decoded scale of block b is
+ * RN32(absmax_code[b] * dq_step[b/256]); the codes are round-half-even of
+ * absmax/step with step = RN32(group max / 255). */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    int32_t block;          /* must be 64 */
+    int32_t double_quant;   /* 0 or 1 */
+    int32_t dq_group;       /* must be 256 when double_quant == 1 */
+    int32_t reserved;
+    uint8_t *packed;
+    float *absmax;
+    uint8_t *absmax_code;
+    float *dq_step;
+} nf4_weight_t;
+
+/* Human-readable name of a return code (static storage). */
+const char *qlora_strerror(int code);
+
+/* Library ABI version (major*100 + minor). */
+int qlora_version(void);
+
+/* Host-side check of a codebook (no device work): 16 finite fp32 values,
+ * strictly increasing, inside [-1, 1], one of them exactly 0.
+ * Returns QLORA_OK or QLORA_EINVAL. */
+int qlora_check_codebook(const float codebook[16]);
+
+/* nf4_quantize -- blockwise 4-bit quantization of W (bitsandbytes article
+ * (CSDN) section 5.2, with section 7.2 double quantization).
+ *   W          device fp32 [q->rows, q->cols], the frozen weight Wt.
+ *   q          host struct naming the output buffers (device); the fields
+ *              selected by q->double_quant are written.
+ *   codebook   host fp32[16] (see qlora_check_codebook).
+ * Per block: a = max|w|; index = argmin_j |w - c_j a| in exact arithmetic,
+ * ties to the lower index; an all-zero block maps to the exact-zero level.
+ * A NaN/Inf weight sets QLORA_STATUS_NONFINITE; that block's outputs are
+ * unspecified.  Reads 4 bytes and writes ~0.52 bytes per weight. */
+int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16],
+                 uint32_t *d_status, void *stream);
+
+/* nf4_dequantize -- W_out[rows, cols] (bf16) = RN_bf16(RN32(a_hat * c_q))
+ * (section 5.2, w_hat = a c_q, in the bf16 compute dtype of section 8.3). */
+int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out,
+                   void *stream);
+
+/* Scratch bytes qlora_forward (which = 0) or qlora_backward (which = 1)
+ * needs for this problem.  Returns 0 when the arguments are invalid. */
+size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t pool_group,
+                            int32_t which);
+
+/* qlora_forward -- y = x . dequant(W4) + (alpha/r) T . B with
+ * T = u . A, u = x (pool_group == 1) or the mean of each run of 64 input
+ * features (pool_group == 64, the pooled adapter of QA-LoRA sections 3-4).
+ *   X       device bf16 [M, Din]
+ *   A       device bf16 [Din/pool_group, r];  B  device bf16 [r, Dout]
+ *   r       1..256;  alpha finite;  pool_group 1 or 64
+ *   Y       device bf16 [M, Dout] (output)
+ *   T_save  device fp32 [M, r] receiving T, or NULL
+ *   workspace/ws_bytes  caller scratch of at least qlora_workspace_size(.., 0)
+ * Accumulation is fp32; y is rounded once to bf16. */
+int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const float codebook[16],
+                  const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                  int32_t pool_group, uint16_t *Y, float *T_save, void *workspace,
+                  size_t ws_bytes, uint32_t *d_status, void *stream);
+
+/* qlora_backward -- gradients of the layer for the upstream gradient dY:
+ *   G  = dY . B^T                               (fp32 [M, r], internal)
+ *   dX = dY . dequant(W4)^T + (s/g) G . A^T     (bf16 [M, Din]; with pooling
+ *                                                each input feature of a
+ *                                                group receives 1/g of it)
+ *   dA = s u^T G                                (fp32 [Din/g, r])
+ *   dB = s T^T dY                               (fp32 [r, Dout])
+ * T_saved is the forward's T (fp32 [M, r]) or NULL to recompute it.  Any of
+ * dX, dA, dB may be NULL to skip it.  No gradient is produced for W4. */
+int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_weight_t *q,
+                   const float codebook[16], const uint16_t *A, const uint16_t *B, int32_t r,
+                   float alpha, int32_t pool_group, const float *T_saved, uint16_t *dX,
+                   float *dA, float *dB, void *workspace, size_t ws_bytes,
+                   uint32_t *d_status, void *stream);
+
+/* ---- Benchmark support (not part of the layer's computation) ----------
+ * Kernel launches made by the library since the last qlora_profile_reset(). */
+int64_t qlora_launch_count(void);
+
+/* When enabled, each launch of the library's main kernels is bracketed by a
+ * CUDA event pair recorded on its launch stream.  Kinds: 0 tensor-core GEMM
+ * (tcgen05), 1 small-M GEMV kernels, 2 quantize kernel. */
+void qlora_profile_enable(int on);
+
+/* Forget recorded events and zero the launch count (host only). */
+void qlora_profile_reset(void);
+
+/* Number of timed launches of `kind` since the reset and their summed
+ * duration in milliseconds; waits for the recorded events to complete. */
+int qlora_profile_read(int32_t kind, int64_t *launches, double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H */

@@ -204,6 +204,7 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, const float cb[16],
     const int zero_idx = zero_level_index(cb);
     int status = 0;
     float *a_all = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+#pragma omp parallel for schedule(static) reduction(| : status)
     for (int64_t b = 0; b < nb; ++b) {
         const float *wb = W + b * 64;
         double a = 0.0;
@@ -269,6 +270,7 @@ void orc_dequantize(int64_t rows, int64_t cols, const float cb[16], int dq,
                     int dq_group, const uint8_t *packed, const float *absmax,
                     const uint8_t *codes, const float *steps, uint16_t *out) {
     const int64_t n = rows * cols;
+#pragma omp parallel for schedule(static)
     for (int64_t e = 0; e < n; ++e) {
         int64_t b = e / 64;
         uint8_t byte = packed[e / 2];
@@ -317,7 +319,7 @@ void orc_forward(const uint16_t *X, int64_t M, int64_t Din, int64_t Dout,
     const double s = alpha / (double)r;
     double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
     orc_adapter_down(X, M, Din, A, r, g, T);
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < Dout; ++n) {
             double base = 0.0;
@@ -353,16 +355,27 @@ void orc_backward_dx(const uint16_t *dY, int64_t M, int64_t Din, int64_t Dout,
     const double s = alpha / (double)r;
     double *G = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
     orc_grad_G(dY, M, Dout, B, r, G);
-#pragma omp parallel for schedule(static)
+    /* Each output dX[m,k] sums n = 0..Dout-1 in ascending order; the loops
+     * run n outside k only so that Wt is read row by row. */
+    const int64_t KC = 256;
+    const int64_t nkc = (Din + KC - 1) / KC;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m)
-        for (int64_t k = 0; k < Din; ++k) {
-            double base = 0.0;
-            for (int64_t n = 0; n < Dout; ++n)
-                base += bf16_to_double(dY[m * Dout + n]) * bf16_to_double(Wt[n * Din + k]);
-            double ad = 0.0;
-            for (int j = 0; j < r; ++j)
-                ad += G[m * r + j] * bf16_to_double(A[(k / g) * r + j]);
-            dX[m * Din + k] = base + s * ad / (double)g;
+        for (int64_t c = 0; c < nkc; ++c) {
+            double acc[256];
+            const int64_t k0 = c * KC, k1 = k0 + KC < Din ? k0 + KC : Din;
+            for (int64_t k = k0; k < k1; ++k) acc[k - k0] = 0.0;
+            for (int64_t n = 0; n < Dout; ++n) {
+                const double dy = bf16_to_double(dY[m * Dout + n]);
+                for (int64_t k = k0; k < k1; ++k)
+                    acc[k - k0] += dy * bf16_to_double(Wt[n * Din + k]);
+            }
+            for (int64_t k = k0; k < k1; ++k) {
+                double ad = 0.0;
+                for (int j = 0; j < r; ++j)
+                    ad += G[m * r + j] * bf16_to_double(A[(k / g) * r + j]);
+                dX[m * Din + k] = acc[k - k0] + s * ad / (double)g;
+            }
         }
     free(G);
 }
@@ -380,22 +393,39 @@ void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
     double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
     orc_grad_G(dY, M, Dout, B, r, G);
     orc_adapter_down(X, M, Din, A, r, g, T);
+    /* Each output sums m = 0..M-1 in ascending order; the loops run m
+     * outside the output column so that x, dY are read row by row. */
     if (dA) {
-#pragma omp parallel for schedule(static)
-        for (int64_t k = 0; k < Da; ++k)
-            for (int j = 0; j < r; ++j) {
-                double acc = 0.0;
-                for (int64_t m = 0; m < M; ++m) acc += adapter_in(X, Din, m, k, g) * G[m * r + j];
-                dA[k * r + j] = s * acc;
-            }
+        const int64_t KC = 64;
+        const int64_t nkc = (Da + KC - 1) / KC;
+#pragma omp parallel for schedule(dynamic)
+        for (int64_t c = 0; c < nkc; ++c) {
+            const int64_t k0 = c * KC, k1 = k0 + KC < Da ? k0 + KC : Da;
+            for (int64_t k = k0; k < k1; ++k)
+                for (int j = 0; j < r; ++j) dA[k * r + j] = 0.0;
+            for (int64_t m = 0; m < M; ++m)
+                for (int64_t k = k0; k < k1; ++k) {
+                    const double u = adapter_in(X, Din, m, k, g);
+                    for (int j = 0; j < r; ++j) dA[k * r + j] += u * G[m * r + j];
+                }
+            for (int64_t k = k0; k < k1; ++k)
+                for (int j = 0; j < r; ++j) dA[k * r + j] *= s;
+        }
     }
     if (dB) {
-#pragma omp parallel for schedule(static)
-        for (int64_t n = 0; n < Dout; ++n)
-            for (int j = 0; j < r; ++j) {
-                double acc = 0.0;
-                for (int64_t m = 0; m < M; ++m) acc += T[m * r + j] * bf16_to_double(dY[m * Dout + n]);
-                dB[(int64_t)j * Dout + n] = s * acc;
+        const int64_t NC = 1024;
+        const int64_t nnc = (Dout + NC - 1) / NC;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+        for (int j = 0; j < r; ++j)
+            for (int64_t c = 0; c < nnc; ++c) {
+                const int64_t n0 = c * NC, n1 = n0 + NC < Dout ? n0 + NC : Dout;
+                double *row = dB + (int64_t)j * Dout;
+                for (int64_t n = n0; n < n1; ++n) row[n] = 0.0;
+                for (int64_t m = 0; m < M; ++m) {
+                    const double t = T[m * r + j];
+                    for (int64_t n = n0; n < n1; ++n) row[n] += t * bf16_to_double(dY[m * Dout + n]);
+                }
+                for (int64_t n = n0; n < n1; ++n) row[n] *= s;
             }
     }
     free(G);

@@ -1,0 +1,136 @@
+"""The C-ABI library: it loads, exports every symbol include/qlora.h declares,
+and rejects invalid arguments on the host (no GPU needed: validation runs
+before anything is enqueued)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import ROOT
+
+import bit_nf4_quantized_22_b200 as q
+from bit_nf4_quantized_22_b200 import _lib
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_nf4_quantized_22_b200 import build
+    build.build()
+    return q.load()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert set(names) == set(_lib.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_strerror(lib):
+    assert lib.qlora_version() == 100
+    assert lib.qlora_strerror(0) == b"ok"
+    assert lib.qlora_strerror(4) == b"workspace too small"
+
+
+def _cb(vals):
+    return (ctypes.c_float * 16)(*vals)
+
+
+def test_codebook_validation(lib):
+    good = q.nf4_codebook().tolist()
+    assert lib.qlora_check_codebook(_cb(good)) == 0
+    bad_order = list(good); bad_order[3], bad_order[4] = bad_order[4], bad_order[3]
+    no_zero = [v if v != 0 else 1e-3 for v in good]
+    out_of_range = list(good); out_of_range[15] = 1.5
+    nan = list(good); nan[2] = float("nan")
+    for b in (bad_order, no_zero, out_of_range, nan):
+        assert lib.qlora_check_codebook(_cb(b)) == _lib.QLORA_EINVAL
+    assert lib.qlora_check_codebook(None) == _lib.QLORA_EINVAL
+
+
+def _wc(rows=64, cols=128, dq=1, block=64, group=256, ptrs=True):
+    fake = 1 << 20 if ptrs else 0   # never dereferenced: validation fails first or no launch
+    return _lib.NF4WeightC(rows, cols, block, dq, group, 0, fake, fake, fake, fake)
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    cb = _cb(q.nf4_codebook().tolist())
+    W = ctypes.c_void_p(1 << 20)
+    E = _lib
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(cols=100)), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(block=32)), cb, None, None) == E.QLORA_EUNSUPPORTED
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(group=128)), cb, None, None) == E.QLORA_EUNSUPPORTED
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=2)), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(ptrs=False)), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(None, ctypes.byref(_wc()), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(ctypes.c_void_p((1 << 20) + 4), ctypes.byref(_wc()), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(W, None, cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_quantize(W, ctypes.byref(_wc()), None, None, None) == E.QLORA_EINVAL
+    # an empty weight is a valid no-op
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(rows=0)), cb, None, None) == E.QLORA_OK
+
+
+def test_layer_rejects_bad_arguments(lib):
+    cb = _cb(q.nf4_codebook().tolist())
+    P = ctypes.c_void_p(1 << 20)
+    w = _wc(rows=64, cols=128)
+    E = _lib
+
+    def fwd(M=4, wc=w, r=8, alpha=16.0, g=1, X=P, Y=P, ws=P, nbytes=1 << 30):
+        return lib.qlora_forward(X, M, ctypes.byref(wc), cb, P, P, r, alpha, g, Y, None, ws, nbytes,
+                                 None, None)
+
+    assert fwd(r=0) == E.QLORA_EINVAL
+    assert fwd(r=257) == E.QLORA_EINVAL
+    assert fwd(alpha=float("inf")) == E.QLORA_EINVAL
+    assert fwd(alpha=float("nan")) == E.QLORA_EINVAL
+    assert fwd(g=2) == E.QLORA_EINVAL
+    assert fwd(M=-1) == E.QLORA_EINVAL
+    assert fwd(X=None) == E.QLORA_EINVAL
+    assert fwd(Y=ctypes.c_void_p((1 << 20) + 2)) == E.QLORA_EINVAL
+    assert fwd(wc=_wc(rows=60)) == E.QLORA_EUNSUPPORTED          # Dout % 8
+    assert fwd(wc=_wc(rows=0)) == E.QLORA_EINVAL
+    assert fwd(nbytes=16) == E.QLORA_EWORKSPACE
+    assert fwd(ws=None) == E.QLORA_EWORKSPACE
+    assert fwd(M=0) == E.QLORA_OK                                 # empty batch: no-op
+    rc = lib.qlora_backward(P, None, 4, ctypes.byref(w), cb, P, P, 8, 16.0, 1, None, P, P, P, P,
+                            1 << 30, None, None)
+    assert rc == E.QLORA_EINVAL
+    # dA needs x
+    rc = lib.qlora_backward(None, P, 4, ctypes.byref(w), cb, P, P, 8, 16.0, 1, None, None, P, None,
+                            P, 1 << 30, None, None)
+    assert rc == E.QLORA_EINVAL
+
+
+def test_workspace_size_deterministic(lib):
+    for M, rows, cols, r, g in [(1, 4096, 4096, 16, 1), (16, 256, 256, 8, 1), (4096, 11008, 4096, 64, 1),
+                                (8192, 28672, 8192, 64, 64), (17, 200, 192, 3, 1)]:
+        w = _wc(rows=rows, cols=cols)
+        a = lib.qlora_workspace_size(M, ctypes.byref(w), r, g, 0)
+        b = lib.qlora_workspace_size(M, ctypes.byref(w), r, g, 1)
+        assert a > 0 and b > 0
+        assert a == lib.qlora_workspace_size(M, ctypes.byref(w), r, g, 0)
+    assert lib.qlora_workspace_size(4, ctypes.byref(_wc(cols=100)), 8, 1, 0) == 0
+    assert lib.qlora_workspace_size(4, ctypes.byref(_wc()), 0, 1, 0) == 0
+
+
+def test_product_codebook_matches_oracle(orc):
+    a = q.nf4_codebook().numpy()
+    b = orc.nf4_codebook()
+    assert np.array_equal(a.view(np.int32), b.view(np.int32))
+
+
+def test_binding_requires_cuda_tensors(lib):
+    W = torch.zeros(64, 64)
+    with pytest.raises(TypeError):
+        q.quantize(W)

@@ -1,0 +1,167 @@
+"""GPU parity of qlora_forward / qlora_backward against the fp64 oracle.
+
+Both kernel paths are covered: the small-M GEMV path (M <= 16) and the
+tensor-core GEMM path (M > 16), with ragged M, Dout and Din, odd ranks, the
+pooled adapter, double quantization on and off, and the full-size workloads
+on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, dev_bf16, host_f64
+from bit_nf4_quantized_22_b200 import synth
+from bit_nf4_quantized_22_b200.synth import LinearSpec
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(orc, qlib, spec: LinearSpec, M: int, cfg: int, lin: int = 0, fwd_only=False,
+             arrays=None, rows=None, check_dadb=True):
+    a = arrays or synth.draw(spec, M, cfg, lin)
+    cb = orc.nf4_codebook()
+    W = torch.from_numpy(a["W"]).cuda()
+    w = qlib.quantize(W, double_quant=spec.double_quant)
+    x, A, B = dev_bf16(a["x"]), dev_bf16(a["A"]), dev_bf16(a["B"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y, T = qlib.forward(x, w, A, B, spec.alpha, spec.pool_group, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_q = orc.quantize(a["W"], cb, spec.double_quant)
+    Wt = orc.dequantize(ref_q, cb)
+    sel = np.arange(M) if rows is None else rows
+    y_ref, T_ref = orc.forward(a["x"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha, spec.pool_group)
+    assert_close(host_f64(y)[sel], y_ref, "y")
+    assert_close(host_f64(T)[sel], T_ref, "T")
+    if fwd_only:
+        return
+    dy = dev_bf16(a["dY"])
+    dX, dA, dB = qlib.backward(x, dy, w, A, B, spec.alpha, spec.pool_group, T=T, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    dX_ref = orc.backward_dx(a["dY"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha, spec.pool_group)
+    assert_close(host_f64(dX)[sel], dX_ref, "dX")
+    if not check_dadb:
+        return
+    dA_ref, dB_ref = orc.backward_dadb(a["x"], a["dY"], a["A"], a["B"], spec.r, spec.alpha,
+                                       spec.pool_group)
+    assert_close(host_f64(dA), dA_ref, "dA")
+    assert_close(host_f64(dB), dB_ref, "dB")
+    # recompute-T path gives the same dB
+    _, _, dB2 = qlib.backward(x, dy, w, A, B, spec.alpha, spec.pool_group, T=None, need_dx=False,
+                              need_dA=False)
+    assert_close(host_f64(dB2), dB_ref, "dB (T recomputed)")
+
+
+def test_config1_full(orc, qlib):
+    cfg = synth.CONFIGS[1]
+    run_case(orc, qlib, cfg["linears"][0], cfg["M"][0], 1)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 17, 100, 300])
+@pytest.mark.parametrize("dq", [False, True])
+def test_ragged_small(orc, qlib, M, dq):
+    spec = LinearSpec("t", 192, 200, 8, 16.0, dq)
+    run_case(orc, qlib, spec, M, 11)
+
+
+@pytest.mark.parametrize("r,alpha", [(1, 1.0), (3, 7.0), (16, 32.0), (64, 128.0), (100, 50.0)])
+@pytest.mark.parametrize("M", [7, 260])
+def test_ranks(orc, qlib, r, alpha, M):
+    spec = LinearSpec("t", 320, 264, r, alpha, True)
+    run_case(orc, qlib, spec, M, 12, lin=r)
+
+
+@pytest.mark.parametrize("M", [3, 16, 130])
+def test_pooled_adapter(orc, qlib, M):
+    spec = LinearSpec("p", 512, 136, 8, 8.0, True, pool_group=64)
+    run_case(orc, qlib, spec, M, 13)
+
+
+def test_pooled_small_din(orc, qlib):
+    """Din/64 not a multiple of 8 (padded pooled buffers)."""
+    spec = LinearSpec("p", 192, 64, 4, 4.0, False, pool_group=64)
+    run_case(orc, qlib, spec, 20, 14)
+    run_case(orc, qlib, spec, 2, 14)
+
+
+def test_worked_example_padded(orc, qlib):
+    """The LoRA worked example (Din=4, Dout=2, r=1) embedded in a Din=64,
+    Dout=8 layer: zero base weight, zero-padded A and x."""
+    A = np.zeros((64, 1), np.float32)
+    A[:4, 0] = [2.0, 0.5, -1.0, 1.5]
+    B = np.zeros((1, 8), np.float32)
+    B[0, :2] = [0.1, -0.2]
+    X = np.zeros((4, 64), np.float32)
+    X[np.arange(4), np.arange(4)] = 1.0
+    arrays = dict(W=np.zeros((8, 64), np.float32), x=synth.bf16_bits(X), A=synth.bf16_bits(A),
+                  B=synth.bf16_bits(B), dY=synth.bf16_bits(np.ones((4, 8), np.float32)))
+    spec = LinearSpec("ex", 64, 8, 1, 1.0, False)
+    run_case(orc, qlib, spec, 4, 0, arrays=arrays)
+    w = qlib.quantize(torch.zeros(8, 64, device="cuda"), double_quant=False)
+    y, _ = qlib.forward(dev_bf16(arrays["x"]), w, dev_bf16(arrays["A"]), dev_bf16(arrays["B"]), 1.0)
+    got = host_f64(y)[:, :2]
+    np.testing.assert_allclose(got, [[0.2, -0.4], [0.05, -0.1], [-0.1, 0.2], [0.15, -0.3]], rtol=2 ** -7)
+
+
+def test_B_zero_is_base_only(orc, qlib):
+    spec = LinearSpec("z", 256, 128, 8, 16.0, True)
+    a = synth.draw(spec, 33, 15)
+    a["B"][:] = 0
+    run_case(orc, qlib, spec, 33, 15, arrays=a)
+    w = qlib.quantize(torch.from_numpy(a["W"]).cuda(), double_quant=True)
+    y, _ = qlib.forward(dev_bf16(a["x"]), w, dev_bf16(a["A"]), dev_bf16(a["B"]), 16.0)
+    Wd = qlib.dequantize(w)
+    ref = (dev_bf16(a["x"]).float() @ Wd.float().t()).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    assert_close(host_f64(y), host_f64(ref), "y vs x @ dequant(W)^T")
+
+
+def test_config2_decode(orc, qlib):
+    cfg = synth.CONFIGS[2]
+    spec = cfg["linears"][0]
+    for M in cfg["M"]:
+        run_case(orc, qlib, spec, M, 2, fwd_only=True)
+
+
+def test_config3_sampled(orc, qlib):
+    cfg = synth.CONFIGS[3]
+    rows = np.array([0, 1, 255, 256, 1023, 2048, 4000, 4095])
+    run_case(orc, qlib, cfg["linears"][0], cfg["M"][0], 3, rows=rows)
+
+
+def test_config4_layer(orc, qlib):
+    cfg = synth.CONFIGS[4]
+    rows = np.array([0, 511, 1024, 2047])
+    for lin, spec in enumerate(cfg["linears"]):
+        if spec.name in ("q", "gate", "down"):
+            run_case(orc, qlib, spec, cfg["M"][0], 4, lin=lin, rows=rows)
+
+
+@pytest.mark.parametrize("lin", [0, 1, 2])
+@pytest.mark.parametrize("M", [1, 16])
+def test_config5_decode(orc, qlib, lin, M):
+    spec = synth.CONFIGS[5]["linears"][lin]
+    run_case(orc, qlib, spec, M, 5, lin=lin)
+
+
+@pytest.mark.parametrize("lin", [0, 1, 2])
+def test_config5_large_sampled(orc, qlib, lin):
+    """M = 8192 on the 70B shapes: y and dX on sampled rows; dA and dB
+    (full reductions over M) are checked on an M = 512 run of the same
+    weights and adapters."""
+    spec = synth.CONFIGS[5]["linears"][lin]
+    rows = np.array([0, 4097, 8191])
+    a = synth.draw(spec, 8192, 5, lin)
+    run_case(orc, qlib, spec, 8192, 5, lin=lin, rows=rows, arrays=a, check_dadb=False)
+    small = dict(W=a["W"], A=a["A"], B=a["B"], x=a["x"][:512].copy(), dY=a["dY"][:512].copy())
+    run_case(orc, qlib, spec, 512, 5, lin=lin, arrays=small)
+
+
+@pytest.mark.parametrize("M", [17, 300])
+def test_warp_mma_large_path(orc, qlib, M, monkeypatch):
+    """The alternative large-M path (dequantize + warp-MMA GEMM) agrees too."""
+    monkeypatch.setenv("QLORA_LARGE_M_PATH", "mma")
+    spec = LinearSpec("t", 192, 200, 8, 16.0, True)
+    run_case(orc, qlib, spec, M, 16)
+    spec = LinearSpec("p", 512, 136, 8, 8.0, True, pool_group=64)
+    run_case(orc, qlib, spec, M, 17)

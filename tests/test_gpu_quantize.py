@@ -1,0 +1,134 @@
+"""GPU parity of nf4_quantize / nf4_dequantize against the oracle: bit-exact
+on packed indices, absmax, double-quant codes and steps, and dequantized bf16
+weights."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import dev_bf16, host_bits, unpack
+from bit_nf4_quantized_22_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quant(qlib, W, dq, cb=None):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w = qlib.quantize(torch.from_numpy(W).cuda(), double_quant=dq, codebook=cb, status=status)
+    torch.cuda.synchronize()
+    return w, int(status.item())
+
+
+def _check_same(orc, qlib, W, dq, cb_np=None):
+    cb_np = orc.nf4_codebook() if cb_np is None else cb_np
+    cb_t = torch.from_numpy(cb_np.copy())
+    ref = orc.quantize(W, cb_np, dq)
+    w, st = _gpu_quant(qlib, W, dq, cb_t)
+    assert st == ref.status
+    gp = w.packed.cpu().numpy()
+    if not np.array_equal(gp, ref.packed):
+        a, b = unpack(gp), unpack(ref.packed)
+        bad = np.flatnonzero(a != b)
+        raise AssertionError(f"{bad.size} indices differ, first at {bad[:5]}: gpu {a[bad[:5]]} ref {b[bad[:5]]}")
+    if dq:
+        assert np.array_equal(w.steps.cpu().numpy().view(np.uint32), ref.steps.view(np.uint32))
+        assert np.array_equal(w.codes.cpu().numpy(), ref.codes)
+    else:
+        assert np.array_equal(w.absmax.cpu().numpy().view(np.uint32), ref.absmax.view(np.uint32))
+    deq = host_bits(qlib.dequantize(w, codebook=cb_t))
+    assert np.array_equal(deq, orc.dequantize(ref, cb_np))
+    return w
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_config1_quantize(orc, qlib, dq):
+    spec = synth.CONFIGS[1]["linears"][0]
+    W = synth.draw(spec, 16, 1, which=("W",))["W"]
+    _check_same(orc, qlib, W, dq)
+
+
+@pytest.mark.parametrize("shape", [(8, 64), (3, 192), (37, 320), (256, 4160)])
+@pytest.mark.parametrize("dq", [False, True])
+def test_ragged_shapes(orc, qlib, shape, dq):
+    """Block counts that leave a partial CTA and a partial double-quant group."""
+    rng = np.random.default_rng(hash(shape) % 2**32)
+    W = (rng.standard_t(4, size=shape) * 0.02).astype(np.float32)
+    _check_same(orc, qlib, W, dq)
+
+
+def test_adversarial_thresholds(orc, qlib):
+    """Weights at and within a few ulps of every decision threshold, for
+    several absmax magnitudes (incl. subnormal-range scales)."""
+    from fractions import Fraction as Fr
+    cb = orc.nf4_codebook()
+    rows = []
+    for a in (1.0, 0.0371, 3.1e-3, 2.0 ** -120, 1.7e30, 6.1e-39):
+        a = np.float32(a)
+        vals = []
+        for j in range(15):
+            t = (Fr(float(cb[j])) + Fr(float(cb[j + 1]))) / 2 * Fr(float(a))
+            x = np.float32(float(t))
+            for k in range(-3, 4):
+                y = x
+                for _ in range(abs(k)):
+                    y = np.nextafter(y, np.float32(np.inf if k > 0 else -np.inf))
+                vals.append(y)
+        vals = np.array(vals, dtype=np.float32)
+        for s in range(0, vals.size, 62):
+            blk = np.zeros(64, np.float32)
+            blk[0], blk[1] = a, -a
+            chunk = vals[s:s + 62]
+            blk[2:2 + chunk.size] = chunk
+            rows.append(blk)
+    W = np.stack(rows).reshape(-1, 64)
+    _check_same(orc, qlib, W, False)
+    _check_same(orc, qlib, W, True)
+
+
+def test_custom_codebooks(orc, qlib):
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((64, 256)) * 0.05).astype(np.float32)
+    W[3, :64] = 0
+    uniform = np.array([-1, -.75, -.5, -.375, -.25, -.125, -.0625, 0, .0625, .125, .25, .375,
+                        .5, .625, .75, 1], dtype=np.float32)
+    tiny = np.array([-1, -.9, -.8, -.7, -.6, -.5, -2.0 ** -60, 0, .5, .6, .7, .75, .8, .85, .9, 1],
+                    dtype=np.float32)
+    for cb in (uniform, tiny, orc.nf4_codebook(1 - 1 / 32)):
+        # exact ties on the uniform table's midpoints
+        W2 = W.copy()
+        W2[0, :16] = (np.concatenate([[1.0], (uniform[:-1] + uniform[1:]) / 2])).astype(np.float32)
+        _check_same(orc, qlib, W2, True, cb)
+
+
+def test_special_blocks_and_status(orc, qlib):
+    W = np.zeros((4, 128), np.float32)
+    W[1, :64] = -0.0
+    W[2, 0], W[2, 1] = 0.5, -0.5
+    W[3, 64:] = 1e-42                       # subnormal block
+    _check_same(orc, qlib, W, True)
+    W[0, 5] = np.nan
+    _, st = _gpu_quant(qlib, W, True)
+    assert st == 1
+    W[0, 5] = np.inf
+    _, st = _gpu_quant(qlib, W, False)
+    assert st == 1
+
+
+def test_empty_weight(qlib):
+    w = qlib.NF4Weight.empty(0, 64, True)
+    qlib.quantize(torch.zeros(0, 64, device="cuda"), out=w)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("cfg,lin", [(3, 0), (4, 6)])
+def test_full_size_quantize(orc, qlib, cfg, lin):
+    """Full-size matrices of the training-shaped workloads, bit-exact."""
+    spec = synth.CONFIGS[cfg]["linears"][lin]
+    W = synth.draw(spec, 1, cfg, lin, which=("W",))["W"]
+    _check_same(orc, qlib, W, spec.double_quant)
+
+
+def test_full_size_quantize_70b(orc, qlib):
+    """The 8192 x 28672 matrix (235M weights), bit-exact on every output."""
+    spec = synth.CONFIGS[5]["linears"][0]
+    W = synth.draw(spec, 1, 5, 0, which=("W",))["W"]
+    _check_same(orc, qlib, W, True)
