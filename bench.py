@@ -78,56 +78,96 @@ def stored_traffic(kernel_file, summary):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling while the timed region runs."""
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons sampled while the timed
+    region runs: NVML polled every 5 ms in a background thread (read-only
+    queries), falling back to `nvidia-smi -lms 200` if NVML is unavailable."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+    SMI_Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, uuid):
         self.uuid = uuid
-        self.proc = None
+        self.samples = []        # (sm_mhz, reasons set, power_w)
+        self.max_mhz = None
+        self.source = None
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200"]
-        if self.uuid:
-            cmd += ["-i", self.uuid]
+        import threading
+        self.stop = threading.Event()
+        self.proc = None
         try:
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nv.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = [(n, getattr(nv, c)) for n, c in self.REASONS if hasattr(nv, c)]
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        self.samples.append((sm, {n for n, m in masks if r & m}, pw))
+                    except Exception:
+                        pass
+                    self.stop.wait(0.005)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml 5 ms"
+        except Exception:
+            self.thread = None
+            cmd = ["nvidia-smi", f"--query-gpu={self.SMI_Q}", "--format=csv,noheader,nounits",
+                   "-lms", "200"] + (["-i", self.uuid] if self.uuid else [])
+            try:
+                self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE,
+                                             stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi 200 ms"
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc:
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(2)
+        if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                out, _ = self.proc.communicate()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in (out or "").splitlines():
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm, self.max_mhz, pw = float(parts[0]), float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                rs = {n for n, v in zip(names, parts[3:7]) if v.lower().startswith("active")}
+                self.samples.append((sm, rs, pw))
 
     def summary(self):
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        sm, mx, reasons = [], None, set()
-        for line in (self.out or "").splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = set()
+        for _, r, _ in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "power_w_max": max(p for _, _, p in self.samples),
+                "samples": len(self.samples), "source": self.source}
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -171,7 +211,7 @@ def run_reference(args, rank):
 
 
 # --------------------------------------------------------------------------- our arm
-def cpu_baseline(rows=256):
+def cpu_baseline(rows=1024):
     """The oracle as it stands on a bounded sample of the workload."""
     import oracle
     spec = synth.CONFIGS[CFG]["linears"][0]
@@ -203,6 +243,7 @@ def run_ours(args, rank, world, dist):
     M = synth.CONFIGS[CFG]["M"][0]
     Din, Dout, r, alpha = spec.Din, spec.Dout, spec.r, spec.alpha
 
+    from bit_nf4_quantized_22_b200.dp import allreduce_adapter_grads
     base = synth.draw(spec, M, CFG, 0, which=("W", "A", "B"))
     batch = synth.draw(spec, M, CFG, rank, which=("x", "dY"))
 
@@ -224,8 +265,7 @@ def run_ours(args, rank, world, dist):
         _, T = q.forward(x, w, A, B, alpha, out=y, workspace=ws_f)
         dX, dA, dB = q.backward(x, dy, w, A, B, alpha, T=T, workspace=ws_b)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            allreduce_adapter_grads(dA, dB)
         return dX, dA, dB
 
     for _ in range(args.warmup):
@@ -410,7 +450,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=16)
     args = ap.parse_args()
     if args.warmup < 3:
