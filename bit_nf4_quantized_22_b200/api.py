@@ -171,6 +171,26 @@ def backward(x: torch.Tensor | None, dy: torch.Tensor, q: NF4Weight, A: torch.Te
     return dX, dA, dB
 
 
+def forward_noalloc(x: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                    alpha: float, pool_group: int = 1, codebook: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, T_out: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None):
+    """qlora_forward_noalloc: the forward with the library's built-in scratch
+    array instead of a workspace.  The caller passes the outputs (`out`,
+    `T_out`); when omitted they are created here, which allocates."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(A, torch.bfloat16, "A", 2)
+    _need(B, torch.bfloat16, "B", 2)
+    M, r = x.shape[0], A.shape[1]
+    y = out if out is not None else torch.empty(M, q.rows, dtype=torch.bfloat16, device=x.device)
+    qc = q.c_struct()
+    rc = load().qlora_forward_noalloc(_ptr(x), M, ctypes.byref(qc), _cb_host(codebook), _ptr(A),
+                                      _ptr(B), r, float(alpha), pool_group, _ptr(y), _ptr(T_out),
+                                      _ptr(status), _stream())
+    _lib.check(rc, "qlora_forward_noalloc")
+    return y, T_out
+
+
 class QLoRALinearFn(torch.autograd.Function):
     """Autograd wrapper: gradients for x, A and B; none for the frozen W4."""
 

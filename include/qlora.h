@@ -145,6 +145,32 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
                    float *dA, float *dB, void *workspace, size_t ws_bytes,
                    uint32_t *d_status, void *stream);
 
+/* ---- Forward without caller-provided scratch -------------------------------
+ * No counterpart on the pages: this entry point exists for callers that cannot
+ * allocate device memory -- code that runs where cudaMalloc is not allowed or
+ * not wanted (inside another allocator's arena, in a process that must not
+ * grow its device footprint after start-up, or a host that simply has no
+ * workspace to hand over).  It computes exactly what qlora_forward computes,
+ * with the same kernels and the same arguments minus the workspace; its
+ * scratch is a fixed array of QLORA_NOALLOC_SCRATCH_BYTES bytes inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *   - Requests needing more scratch than that return QLORA_EWORKSPACE before
+ *     anything is enqueued (qlora_workspace_size(M, q, r, pool_group, 0)
+ *     tells the need; decode-sized calls fit, e.g. M <= 16 at 4096 x 4096).
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; each
+ *     call clears what it needs zeroed.  Calls that overlap on the GPU (two
+ *     streams, or two host threads) race on the array: serialize them. */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int qlora_forward_noalloc(const uint16_t *X, int64_t M, const nf4_weight_t *q,
+                          const float codebook[16], const uint16_t *A, const uint16_t *B,
+                          int32_t r, float alpha, int32_t pool_group, uint16_t *Y, float *T_save,
+                          uint32_t *d_status, void *stream);
+
 /* ---- Benchmark support (not part of the layer's computation) ----------
  * Kernel launches made by the library since the last qlora_profile_reset(). */
 int64_t qlora_launch_count(void);
