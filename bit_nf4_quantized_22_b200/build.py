@@ -13,8 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqlora.so")
-SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "adapter.cu", "umma_gemm.cu", "profile.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "mma_gemm.cuh"]
+SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "adapter.cu", "umma_gemm.cu", "profile.cu", "noalloc.cu", "umma_skinny.cu"]
+HEADERS = ["common.cuh", "mma_gemm.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

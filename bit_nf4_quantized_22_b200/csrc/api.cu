@@ -31,6 +31,21 @@ int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H
                   uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp, cudaStream_t st);
 int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN);
 int launch_mma_gemm(MmaGemmArgs a, int bn, cudaStream_t st);
+// umma_skinny.cu
+struct SkinnySeg {
+    const uint16_t *a;
+    int64_t lda;
+    int a_kmajor;
+    const uint16_t *b;
+    int64_t ldb;
+    int b_kmajor;
+    int64_t qext;
+    int64_t R;
+};
+int skinny_k_tiles(const SkinnySeg *segs, int nseg);
+void skinny_splits(int64_t P, int64_t Q, int nk, int *splits, int *per);
+int launch_umma_skinny(const SkinnySeg *segs, int nseg, int64_t P, int64_t Q, int64_t Qp,
+                       float *partial, uint32_t *d_status, cudaStream_t st);
 // umma_gemm.cu
 int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t &q,
                       const Codebook &cb, const uint16_t *sAct, int r, const uint16_t *adapter,
@@ -117,10 +132,107 @@ Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
     return d;
 }
 
-int t_splits(const Dims &d) { return mma_choose_splits(d.M, d.r, d.g > 1 ? 2 * d.Da : d.Din, 64); }
-int g_splits(const Dims &d) { return mma_choose_splits(d.M, d.r, d.Dout, 64); }
-int da_splits(const Dims &d) { return mma_choose_splits(d.Da, 2 * d.rp, (d.g > 1 ? 2 : 1) * d.M, 128); }
-int db_splits(const Dims &d) { return mma_choose_splits(d.Dout, 2 * d.rp, d.M, 128); }
+// ---------------------------------------------------------------- adapter products
+// C[P, Q] = sum over segments of A(p,t) B(t,q), as fp32 split-K partials
+// [splits][P][Qp]; run on the tcgen05 engine, or on the warp-MMA engine when
+// the warp-MMA path is selected.
+struct Prod {
+    SkinnySeg seg[2];
+    int nseg;
+    int64_t P, Q;
+};
+struct ProdPlan {
+    int splits;
+    int64_t Qp;
+};
+
+ProdPlan plan_prod(const Prod &pr, bool mma) {
+    ProdPlan pl;
+    if (mma) {
+        int64_t R = 0;
+        for (int i = 0; i < pr.nseg; ++i) R += pr.seg[i].R;
+        pl.splits = mma_choose_splits(pr.P, pr.Q, R, pr.Q <= 64 ? 64 : 128);
+        pl.Qp = pr.Q;
+    } else {
+        int per = 1;
+        skinny_splits(pr.P, pr.Q, skinny_k_tiles(pr.seg, pr.nseg), &pl.splits, &per);
+        pl.Qp = round_up(pr.Q, 4);
+    }
+    return pl;
+}
+
+size_t prod_partial_floats(const Prod &pr, bool mma) {
+    const ProdPlan pl = plan_prod(pr, mma);
+    return (size_t)pl.splits * pr.P * pl.Qp;
+}
+
+int run_prod(const Prod &pr, bool mma, float *partial, uint32_t *status, cudaStream_t st,
+             ProdPlan *plan) {
+    *plan = plan_prod(pr, mma);
+    if (!mma) return launch_umma_skinny(pr.seg, pr.nseg, pr.P, pr.Q, plan->Qp, partial, status, st);
+    MmaGemmArgs a{};
+    for (int i = 0; i < pr.nseg; ++i) {
+        const SkinnySeg &g = pr.seg[i];
+        a.seg[i] = MmaSeg{MmaOperand{g.a, g.lda, g.a_kmajor}, MmaOperand{g.b, g.ldb, g.b_kmajor}, g.R};
+    }
+    a.nseg = pr.nseg;
+    a.P = pr.P;
+    a.Q = pr.Q;
+    a.splits = plan->splits;
+    a.partial = partial;
+    return launch_mma_gemm(a, pr.Q <= 64 ? 64 : 128, st);
+}
+
+// T = u . A    (u = x [M, Din], or pooled hi/lo [M, Dap]; A padded [Da, rp])
+Prod prod_T(const Dims &d, const uint16_t *X, const uint16_t *Apad, const uint16_t *ph,
+            const uint16_t *pl) {
+    Prod pr{};
+    if (d.g == 1) {
+        pr.seg[0] = SkinnySeg{X, d.Din, 1, Apad, d.rp, 0, d.rp, d.Din};
+        pr.nseg = 1;
+    } else {
+        pr.seg[0] = SkinnySeg{ph, d.Dap, 1, Apad, d.rp, 0, d.rp, d.Da};
+        pr.seg[1] = SkinnySeg{pl, d.Dap, 1, Apad, d.rp, 0, d.rp, d.Da};
+        pr.nseg = 2;
+    }
+    pr.P = d.M;
+    pr.Q = d.r;
+    return pr;
+}
+// G = dY . B^T   (B [r, Dout] is K-major for this product)
+Prod prod_G(const Dims &d, const uint16_t *dY, const uint16_t *B) {
+    Prod pr{};
+    pr.seg[0] = SkinnySeg{dY, d.Dout, 1, B, d.Dout, 1, d.r, d.Dout};
+    pr.nseg = 1;
+    pr.P = d.M;
+    pr.Q = d.r;
+    return pr;
+}
+// dA-sum = u^T . [G_hi | G_lo]   (reduction over tokens; both MN-major)
+Prod prod_dA(const Dims &d, const uint16_t *X, const uint16_t *ph, const uint16_t *pl,
+             const uint16_t *Gsplit) {
+    Prod pr{};
+    if (d.g == 1) {
+        pr.seg[0] = SkinnySeg{X, d.Din, 0, Gsplit, 2 * d.rp, 0, 2 * d.rp, d.M};
+        pr.nseg = 1;
+    } else {
+        pr.seg[0] = SkinnySeg{ph, d.Dap, 0, Gsplit, 2 * d.rp, 0, 2 * d.rp, d.M};
+        pr.seg[1] = SkinnySeg{pl, d.Dap, 0, Gsplit, 2 * d.rp, 0, 2 * d.rp, d.M};
+        pr.nseg = 2;
+    }
+    pr.P = d.Da;
+    pr.Q = 2 * d.rp;
+    return pr;
+}
+// dB^T-sum = dY^T . [T_hi | T_lo]
+Prod prod_dB(const Dims &d, const uint16_t *dY, const uint16_t *Tsplit) {
+    Prod pr{};
+    pr.seg[0] = SkinnySeg{dY, d.Dout, 0, Tsplit, 2 * d.rp, 0, 2 * d.rp, d.M};
+    pr.nseg = 1;
+    pr.P = d.Dout;
+    pr.Q = 2 * d.rp;
+    return pr;
+}
 
 // Workspace pieces.  The same function sizes (base == nullptr) and carves.
 struct FwdWs {
@@ -141,7 +253,7 @@ size_t layout_fwd(const Dims &d, bool have_tsave, void *base, FwdWs *w) {
         x.pl = b.take<uint16_t>(d.M * d.Dap);
     }
     if (!have_tsave) x.T32 = b.take<float>(d.M * d.r);
-    x.Tpart = b.take<float>((size_t)t_splits(d) * d.M * d.r);
+    x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0), d.mma_large));
     if (d.small) {
         x.gemv_part = b.take<float>(gemv_fwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
     } else {
@@ -157,7 +269,7 @@ size_t layout_bwd(const Dims &d, bool have_tsaved, bool want_dx, bool want_da, b
     Bump b(base);
     BwdWs x{};
     x.G32 = b.take<float>(d.M * d.r);
-    x.Gpart = b.take<float>((size_t)g_splits(d) * d.M * d.r);
+    x.Gpart = b.take<float>(prod_partial_floats(prod_G(d, 0, 0), d.mma_large));
     if (want_da) x.Gsplit = b.take<uint16_t>(d.M * 2 * d.rp);
     if (d.g > 1 && (want_da || (want_db && !have_tsaved))) {
         x.ph = b.take<uint16_t>(d.M * d.Dap);
@@ -167,12 +279,12 @@ size_t layout_bwd(const Dims &d, bool have_tsaved, bool want_dx, bool want_da, b
         if (!have_tsaved) {
             x.Apad = b.take<uint16_t>(d.Da * d.rp);
             x.T32 = b.take<float>(d.M * d.r);
-            x.Tpart = b.take<float>((size_t)t_splits(d) * d.M * d.r);
+            x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0), d.mma_large));
         }
         x.Tsplit = b.take<uint16_t>(d.M * 2 * d.rp);
-        x.dBpart = b.take<float>((size_t)db_splits(d) * d.Dout * 2 * d.rp);
+        x.dBpart = b.take<float>(prod_partial_floats(prod_dB(d, 0, 0), d.mma_large));
     }
-    if (want_da) x.dApart = b.take<float>((size_t)da_splits(d) * d.Da * 2 * d.rp);
+    if (want_da) x.dApart = b.take<float>(prod_partial_floats(prod_dA(d, 0, 0, 0, 0), d.mma_large));
     if (want_dx) {
         if (d.small) {
             x.gemv_part = b.take<float>(gemv_bwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
@@ -219,26 +331,13 @@ Codebook to_cb(const float *c) {
 // T = u . A  ->  T32 [M, r] (and s*T as bf16 into sT [M, rp64] if sT)
 int run_adapter_down(const Dims &d, const uint16_t *X, const uint16_t *A, uint16_t *Apad,
                      const uint16_t *ph, const uint16_t *pl, float *Tpart, float *T32, float s,
-                     uint16_t *sT, cudaStream_t st) {
+                     uint16_t *sT, uint32_t *status, cudaStream_t st) {
     RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st));
-    MmaGemmArgs a{};
-    const MmaOperand Bop{Apad, d.rp, 0};
-    if (d.g == 1) {
-        a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 1}, Bop, d.Din};
-        a.nseg = 1;
-    } else {
-        a.seg[0] = MmaSeg{MmaOperand{ph, d.Dap, 1}, Bop, d.Da};
-        a.seg[1] = MmaSeg{MmaOperand{pl, d.Dap, 1}, Bop, d.Da};
-        a.nseg = 2;
-    }
-    a.P = d.M;
-    a.Q = d.r;
-    a.splits = t_splits(d);
-    a.partial = Tpart;
-    RC(launch_mma_gemm(a, 64, st));
+    ProdPlan plan;
+    RC(run_prod(prod_T(d, X, Apad, ph, pl), d.mma_large, Tpart, status, st, &plan));
     if (sT && cudaMemsetAsync(sT, 0, d.M * d.rp64 * sizeof(uint16_t), st) != cudaSuccess)
         return QLORA_ECUDA;
-    return launch_reduce(Tpart, a.splits, d.M, d.r, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
+    return launch_reduce(Tpart, plan.splits, d.M, plan.Qp, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
                          nullptr, 0, st);
 }
 
@@ -316,7 +415,8 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
     float *T32 = T_save ? T_save : w.T32;
 
     if (d.g > 1) RC(run_pool(d, X, w.ph, w.pl, st));
-    RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT, st));
+    RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT,
+                        d_status, st));
     if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, st);
     if (!d.mma_large) return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
     // warp-MMA path: dequantize to a bf16 copy, then one two-segment GEMM
@@ -357,20 +457,14 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
 
     // G = dY . B^T  (fp32), s*G (bf16, large M), hi/lo split (for dA)
     {
-        MmaGemmArgs a{};
-        a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 1}, MmaOperand{B, d.Dout, 1}, d.Dout};
-        a.nseg = 1;
-        a.P = M;
-        a.Q = r;
-        a.splits = g_splits(d);
-        a.partial = w.Gpart;
-        RC(launch_mma_gemm(a, 64, st));
+        ProdPlan pl;
+        RC(run_prod(prod_G(d, dY, B), d.mma_large, w.Gpart, d_status, st, &pl));
         uint16_t *sG = (want_dx && !d.small) ? w.sG : nullptr;
         if (sG && cudaMemsetAsync(sG, 0, M * d.rp64 * 2, st) != cudaSuccess) return QLORA_ECUDA;
         if (w.Gsplit && cudaMemsetAsync(w.Gsplit, 0, M * 2 * d.rp * 2, st) != cudaSuccess)
             return QLORA_ECUDA;
-        RC(launch_reduce(w.Gpart, a.splits, M, r, 0, r, 1.f, w.G32, r, 1, s, sG, d.rp64, w.Gsplit,
-                         d.rp, st));
+        RC(launch_reduce(w.Gpart, pl.splits, M, pl.Qp, 0, r, 1.f, w.G32, r, 1, s, sG, d.rp64,
+                         w.Gsplit, d.rp, st));
     }
     if (d.g > 1 && w.ph) RC(run_pool(d, X, w.ph, w.pl, st));
 
@@ -398,40 +492,21 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
         }
     }
     if (want_da) {
-        MmaGemmArgs a{};
-        const MmaOperand Gop{w.Gsplit, 2 * d.rp, 0};
-        if (d.g == 1) {
-            a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 0}, Gop, M};
-            a.nseg = 1;
-        } else {
-            a.seg[0] = MmaSeg{MmaOperand{w.ph, d.Dap, 0}, Gop, M};
-            a.seg[1] = MmaSeg{MmaOperand{w.pl, d.Dap, 0}, Gop, M};
-            a.nseg = 2;
-        }
-        a.P = d.Da;
-        a.Q = 2 * d.rp;
-        a.splits = da_splits(d);
-        a.partial = w.dApart;
-        RC(launch_mma_gemm(a, 128, st));
-        RC(launch_reduce(w.dApart, a.splits, d.Da, 2 * d.rp, d.rp, r, s, dA, r, 1, 0.f, nullptr, 0,
+        ProdPlan pl;
+        RC(run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), d.mma_large, w.dApart, d_status, st, &pl));
+        RC(launch_reduce(w.dApart, pl.splits, d.Da, pl.Qp, d.rp, r, s, dA, r, 1, 0.f, nullptr, 0,
                          nullptr, 0, st));
     }
     if (want_db) {
         const float *T32 = T_saved;
         if (!T32) {
-            RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, w.T32, s, nullptr, st));
+            RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, w.T32, s, nullptr, d_status, st));
             T32 = w.T32;
         }
         RC(launch_split_f32(T32, M, r, d.rp, w.Tsplit, st));
-        MmaGemmArgs a{};
-        a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 0}, MmaOperand{w.Tsplit, 2 * d.rp, 0}, M};
-        a.nseg = 1;
-        a.P = d.Dout;
-        a.Q = 2 * d.rp;
-        a.splits = db_splits(d);
-        a.partial = w.dBpart;
-        RC(launch_mma_gemm(a, 128, st));
-        RC(launch_reduce(w.dBpart, a.splits, d.Dout, 2 * d.rp, d.rp, r, s, dB, 1, d.Dout, 0.f,
+        ProdPlan pl;
+        RC(run_prod(prod_dB(d, dY, w.Tsplit), d.mma_large, w.dBpart, d_status, st, &pl));
+        RC(launch_reduce(w.dBpart, pl.splits, d.Dout, pl.Qp, d.rp, r, s, dB, 1, d.Dout, 0.f,
                          nullptr, 0, nullptr, 0, st));
     }
     return QLORA_OK;

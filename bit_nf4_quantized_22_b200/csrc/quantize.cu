@@ -7,6 +7,7 @@
 // in the high nibble.  Double quantization (section 7.2): per 256 blocks,
 // step f = RN32(max a / 255), code = round-half-even(a / f) in [0, 255].
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace qlora {
 namespace {
@@ -52,25 +53,54 @@ __device__ __forceinline__ uint32_t level_index(float w, const float t[15]) {
     return (uint32_t(b3) << 3) | (uint32_t(b2) << 2) | (uint32_t(b1) << 1) | uint32_t(b0);
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
-k_nf4_quantize(const float *__restrict__ W, int64_t nb, Codebook cb, int zero_idx, int dq,
-               uint8_t *__restrict__ packed, float *__restrict__ absmax,
+// One CTA per double-quant group of 256 blocks (64 KB of fp32 weights).
+// The group is brought into shared memory by two TMA tile loads (columns
+// 0-31 and 32-63 of the [nb, 64] view, 128-byte swizzle), so the DRAM stream
+// is sequential and thread t -- owning block b0 + t -- reads its row with
+// 16-byte loads that hit 8 different bank groups per 8 threads.
+constexpr int kQuantSmem = 2 * 256 * 128 + 1024;
+
+__global__ void __launch_bounds__(kQuantThreads, 2)
+k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, int zero_idx,
+               int dq, uint8_t *__restrict__ packed, float *__restrict__ absmax,
                uint8_t *__restrict__ codes, float *__restrict__ steps,
                uint32_t *__restrict__ status) {
-    const int64_t b = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x;
+    extern __shared__ __align__(1024) uint8_t qsm_raw[];
+    __shared__ __align__(8) uint64_t bar_storage;
+    __shared__ int abort_flag;
+    __shared__ float warp_max[kQuantThreads / 32];
+    const uint32_t raw = smem_u32(qsm_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    const uint32_t bar = smem_u32(&bar_storage);
+    const int64_t b0 = (int64_t)blockIdx.x * kQuantThreads;
+    const int64_t b = b0 + threadIdx.x;
     const bool valid = b < nb;
-    float w[64];
-    if (valid) {
-        const float4 *src = reinterpret_cast<const float4 *>(W + b * 64);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 v = __ldg(src + i);
-            w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) w[i] = 0.f;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        tc::fence_proxy_async();
+        tc::mbar_expect_tx(bar, 2 * 256 * 128);
+        tc::tma_load_2d(sbase, &tW, 0, (int)b0, bar);
+        tc::tma_load_2d(sbase + 256 * 128, &tW, 32, (int)b0, bar);
     }
+    __syncthreads();
+    const bool arrived = tc::mbar_wait(bar, 0, &abort_flag);
+    if (!arrived && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
+
+    float w[64];
+    const uint32_t row = threadIdx.x, sw = row & 7;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = tc::lds128(sbase + h * 256 * 128 + row * 128 + ((c ^ sw) << 4));
+            w[32 * h + 4 * c + 0] = __uint_as_float(v.x);
+            w[32 * h + 4 * c + 1] = __uint_as_float(v.y);
+            w[32 * h + 4 * c + 2] = __uint_as_float(v.z);
+            w[32 * h + 4 * c + 3] = __uint_as_float(v.w);
+        }
     float a = 0.f;
     uint32_t bad = 0;
 #pragma unroll
@@ -78,7 +108,8 @@ k_nf4_quantize(const float *__restrict__ W, int64_t nb, Codebook cb, int zero_id
         a = fmaxf(a, fabsf(w[i]));
         bad |= ((__float_as_uint(w[i]) & 0x7f800000u) == 0x7f800000u);
     }
-    if (bad && status) atomicOr(status, QLORA_STATUS_NONFINITE);
+    if (valid && bad && status) atomicOr(status, QLORA_STATUS_NONFINITE);
+    if (!valid) a = 0.f;
 
     if (valid) {
         uint32_t out[8];
@@ -110,8 +141,7 @@ k_nf4_quantize(const float *__restrict__ W, int64_t nb, Codebook cb, int zero_id
 
     if (dq) {
         // group max over this CTA's 256 blocks (one double-quant group)
-        __shared__ float warp_max[kQuantThreads / 32];
-        float m = valid ? a : 0.f;
+        float m = a;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
@@ -167,9 +197,15 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
     const int64_t grid = (nb + kQuantThreads - 1) / kQuantThreads;
+    // the weight viewed as [nb rows][64 fp32], loaded 32 columns x 256 rows at a time
+    CUtensorMap tW;
+    if (!tc::make_map(&tW, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, (uint64_t)nb, 256, 32, 256,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return QLORA_EUNSUPPORTED;
+    cudaFuncSetAttribute(k_nf4_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
     prof_begin(kProfQuant, st);
-    k_nf4_quantize<<<(unsigned)grid, kQuantThreads, 0, st>>>(
-        W, nb, cb, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
+    k_nf4_quantize<<<(unsigned)grid, kQuantThreads, kQuantSmem, st>>>(
+        tW, nb, cb, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
         d_status);
     prof_end(kProfQuant, st);
     QLORA_LAUNCH_CHECK();
