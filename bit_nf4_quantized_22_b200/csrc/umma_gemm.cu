@@ -263,18 +263,16 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             valid = row < p.Dout && col < p.Din;
             return row * nbr + col / 64;
         };
-        bool v0 = false;
-        ScaleRaw pf = fetch_scale(p.sc, scale_index(0, v0), v0);
-        for (int it = 0; it < p.nk && ok; ++it) {
+        auto fetch = [&](int kt) -> ScaleRaw {
+            bool v = false;
+            const int64_t b = kt < p.nk ? scale_index(kt, v) : 0;
+            return fetch_scale(p.sc, b, v && kt < p.nk);
+        };
+        // one k-tile of dequantization, given its (already fetched) scale
+        auto body = [&](int it, const ScaleRaw &cur) -> bool {
             const int s = it % kStages;
-            const ScaleRaw cur = pf;
-            if (it + 1 < p.nk) {
-                bool v = false;
-                const int64_t b = scale_index(it + 1, v);
-                pf = fetch_scale(p.sc, b, v);
-            }
-            ok = __all_sync(0xffffffffu, mbar_wait(full_p(s), (it / kStages) & 1, abort_flag));
-            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(full_p(s), (it / kStages) & 1, abort_flag)))
+                return false;
             const uint32_t sp = base + s * kStageBytes + kABytes;
             const uint32_t sb = sp + kPBytes;
             const float ah = decode_scale(cur, p.sc.dq);
@@ -291,6 +289,22 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(bready(s));
+            return true;
+        };
+        // scales are fetched three k-tiles ahead of use
+        ScaleRaw r0 = fetch(0), r1 = fetch(1), r2 = fetch(2);
+        for (int it = 0; it < p.nk && ok; it += 3) {
+            ScaleRaw cur = r0;
+            r0 = fetch(it + 3);
+            ok = body(it, cur);
+            if (!ok || it + 1 >= p.nk) break;
+            cur = r1;
+            r1 = fetch(it + 4);
+            ok = body(it + 1, cur);
+            if (!ok || it + 2 >= p.nk) break;
+            cur = r2;
+            r2 = fetch(it + 5);
+            ok = body(it + 2, cur);
         }
         if (!ok) *abort_flag = 1;
 
