@@ -433,7 +433,7 @@ def decode_lines(args, q, lib, torch, dev, hbm, flush):
             kern_ms = ms.value / max(1, n.value)
             res[f"{spec.Din}x{spec.Dout}_M{M}"] = {
                 "forward_ms": step, "weight_GBps": wb / (step / 1e3) / 1e9,
-                "kernel": "k_gemv_fwd", "kernel_ms": kern_ms,
+                "kernel": "k_gemv_fwd_stream", "kernel_ms": kern_ms,
                 "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
                 "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None,
                 "tflops": (2 * M * spec.Din * spec.Dout + 2 * M * spec.r * (spec.Din + spec.Dout)) / (step / 1e3) / 1e12,

@@ -16,7 +16,7 @@ size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout);
 size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout);
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, cudaStream_t st);
+                    float *partial, uint32_t *d_status, cudaStream_t st);
 int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *G, const uint16_t *Al, int r, int pool, float s, uint16_t *dX,
                     float *partial, cudaStream_t st);
@@ -417,7 +417,7 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
     if (d.g > 1) RC(run_pool(d, X, w.ph, w.pl, st));
     RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT,
                         d_status, st));
-    if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, st);
+    if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, d_status, st);
     if (!d.mma_large) return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
     // warp-MMA path: dequantize to a bf16 copy, then one two-segment GEMM
     RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));

@@ -9,6 +9,7 @@
 // Partial sums over the reduction are written per split and reduced by a
 // finalize kernel that also adds the rank-r adapter term.
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace qlora {
 namespace {
@@ -176,6 +177,208 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
         }
 }
 
+// ------------------------------------------------------------------ forward, streamed
+// Persistent variant: one CTA per SM walks a contiguous range of
+// (input-slice, 128-row) tiles.  A producer warp streams each tile's packed
+// weights (128 rows x 512 bytes, four 128-byte-swizzled TMA boxes) and its
+// scale codes into a two-stage shared-memory ring, so ~70 KB per SM are in
+// flight independently of registers; eight compute warps decode from shared
+// memory exactly as k_gemv_fwd does from registers.  Needs the scale rows to
+// be TMA-tileable: Din/64 a multiple of 16 (codes) or of 4 (fp32 absmax).
+constexpr int kStRows = 128, kStBlocks = 16;              // tile: 128 rows x 1024 inputs
+constexpr int kStPacked = kStRows * kStBlocks * 32;       // 64 KB
+constexpr int kStStage = kStPacked + 8192;                // + scale tile (codes 2 KB / fp32 8 KB)
+constexpr int kStStages = 2;
+constexpr int kStThreads = (kGemvWarps + 1) * 32;
+constexpr int kStLut = 256 * 32 * 4;
+constexpr int kStX = (16 * (kFwdKS + 8) * 2 + 1023) / 1024 * 1024;
+constexpr int kStSmem = kStLut + kStX + kStStages * kStStage + 1024 + 256;
+
+template <int NT>
+__global__ void __launch_bounds__(kStThreads, 1)
+k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmC,
+                  const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout, ScaleSrc sc,
+                  Codebook cb, int ntr, int ntiles, float *__restrict__ partial,
+                  uint32_t *__restrict__ status) {
+    extern __shared__ __align__(1024) uint8_t ssm[];
+    const uint32_t raw = smem_u32(ssm);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = ssm + (base - raw);
+    uint32_t *lut = reinterpret_cast<uint32_t *>(gbase);
+    uint16_t(*sx)[kFwdKS + 8] = reinterpret_cast<uint16_t(*)[kFwdKS + 8]>(gbase + kStLut);
+    const uint32_t ring = base + kStLut + kStX;          // 1 KB aligned, as 128-byte swizzling needs
+    const uint32_t bar0 = ring + kStStages * kStStage;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kStStages + s); };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + (bar0 - base) + 64);
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int G = gridDim.x;
+    const int t0 = (int)((int64_t)blockIdx.x * ntiles / G);
+    const int t1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / G);
+    const int64_t nbr = Din / 64;
+
+    // the codebook goes through shared memory: indexing the parameter array
+    // by a thread-dependent value would copy it to the stack
+    float *cbs = reinterpret_cast<float *>(gbase + (bar0 - base) + 128);
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
+        for (int s = 0; s < kStStages; ++s) {
+            tc::mbar_init(full(s), 1);
+            tc::mbar_init(empty(s), kGemvWarps);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        tc::fence_proxy_async();
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {   // pair table, one entry per thread (see k_gemv_fwd)
+        const int e = threadIdx.x;
+        const uint32_t v = bf16x2_bits(cbs[e >> 4], cbs[e & 15]);
+        uint4 *row = reinterpret_cast<uint4 *>(lut + e * 32);
+        const uint4 vv = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) row[(i + lane) & 7] = vv;
+    }
+    for (int i = threadIdx.x; i < (16 - M) * (kFwdKS / 8); i += blockDim.x) {
+        const int m = M + i / (kFwdKS / 8), kc = (i % (kFwdKS / 8)) * 8;
+        *reinterpret_cast<uint4 *>(&sx[m][kc]) = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    bool ok = true;
+
+    if (warp == kGemvWarps) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint32_t cbytes = sc.dq ? kStRows * 16 : kStRows * 16 * 4;
+            for (int i = 0, tt = t0; tt < t1 && ok; ++i, ++tt) {
+                const int s = i % kStStages;
+                if (i >= kStStages) ok = tc::mbar_wait(empty(s), ((i / kStStages) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                const int z = tt / ntr, rt = tt % ntr;
+                const uint32_t st = ring + s * kStStage;
+                tc::mbar_expect_tx(full(s), kStPacked + cbytes);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    tc::tma_load_2d(st + q * (kStRows * 128), &tmP, z * (kFwdKS / 2) + 128 * q,
+                                    rt * kStRows, full(s));
+                tc::tma_load_2d(st + kStPacked, &tmC, z * kStBlocks, rt * kStRows, full(s));
+            }
+            if (!ok) *abort_flag = 1;
+        }
+    } else {
+        // ---------------------------------------------------------- compute warps
+        const uint32_t *lut_lane = lut + lane;
+        auto lookup = [&](uint32_t word, int i) -> uint32_t {
+            return lut_lane[__byte_perm(word, 0u, 0x4440u + i) << 5];
+        };
+        const int rl = warp * 16 + g;                  // rows rl and rl + 8 of the tile
+        // Every compute warp walks the same tiles and meets the same named
+        // barriers; after a failed wait a warp keeps walking (skipping the
+        // work) so that no other warp is left at a barrier.
+        int prev_z = -1;
+        for (int i = 0, tt = t0; tt < t1; ++i, ++tt) {
+            const int s = i % kStStages;
+            const int z = tt / ntr, rt = tt % ntr;
+            const int64_t k0 = (int64_t)z * kFwdKS;
+            const int64_t row0 = (int64_t)rt * kStRows + rl;
+            const bool ok0 = row0 < Dout, ok1 = row0 + 8 < Dout;
+            // with double quantization a row's 16 blocks of this slice start at a
+            // multiple of 16 and so lie inside one group of 256 blocks
+            float step0 = 0.f, step1 = 0.f;
+            if (sc.dq) {
+                if (ok0) step0 = __ldg(sc.step + ((row0 * nbr + z * kStBlocks) >> 8));
+                if (ok1) step1 = __ldg(sc.step + (((row0 + 8) * nbr + z * kStBlocks) >> 8));
+            }
+            if (z != prev_z) {                         // stage x[:M, k0 : k0 + 1024]
+                asm volatile("bar.sync 1, %0;\n" ::"n"(kGemvWarps * 32));
+                for (int j = threadIdx.x; j < M * (kFwdKS / 8); j += kGemvWarps * 32) {
+                    const int m = j / (kFwdKS / 8), kc = (j % (kFwdKS / 8)) * 8;
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (k0 + kc < Din) v = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)m * Din + k0 + kc));
+                    *reinterpret_cast<uint4 *>(&sx[m][kc]) = v;
+                }
+                asm volatile("bar.sync 1, %0;\n" ::"n"(kGemvWarps * 32));
+                prev_z = z;
+            }
+            if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (i / kStStages) & 1, abort_flag));
+            if (!ok) {
+                *abort_flag = 1;
+                continue;
+            }
+            const uint32_t st = ring + s * kStStage;
+            const int nblk = (int)((Din - k0) / 64 < kStBlocks ? (Din - k0) / 64 : kStBlocks);
+            float acc[NT][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+#pragma unroll 4
+            for (int b = 0; b < kStBlocks; ++b) {
+                if (b >= nblk) break;
+                // packed: box q = b/4 holds rows x 128 B; this lane's 8 bytes of
+                // block b are 16-byte chunk 2(b%4) + t/2 (swizzled by row), half t%2
+                const uint32_t chunk = 2 * (b & 3) + (t >> 1);
+                const uint32_t boff = st + (b >> 2) * (kStRows * 128) + ((chunk ^ (rl & 7)) << 4) + 8 * (t & 1);
+                uint2 w0, w1;
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0.x), "=r"(w0.y) : "r"(boff + rl * 128) : "memory");
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w1.x), "=r"(w1.y) : "r"(boff + (rl + 8) * 128) : "memory");
+                float a0 = 0.f, a1 = 0.f;
+                if (sc.dq) {
+                    const uint8_t *cs = gbase + (st - base) + kStPacked;
+                    a0 = __fmul_rn((float)cs[rl * 16 + b], step0);
+                    a1 = __fmul_rn((float)cs[(rl + 8) * 16 + b], step1);
+                } else {
+                    const float *as = reinterpret_cast<const float *>(gbase + (st - base) + kStPacked);
+                    a0 = as[rl * 16 + b];
+                    a1 = as[(rl + 8) * 16 + b];
+                }
+                float tmp[NT][4];
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) tmp[n][e] = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t x0 = q < 2 ? w0.x : w0.y;
+                    const uint32_t x1 = q < 2 ? w1.x : w1.y;
+                    const int i0 = (2 * q) & 3;
+                    const uint32_t a[4] = {lookup(x0, i0), lookup(x1, i0), lookup(x0, i0 + 1),
+                                           lookup(x1, i0 + 1)};
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][64 * b + 16 * t + 4 * q]);
+                        const uint32_t bb[2] = {xv.x, xv.y};
+                        mma_bf16_16816(tmp[n], a, bb);
+                    }
+                }
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    acc[n][0] = fmaf(a0, tmp[n][0], acc[n][0]);
+                    acc[n][1] = fmaf(a0, tmp[n][1], acc[n][1]);
+                    acc[n][2] = fmaf(a1, tmp[n][2], acc[n][2]);
+                    acc[n][3] = fmaf(a1, tmp[n][3], acc[n][3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty(s));
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int m = 8 * n + 2 * t + (e & 1);
+                    const int64_t row = row0 + 8 * (e >> 1);
+                    if (m < M && row < Dout) partial[((int64_t)z * M + m) * Dout + row] = acc[n][e];
+                }
+        }
+    }
+    if (!ok && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
+    __syncwarp();
+    __syncthreads();
+}
+
 // y[m, n] = sum_split partial + s * sum_j T[m, j] B[j, n]
 __global__ void k_gemv_fwd_finalize(const float *__restrict__ partial, int nsplit, int M,
                                     int64_t Dout, const float *__restrict__ T,
@@ -329,21 +532,62 @@ size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     return nsplit > 1 ? (size_t)nsplit * M * Din * sizeof(float) : 0;
 }
 
+static int num_sms_gemv() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, cudaStream_t st) {
+                    float *partial, uint32_t *d_status, cudaStream_t st) {
     const int64_t Din = q.cols, Dout = q.rows;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
     const int64_t nsplit = (Din + kFwdKS - 1) / kFwdKS;
-    const size_t smem = 256 * 32 * 4 + 16 * (kFwdKS + 8) * 2;   // pair table + x slice
-    dim3 grid((unsigned)((Dout + kFwdRows - 1) / kFwdRows), (unsigned)nsplit);
+    const int64_t nbr = Din / 64;
+    // streamed kernel: scale rows must be TMA-tileable (row pitch a multiple
+    // of 16 bytes) and the weight at least one slice wide; else the register kernel
+    bool stream = Din >= kFwdKS && (q.double_quant ? (nbr % 16 == 0) : (nbr % 4 == 0));
+    CUtensorMap tmP, tmC;
+    if (stream) {
+        stream = tc::make_map(&tmP, q.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Din / 2, Dout, Din / 2,
+                              128, kStRows, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (q.double_quant)
+            stream = stream && tc::make_map(&tmC, q.absmax_code, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nbr,
+                                            Dout, nbr, 16, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+        else
+            stream = stream && tc::make_map(&tmC, q.absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, nbr,
+                                            Dout, nbr * 4, 16, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
     prof_begin(kProfGemv, st);
-    if (M <= 8) {
-        cudaFuncSetAttribute(k_gemv_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemv_fwd<1><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
+    if (stream) {
+        const int ntr = (int)((Dout + kStRows - 1) / kStRows);
+        const int ntiles = (int)(ntr * nsplit);
+        const int grid = ntiles < num_sms_gemv() ? ntiles : num_sms_gemv();
+        if (M <= 8) {
+            cudaFuncSetAttribute(k_gemv_fwd_stream<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
+            k_gemv_fwd_stream<1><<<grid, kStThreads, kStSmem, st>>>(tmP, tmC, X, M, Din, Dout, sc, cb,
+                                                                     ntr, ntiles, partial, d_status);
+        } else {
+            cudaFuncSetAttribute(k_gemv_fwd_stream<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
+            k_gemv_fwd_stream<2><<<grid, kStThreads, kStSmem, st>>>(tmP, tmC, X, M, Din, Dout, sc, cb,
+                                                                     ntr, ntiles, partial, d_status);
+        }
     } else {
-        cudaFuncSetAttribute(k_gemv_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemv_fwd<2><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
+        const size_t smem = 256 * 32 * 4 + 16 * (kFwdKS + 8) * 2;   // pair table + x slice
+        dim3 grid((unsigned)((Dout + kFwdRows - 1) / kFwdRows), (unsigned)nsplit);
+        if (M <= 8) {
+            cudaFuncSetAttribute(k_gemv_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            k_gemv_fwd<1><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
+        } else {
+            cudaFuncSetAttribute(k_gemv_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            k_gemv_fwd<2><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
+        }
     }
     prof_end(kProfGemv, st);
     QLORA_LAUNCH_CHECK();

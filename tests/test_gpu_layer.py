@@ -64,6 +64,19 @@ def test_ragged_small(orc, qlib, M, dq):
     run_case(orc, qlib, spec, M, 11)
 
 
+@pytest.mark.parametrize("M,Din,Dout,dq", [
+    (1, 1536, 296, False),    # streamed GEMV: ragged 128-row tile, last input slice half full
+    (16, 1536, 296, False),
+    (9, 3072, 1000, True),    # streamed GEMV, double quantization, 3 slices
+    (4, 2048, 4104, True),    # more tiles than SMs
+    (3, 1088, 264, True),     # Din/64 = 17: scale rows not tileable -> register GEMV
+    (12, 4160, 136, False),   # Din/64 = 65 (odd): register GEMV, ragged slice
+])
+def test_gemv_paths(orc, qlib, M, Din, Dout, dq):
+    spec = LinearSpec("g", Din, Dout, 8, 16.0, dq)
+    run_case(orc, qlib, spec, M, 14, lin=Din + Dout)
+
+
 @pytest.mark.parametrize("r,alpha", [(1, 1.0), (3, 7.0), (16, 32.0), (64, 128.0), (100, 50.0)])
 @pytest.mark.parametrize("M", [7, 260])
 def test_ranks(orc, qlib, r, alpha, M):
