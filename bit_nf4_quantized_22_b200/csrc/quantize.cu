@@ -6,6 +6,8 @@
 // (exact arithmetic, first index on ties); two indices per byte, element 2i
 // in the high nibble.  Double quantization (section 7.2): per 256 blocks,
 // step f = RN32(max a / 255), code = round-half-even(a / f) in [0, 255].
+#include <cmath>
+
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -13,6 +15,14 @@ namespace qlora {
 namespace {
 
 constexpr int kQuantThreads = 256;   // one thread per block, one CTA per DQ group
+
+// Tables of the fast kernel: T[bin] for 32 bins, four bits each, and the
+// halved codebook midpoints h_k = (c_k + c_{k+1}) / 2 when each is exact in
+// fp64 with at most 29 significant bits (then h_k * a is exact in fp64).
+struct QuantBins {
+    uint32_t nib[4];
+    double half[15];
+};
 
 __device__ __forceinline__ float next_up(float x) {
     const uint32_t u = __float_as_uint(x);
@@ -51,6 +61,36 @@ __device__ __forceinline__ uint32_t level_index(float w, const float t[15]) {
                         : (b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]));
     const bool b0 = w >= t0;
     return (uint32_t(b3) << 3) | (uint32_t(b2) << 2) | (uint32_t(b1) << 1) | uint32_t(b0);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Double-quant code RNE(a / f) clamped to [0, 255].  For f in [2^-100, 2^100]:
+// an approximate quotient c (within one of the answer, as a / f <= 256 and
+// the approximation errs by < 2^-14), then the signs of a - (c +- 1/2) f
+// from one fma each -- a correctly rounded fma has the sign of the exact
+// value and is zero only when it is -- decide c - 1, c or c + 1, ties to
+// even.  Other f: the quotient in fp64, whose rint is exact for these ratios.
+__device__ __forceinline__ int dq_code(float a, float f) {
+    if (!(f > 0.f)) return 0;
+    float c;
+    if (f >= 0x1p-100f && f <= 0x1p100f) {
+        c = rintf(__fmul_rn(a, rcp_approx(f)));
+        const float hi = fmaf(-(c + 0.5f), f, a);
+        const float lo = fmaf(-(c - 0.5f), f, a);
+        const bool odd = ((int)c & 1) != 0;
+        if (hi > 0.f || (hi == 0.f && odd))
+            c += 1.f;
+        else if (lo < 0.f || (lo == 0.f && odd))
+            c -= 1.f;
+    } else {
+        c = (float)rint(__ddiv_rn((double)a, (double)f));
+    }
+    return (int)fminf(fmaxf(c, 0.f), 255.f);
 }
 
 // One CTA per double-quant group of 256 blocks (64 KB of fp32 weights).
@@ -165,6 +205,159 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
     }
 }
 
+// ------------------------------------------------------------------ fast path
+// One CTA per group of 256 blocks, brought in by four 16 KB bulk copies so
+// work starts when the first quarter lands.  A warp takes two blocks at a
+// time: lanes 0-15 the first, 16-31 the second, four consecutive weights per
+// lane.  Lane j of a half also holds the exact threshold tau_j of its block
+// (lane 15: +inf).  A weight's index then costs one table lookup and one
+// exact compare instead of a four-level search:
+//   bin = RN(K * (w * RN(1/a)) + 16)          (approximate)
+//   j~  = T[bin]                              (thresholds surely below the bin)
+//   q   = j~ + (w >= tau_{j~})
+// The host builds T for the codebook and proves that every bin, widened by a
+// margin far above the error of the approximate w/a, holds at most one
+// threshold; only then is this kernel used, and the one compare is exact.
+// Blocks with a = 0, a tiny or huge a, or a non-finite weight take the
+// branch-free search (warp-uniform branch).
+constexpr float kBinK = 15.49f;
+constexpr float kBinC = 12582928.0f;   // 1.5 * 2^23 + 16: the low 5 bits of the sum are the bin
+constexpr int kQfThreads = 256;
+constexpr int kQfSmem = 256 * 64 * 4;
+
+template <bool kExactHalf>
+__global__ void __launch_bounds__(kQfThreads, 3)
+k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins,
+                    int zero_idx, int dq, uint8_t *__restrict__ packed,
+                    float *__restrict__ absmax, uint8_t *__restrict__ codes,
+                    float *__restrict__ steps, uint32_t *__restrict__ status) {
+    extern __shared__ __align__(128) float qw[];   // [256 blocks][64 weights]
+    __shared__ __align__(8) uint64_t bars[4];
+    __shared__ float s_a[kQfThreads];
+    __shared__ float s_cb[16];
+    __shared__ double s_half[16];
+    __shared__ uint32_t s_lut[32];
+    __shared__ float warp_max[kQfThreads / 32];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t b0 = (int64_t)blockIdx.x * 256;
+    const int nblk = (int)(nb - b0 < 256 ? nb - b0 : 256);
+    s_a[threadIdx.x] = 0.f;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::mbar_init(smem_u32(&bars[c]), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        tc::fence_proxy_async();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int n = nblk - 64 * c;
+            if (n > 0) {
+                const uint32_t bytes = (uint32_t)(n < 64 ? n : 64) * 256u;
+                tc::mbar_expect_tx(smem_u32(&bars[c]), bytes);
+                tc::bulk_load(smem_u32(qw) + c * 16384u, W + (b0 + 64 * c) * 64, bytes, smem_u32(&bars[c]));
+            }
+        }
+        // parameter arrays are copied with constant indices only (a
+        // lane-dependent index would put the whole parameter on the stack)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s_cb[j] = cb.c[j];
+#pragma unroll
+        for (int j = 0; j < 15; ++j) s_half[j] = bins.half[j];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s_lut[i] = (bins.nib[i >> 3] >> (4 * (i & 7))) & 15u;
+    }
+    __syncthreads();
+    const int j = lane & 15, half = lane >> 4;
+    const float c_lo = s_cb[j < 15 ? j : 14], c_hi = s_cb[j < 15 ? j + 1 : 15];
+    const double hk = s_half[j < 15 ? j : 14];
+    const uint32_t lut = s_lut[lane];
+    bool ok = true;
+    uint32_t bad_any = 0;
+    for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(smem_u32(&bars[c]), 0, &abort_flag));
+        if (!ok) {
+            abort_flag = 1;
+            break;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int bl = 64 * c + 2 * (warp + 8 * i) + half;   // block within the group
+            const bool valid = bl < nblk;
+            float w[4] = {0.f, 0.f, 0.f, 0.f};
+            if (valid) {
+                const float4 v = *reinterpret_cast<const float4 *>(qw + bl * 64 + 4 * j);
+                w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+            }
+            // max |w| on the bit patterns: NaN and Inf sort above every finite value
+            uint32_t m = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m = max(m, __float_as_uint(w[k]) & 0x7fffffffu);
+            const uint32_t m0 = __reduce_max_sync(0xffffffffu, half ? 0u : m);
+            const uint32_t m1 = __reduce_max_sync(0xffffffffu, half ? m : 0u);
+            const uint32_t ab = half ? m1 : m0;
+            const float a = __uint_as_float(ab);
+            const bool bad = ab >= 0x7f800000u;
+            // tau_j: the smallest fp32 above the exact midpoint h_j * a
+            float tau;
+            if (kExactHalf)
+                tau = next_up(__double2float_rd(__dmul_rn(hk, (double)a)));
+            else
+                tau = exact_threshold(c_lo, c_hi, a);
+            if (j == 15) tau = __uint_as_float(0x7f800000u);
+            const bool fast = ab >= 0x0d800000u && ab <= 0x71800000u;   // 2^-100 <= a <= 2^100
+            uint32_t qv[4];
+            if (__all_sync(0xffffffffu, fast || !valid)) {
+                const float kr = __fmul_rn(kBinK, rcp_approx(a));   // K / a, relative error < 2^-22
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float y = fmaf(w[k], kr, kBinC);
+                    const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
+                    const float t = __shfl_sync(0xffffffffu, tau, (int)jt, 16);
+                    qv[k] = jt + (w[k] >= t ? 1u : 0u);
+                }
+            } else {
+                float t[15];
+#pragma unroll
+                for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k, 16);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[k], t);
+            }
+            if (valid) {
+                // weights 4j..4j+3 -> bytes 2j, 2j+1; element 2i in the high nibble
+                const uint32_t v = qv[1] | (qv[0] << 4) | (qv[3] << 8) | (qv[2] << 12);
+                *reinterpret_cast<uint16_t *>(packed + (b0 + bl) * 32 + 2 * j) = (uint16_t)v;
+                if (j == 0) {
+                    s_a[bl] = a;
+                    if (!dq) absmax[b0 + bl] = a;
+                    bad_any |= bad;
+                }
+            }
+        }
+    }
+    if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
+    if (!ok && lane == 0 && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
+
+    if (dq) {
+        __syncthreads();
+        const bool valid = threadIdx.x < nblk;
+        const float a = s_a[threadIdx.x];
+        float mx = a;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) warp_max[warp] = mx;
+        __syncthreads();
+        float gm = warp_max[0];
+#pragma unroll
+        for (int i = 1; i < kQfThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
+        const float f = __fdiv_rn(gm, 255.f);
+        if (threadIdx.x == 0) steps[blockIdx.x] = f;
+        if (valid) {
+            codes[b0 + threadIdx.x] = (uint8_t)dq_code(a, f);
+        }
+    }
+}
+
 // Dequantize: 4 threads per block; thread i of the 4 owns packed bytes
 // [4i, 4i+4) and [16+4i, 16+4i+4) of its block, i.e. output elements
 // [8i, 8i+8) and [32+8i, 32+8i+8), so each group of 4 threads reads 16
@@ -192,10 +385,73 @@ k_nf4_dequantize(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t nb, Co
 
 }  // namespace
 
+// T[bin] of the fast kernel for this codebook, or false when some bin,
+// widened by the margin, holds two thresholds (levels closer than about
+// 1/K apart): bin i holds every u with RN(K u + 16) = i.  The margin 2^-18
+// bounds both the error of w * RN(1/a) against w/a (< 2^-22 for |w| <= a) and
+// the distance of an exact threshold tau_k / a from its midpoint m_k.
+bool make_quant_bins(const Codebook &cb, QuantBins *out) {
+    const double K = (double)kBinK, margin = std::ldexp(1.0, -18);
+    double m[15];
+    for (int k = 0; k < 15; ++k) m[k] = ((double)cb.c[k] + (double)cb.c[k + 1]) * 0.5;
+    QuantBins qb{};
+    for (int i = 0; i < 32; ++i) {
+        const double lo = (i - 16.5) / K - margin, hi = (i - 15.5) / K + margin;
+        int below = 0, inside = 0;
+        for (int k = 0; k < 15; ++k) {
+            if (m[k] + margin < lo)
+                ++below;
+            else if (m[k] - margin <= hi)
+                ++inside;
+        }
+        if (inside > 1) return false;
+        qb.nib[i >> 3] |= (uint32_t)below << (4 * (i & 7));
+    }
+    *out = qb;
+    return true;
+}
+
+// Fills bins->half; true when every (c_k + c_{k+1}) / 2 is exact in fp64 and
+// has at most 29 significant bits, so that its product with any fp32 scale
+// is exact in fp64.
+bool make_exact_halves(const Codebook &cb, QuantBins *bins) {
+    bool ok = true;
+    for (int k = 0; k < 15; ++k) {
+        const double x = cb.c[k], y = cb.c[k + 1];
+        const double s = x + y;
+        const double bb = s - x;
+        const double err = (x - (s - bb)) + (y - bb);   // TwoSum: s + err == x + y
+        const double h = s * 0.5;
+        bins->half[k] = h;
+        if (err != 0.0) ok = false;
+        if (h != 0.0) {
+            int e;
+            const double m = std::frexp(std::fabs(h), &e);          // m in [0.5, 1)
+            const uint64_t bits = (uint64_t)std::ldexp(m, 53);      // exact: 53-bit integer
+            const int tz = __builtin_ctzll(bits);
+            if (53 - tz > 29) ok = false;
+        }
+    }
+    return ok;
+}
+
 int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
                         uint32_t *d_status, cudaStream_t st) {
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
+    QuantBins bins;
+    if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && make_quant_bins(cb, &bins)) {
+        const bool exact_half = make_exact_halves(cb, &bins);
+        auto kern = exact_half ? k_nf4_quantize_fast<true> : k_nf4_quantize_fast<false>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQfSmem);
+        prof_begin(kProfQuant, st);
+        kern<<<(unsigned)((nb + 255) / 256), kQfThreads, kQfSmem, st>>>(
+            W, nb, cb, bins, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
+            d_status);
+        prof_end(kProfQuant, st);
+        QLORA_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
     const int64_t grid = (nb + kQuantThreads - 1) / kQuantThreads;
     // the weight viewed as [nb rows][64 fp32], loaded 32 columns x 256 rows at a time
     CUtensorMap tW;

@@ -92,10 +92,16 @@ def test_custom_codebooks(orc, qlib):
                         .5, .625, .75, 1], dtype=np.float32)
     tiny = np.array([-1, -.9, -.8, -.7, -.6, -.5, -2.0 ** -60, 0, .5, .6, .7, .75, .8, .85, .9, 1],
                     dtype=np.float32)
-    for cb in (uniform, tiny, orc.nf4_codebook(1 - 1 / 32)):
-        # exact ties on the uniform table's midpoints
+    # levels at least 0.1 apart: thresholds far enough apart for the bin-table kernel
+    wide = np.array([-1, -.85, -.7, -.55, -.4, -.25, -.1, 0, .1, .25, .4, .55, .7, .8, .9, 1],
+                    dtype=np.float32)
+    for cb in (uniform, tiny, orc.nf4_codebook(1 - 1 / 32), wide):
+        # exact ties on the uniform table's midpoints, and on this table's own
         W2 = W.copy()
         W2[0, :16] = (np.concatenate([[1.0], (uniform[:-1] + uniform[1:]) / 2])).astype(np.float32)
+        W2[1, :16] = (np.concatenate([[1.0], (cb[:-1] + cb[1:]) / 2])).astype(np.float32)
+        W2[1, 16:31] = np.nextafter(W2[1, 1:16], np.float32(-np.inf))
+        W2[1, 31:46] = np.nextafter(W2[1, 1:16], np.float32(np.inf))
         _check_same(orc, qlib, W2, True, cb)
 
 
@@ -105,12 +111,42 @@ def test_special_blocks_and_status(orc, qlib):
     W[2, 0], W[2, 1] = 0.5, -0.5
     W[3, 64:] = 1e-42                       # subnormal block
     _check_same(orc, qlib, W, True)
+    # scales outside [2^-100, 2^100] take the search path of the fast kernel
+    rng = np.random.default_rng(5)
+    W2 = (rng.standard_normal((4, 256)) * 0.05).astype(np.float32)
+    W2[0, :64] *= np.float32(2.0 ** 110)
+    W2[1, 64:128] *= np.float32(2.0 ** -110)
+    W2[2, 128:192] *= np.float32(2.0 ** 100)
+    W2[3, 192:] *= np.float32(2.0 ** -96)
+    _check_same(orc, qlib, W2, False)
+    _check_same(orc, qlib, W2, True)
     W[0, 5] = np.nan
     _, st = _gpu_quant(qlib, W, True)
     assert st == 1
     W[0, 5] = np.inf
     _, st = _gpu_quant(qlib, W, False)
     assert st == 1
+
+
+def test_double_quant_code_ties(orc, qlib):
+    """Block scales on and next to the code midpoints: group max 255/16 makes
+    the step exactly 1/16, so a = (k + 1/2)/16 is a tie that rounds to even."""
+    rng = np.random.default_rng(17)
+    nb = 256
+    a = np.empty(nb, np.float32)
+    a[0] = 255 / 16
+    k = np.arange(1, nb) % 255
+    ties = ((k + 0.5) / 16).astype(np.float32)
+    a[1:] = ties
+    a[100:140] = np.nextafter(ties[99:139], np.float32(np.inf))
+    a[140:180] = np.nextafter(ties[139:179], np.float32(-np.inf))
+    blocks = (rng.uniform(-1, 1, (nb, 64)) * a[:, None] * 0.9).astype(np.float32)
+    blocks[:, 7] = -a
+    W = blocks.reshape(4, 64 * 64)
+    _check_same(orc, qlib, W, True)
+    ref = orc.quantize(W, orc.nf4_codebook(), True)
+    assert ref.steps[0] == np.float32(1 / 16)
+    assert list(ref.codes[1:4]) == [2, 2, 4] and ref.codes[255] == 0   # 1.5, 2.5, 3.5, 0.5
 
 
 def test_empty_weight(qlib):
