@@ -66,6 +66,8 @@ def _L():
         lib.orc_forward.restype = None
         lib.orc_forward.argtypes = [P, i64, i64, i64, P, P, P, ctypes.c_int, ctypes.c_double,
                                     ctypes.c_int, P, P]
+        lib.orc_merge.restype = None
+        lib.orc_merge.argtypes = [i64, i64, P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_int, P]
         lib.orc_grad_G.restype = None
         lib.orc_grad_G.argtypes = [P, i64, i64, P, ctypes.c_int, P]
         lib.orc_backward_dx.restype = None
@@ -174,6 +176,18 @@ def forward(X, Wt, A, B, r: int, alpha: float, pool_group: int = 1):
     _L().orc_forward(_p(X), M, Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha), pool_group,
                      _p(Y), _p(T))
     return Y, T
+
+
+def merge(Wt, A, B, r: int, alpha: float, pool_group: int = 1) -> np.ndarray:
+    """W_eff fp64 [Dout, Din] = dequantized Wt + (alpha/r) (A B) in the stored
+    orientation; pooled: (alpha/r)/g (A_p B) shared by each group's inputs."""
+    Wt = _c(Wt, np.uint16)
+    A = _c(A, np.uint16)
+    B = _c(B, np.uint16)
+    Dout, Din = Wt.shape
+    out = np.zeros((Dout, Din), dtype=np.float64)
+    _L().orc_merge(Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha), pool_group, _p(out))
+    return out
 
 
 def grad_G(dY, B, r: int) -> np.ndarray:

@@ -433,6 +433,28 @@ void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
 }
 
 /* Threads the OpenMP runtime will use for the parallel loops above. */
+/* Adapter merge for inference: W_eff = dequant(W4) + s * (A . B), written in
+ * the stored orientation [Dout][Din]:
+ *   W_eff[n][k] = Wt[n][k] + s * sum_j A[k][j] B[j][n]               (g = 1)
+ *   W_eff[n][k] = Wt[n][k] + (s/g) * sum_j A_p[k/g][j] B[j][n]       (pooled)
+ * ([BLOG] section 2, W_eff = dequant(W4) + (alpha/r) A B; [CSDN] 12.10, merging
+ * the adapter into the weight for deployment; [BLOG] section 5, every input of
+ * a group shares the update (A_p B)/g.)  The pooled form is the one for which
+ * x . W_eff^T equals the layer's forward, since pool(x) averages a group.
+ * Wt is the bf16 dequantized weight; the result is exact fp64 arithmetic on it. */
+void orc_merge(int64_t Din, int64_t Dout, const uint16_t *Wt, const uint16_t *A,
+               const uint16_t *B, int r, double alpha, int g, double *out) {
+    const double s = alpha / (double)r;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < Dout; ++n)
+        for (int64_t k = 0; k < Din; ++k) {
+            double ad = 0.0;
+            for (int j = 0; j < r; ++j)
+                ad += bf16_to_double(A[(k / g) * r + j]) * bf16_to_double(B[(int64_t)j * Dout + n]);
+            out[n * Din + k] = bf16_to_double(Wt[n * Din + k]) + (s / (double)g) * ad;
+        }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);
