@@ -11,12 +11,17 @@ namespace qlora {
 int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
                         uint32_t *d_status, cudaStream_t st);
 int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *out, cudaStream_t st);
+// merge.cu
+int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, const uint16_t *B,
+                 int r, int gp, float s, uint16_t *W_out, cudaStream_t st);
 // gemv.cu
 size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout);
 size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout);
+size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r);
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, uint32_t *d_status, cudaStream_t st);
+                    float *partial, uint32_t *d_status, cudaStream_t st,
+                    const uint16_t *Aad = nullptr, float *Tpart = nullptr, float *T_out = nullptr);
 int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *G, const uint16_t *Al, int r, int pool, float s, uint16_t *dX,
                     float *partial, cudaStream_t st);
@@ -237,7 +242,7 @@ Prod prod_dB(const Dims &d, const uint16_t *dY, const uint16_t *Tsplit) {
 // Workspace pieces.  The same function sizes (base == nullptr) and carves.
 struct FwdWs {
     uint16_t *Apad, *ph, *pl, *sT, *Wdeq;
-    float *T32, *Tpart, *gemv_part;
+    float *T32, *Tpart, *gemv_part, *gemv_tpart;
 };
 struct BwdWs {
     uint16_t *Apad, *ph, *pl, *sG, *Gsplit, *Tsplit, *Aext, *Wdeq;
@@ -256,6 +261,7 @@ size_t layout_fwd(const Dims &d, bool have_tsave, void *base, FwdWs *w) {
     x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0), d.mma_large));
     if (d.small) {
         x.gemv_part = b.take<float>(gemv_fwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
+        if (d.g == 1) x.gemv_tpart = b.take<float>(gemv_fwd_tpart_floats((int)d.M, d.Din, d.r));
     } else {
         x.sT = b.take<uint16_t>(d.M * d.rp64);
         if (d.mma_large) x.Wdeq = b.take<uint16_t>(d.Dout * d.Din);
@@ -385,6 +391,19 @@ int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_
     return launch_nf4_dequantize(*q, to_cb(codebook), W_out, (cudaStream_t)stream);
 }
 
+int qlora_merge(const nf4_weight_t *q, const float codebook[16], const uint16_t *A,
+                const uint16_t *B, int32_t r, float alpha, int32_t pool_group, uint16_t *W_out,
+                void *stream) {
+    RC(check_weight(q, false));
+    RC(check_codebook(codebook, nullptr));
+    if (r < 1 || r > QLORA_MAX_RANK || !std::isfinite(alpha)) return QLORA_EINVAL;
+    if (pool_group != 1 && pool_group != 64) return QLORA_EINVAL;
+    if (q->rows * q->cols == 0) return QLORA_OK;
+    if (!A || !B || !W_out || !aligned16(W_out)) return QLORA_EINVAL;
+    return launch_merge(*q, to_cb(codebook), A, B, r, pool_group, alpha / (float)r, W_out,
+                        (cudaStream_t)stream);
+}
+
 size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t pool_group,
                             int32_t which) {
     static const float kCb[16] = {-1, -.875f, -.75f, -.625f, -.5f, -.375f, -.25f, 0,
@@ -414,6 +433,13 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
     const float s = alpha / (float)r;
     float *T32 = T_save ? T_save : w.T32;
 
+    if (d.small && d.g == 1) {
+        // one streamed kernel computes the base product and the adapter-down
+        // partials, one finalize reduces both; else the general sequence
+        const int rc = launch_gemv_fwd(X, (int)M, *q, cb, nullptr, B, r, s, Y, w.gemv_part, d_status,
+                                       st, A, w.gemv_tpart, T32);
+        if (rc != QLORA_EUNSUPPORTED) return rc;
+    }
     if (d.g > 1) RC(run_pool(d, X, w.ph, w.pl, st));
     RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT,
                         d_status, st));

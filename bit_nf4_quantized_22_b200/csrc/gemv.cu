@@ -179,38 +179,64 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
 
 // ------------------------------------------------------------------ forward, streamed
 // Persistent variant: one CTA per SM walks a contiguous range of
-// (input-slice, 128-row) tiles.  A producer warp streams each tile's packed
-// weights (128 rows x 512 bytes, four 128-byte-swizzled TMA boxes) and its
-// scale codes into a two-stage shared-memory ring, so ~70 KB per SM are in
-// flight independently of registers; eight compute warps decode from shared
-// memory exactly as k_gemv_fwd does from registers.  Needs the scale rows to
-// be TMA-tileable: Din/64 a multiple of 16 (codes) or of 4 (fp32 absmax).
+// (input-slice, 128-row) tiles, slices of 1024 inputs.  A producer warp
+// streams each tile as two half-tiles (128 rows x 256 packed bytes, two
+// 128-byte-swizzled TMA boxes, plus the rows' scale codes) through a
+// three-stage shared-memory ring, so loads run ahead independently of
+// registers.
+//
+// Sixteen compute warps: warps w and w + 8 own the same 16 rows and take
+// the even and the odd 64-blocks of each half-tile, four blocks each; the
+// two warps' sums meet in shared memory once per tile (even + odd).
+//
+// Decode: the byte -> bf16-pair table has one 256-byte row per byte value,
+// lane l's copy at +4l, so the shared address of a lookup is exactly
+// (byte << 8) | 4l: one byte permute builds it from the packed word and a
+// per-lane constant.  The x slice rows are 2056 bytes apart (= 8 mod 128),
+// which puts the 32 lanes' 8-byte fragment loads on distinct bank pairs.
+//
+// With an adapter (Aad), ceil(r/16) tiles of slice z, spread over its row
+// tiles, also compute the adapter-down partials of one rank tile each,
+// Tpart[z][b][m][j] = sum over the 64 inputs k of block b of x[m][k] A[k][j],
+// warp w taking block w, as MMAs with the 16 ranks on the M side (A^T
+// gathered from the row-major A) and the tokens on the N side.  Needs the scale rows to be TMA-tileable: Din/64 a
+// multiple of 16 (codes) or of 4 (fp32 absmax).
 constexpr int kStRows = 128, kStBlocks = 16;              // tile: 128 rows x 1024 inputs
-constexpr int kStPacked = kStRows * kStBlocks * 32;       // 64 KB
-constexpr int kStStage = kStPacked + 8192;                // + scale tile (codes 2 KB / fp32 8 KB)
-constexpr int kStStages = 2;
-constexpr int kStThreads = (kGemvWarps + 1) * 32;
-constexpr int kStLut = 256 * 32 * 4;
-constexpr int kStX = (16 * (kFwdKS + 8) * 2 + 1023) / 1024 * 1024;
-constexpr int kStSmem = kStLut + kStX + kStStages * kStStage + 1024 + 256;
+constexpr int kStHalf = kStRows * 8 * 32;                 // half-tile packed bytes: 32 KB
+constexpr int kStStage = kStHalf + 4096;                  // + scales (codes 2 KB / fp32 4 KB)
+constexpr int kStStages = 3;
+constexpr int kStCompute = 16;                            // compute warps
+static_assert(kStCompute == kStBlocks, "the adapter-down work gives each warp one block");
+constexpr int kStThreads = (kStCompute + 1) * 32;
+constexpr int kStLut = 256 * 256;                         // 64 KB, must start the buffer
+constexpr int kStXPitch = kFwdKS + 4;                     // bf16 elements per x row
+constexpr int kStX = (16 * kStXPitch * 2 + 1023) / 1024 * 1024;
+constexpr int kStRed = 2 * 8 * 32 * 8 * 4;                // two buffers of the odd warps' sums
+constexpr int kStSmem = kStLut + kStX + kStStages * kStStage + kStRed + 1024 + 256;
 
 template <int NT>
 __global__ void __launch_bounds__(kStThreads, 1)
 k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmC,
                   const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout, ScaleSrc sc,
                   Codebook cb, int ntr, int ntiles, float *__restrict__ partial,
+                  const uint16_t *__restrict__ Aad, int r, float *__restrict__ Tpart,
                   uint32_t *__restrict__ status) {
     extern __shared__ __align__(1024) uint8_t ssm[];
     const uint32_t raw = smem_u32(ssm);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = ssm + (base - raw);
-    uint32_t *lut = reinterpret_cast<uint32_t *>(gbase);
-    uint16_t(*sx)[kFwdKS + 8] = reinterpret_cast<uint16_t(*)[kFwdKS + 8]>(gbase + kStLut);
-    const uint32_t ring = base + kStLut + kStX;          // 1 KB aligned, as 128-byte swizzling needs
-    const uint32_t bar0 = ring + kStStages * kStStage;
+    const uint8_t *lutb = gbase;                                  // [256][256 B]
+    uint16_t(*sx)[kStXPitch] = reinterpret_cast<uint16_t(*)[kStXPitch]>(gbase + kStLut);
+    const uint32_t ring = base + kStLut + kStX;                   // 1 KB aligned
+    uint8_t *gring = gbase + kStLut + kStX;
+    float *red = reinterpret_cast<float *>(gring + kStStages * kStStage);   // [2][8][32][8]
+    const uint32_t bar0 = ring + kStStages * kStStage + kStRed;
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (kStStages + s); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + (bar0 - base) + 64);
+    // the codebook goes through shared memory: indexing the parameter array
+    // by a thread-dependent value would copy it to the stack
+    float *cbs = reinterpret_cast<float *>(gbase + (bar0 - base) + 128);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -219,68 +245,78 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
     const int t1 = (int)((int64_t)(blockIdx.x + 1) * ntiles / G);
     const int64_t nbr = Din / 64;
 
-    // the codebook goes through shared memory: indexing the parameter array
-    // by a thread-dependent value would copy it to the stack
-    float *cbs = reinterpret_cast<float *>(gbase + (bar0 - base) + 128);
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
         for (int s = 0; s < kStStages; ++s) {
             tc::mbar_init(full(s), 1);
-            tc::mbar_init(empty(s), kGemvWarps);
+            tc::mbar_init(empty(s), kStCompute);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
         tc::fence_proxy_async();
     }
     __syncthreads();
-    if (threadIdx.x < 256) {   // pair table, one entry per thread (see k_gemv_fwd)
+    if (threadIdx.x < 256) {   // table row e: 32 copies of (c[e >> 4], c[e & 15]) in bf16
         const int e = threadIdx.x;
         const uint32_t v = bf16x2_bits(cbs[e >> 4], cbs[e & 15]);
-        uint4 *row = reinterpret_cast<uint4 *>(lut + e * 32);
+        uint4 *row = reinterpret_cast<uint4 *>(gbase + e * 256);
         const uint4 vv = make_uint4(v, v, v, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) row[(i + lane) & 7] = vv;
     }
-    for (int i = threadIdx.x; i < (16 - M) * (kFwdKS / 8); i += blockDim.x) {
-        const int m = M + i / (kFwdKS / 8), kc = (i % (kFwdKS / 8)) * 8;
-        *reinterpret_cast<uint4 *>(&sx[m][kc]) = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < (16 - M) * (kFwdKS / 4); i += blockDim.x) {
+        const int m = M + i / (kFwdKS / 4), kc = (i % (kFwdKS / 4)) * 4;
+        *reinterpret_cast<uint2 *>(&sx[m][kc]) = make_uint2(0u, 0u);
     }
     __syncthreads();
     bool ok = true;
+    auto halves = [&](int z) {   // half-tiles holding data in slice z
+        const int64_t nb = (Din - (int64_t)z * kFwdKS) / 64;
+        return nb > 8 ? 2 : 1;
+    };
 
-    if (warp == kGemvWarps) {
+    if (warp == kStCompute) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            const uint32_t cbytes = sc.dq ? kStRows * 16 : kStRows * 16 * 4;
-            for (int i = 0, tt = t0; tt < t1 && ok; ++i, ++tt) {
-                const int s = i % kStStages;
-                if (i >= kStStages) ok = tc::mbar_wait(empty(s), ((i / kStStages) & 1) ^ 1, abort_flag);
-                if (!ok) break;
+            const uint32_t cbytes = sc.dq ? kStRows * 16 : kStRows * 8 * 4;
+            int hi = 0;
+            for (int tt = t0; tt < t1 && ok; ++tt) {
                 const int z = tt / ntr, rt = tt % ntr;
-                const uint32_t st = ring + s * kStStage;
-                tc::mbar_expect_tx(full(s), kStPacked + cbytes);
+                const int nh = halves(z);
+                for (int h = 0; h < nh && ok; ++h, ++hi) {
+                    const int s = hi % kStStages;
+                    if (hi >= kStStages) ok = tc::mbar_wait(empty(s), ((hi / kStStages) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    const uint32_t st = ring + s * kStStage;
+                    tc::mbar_expect_tx(full(s), kStHalf + cbytes);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    tc::tma_load_2d(st + q * (kStRows * 128), &tmP, z * (kFwdKS / 2) + 128 * q,
-                                    rt * kStRows, full(s));
-                tc::tma_load_2d(st + kStPacked, &tmC, z * kStBlocks, rt * kStRows, full(s));
+                    for (int q = 0; q < 2; ++q)
+                        tc::tma_load_2d(st + q * (kStRows * 128), &tmP,
+                                        z * (kFwdKS / 2) + h * 256 + 128 * q, rt * kStRows, full(s));
+                    if (sc.dq)   // the whole slice's 16 codes per row, read by both halves
+                        tc::tma_load_2d(st + kStHalf, &tmC, z * kStBlocks, rt * kStRows, full(s));
+                    else
+                        tc::tma_load_2d(st + kStHalf, &tmC, z * kStBlocks + 8 * h, rt * kStRows, full(s));
+                }
             }
             if (!ok) *abort_flag = 1;
         }
     } else {
         // ---------------------------------------------------------- compute warps
-        const uint32_t *lut_lane = lut + lane;
-        auto lookup = [&](uint32_t word, int i) -> uint32_t {
-            return lut_lane[__byte_perm(word, 0u, 0x4440u + i) << 5];
+        // lookup address = (byte << 8) | 4 * lane, from one permute
+        const uint32_t lanebits = 4u * lane;
+        auto lookup = [&](uint32_t word, int k) -> uint32_t {
+            const uint32_t off = __byte_perm(word, lanebits, 0x5504u | ((uint32_t)k << 4));
+            return *reinterpret_cast<const uint32_t *>(lutb + off);
         };
-        const int rl = warp * 16 + g;                  // rows rl and rl + 8 of the tile
+        const int rl = (warp & 7) * 16 + g;            // rows rl and rl + 8 of the tile
+        const int bpar = warp >> 3;                    // this warp's blocks: b = bpar mod 2
         // Every compute warp walks the same tiles and meets the same named
         // barriers; after a failed wait a warp keeps walking (skipping the
         // work) so that no other warp is left at a barrier.
-        int prev_z = -1;
-        for (int i = 0, tt = t0; tt < t1; ++i, ++tt) {
-            const int s = i % kStStages;
+        int prev_z = -1, hi = 0, rpar = 0;
+        for (int tt = t0; tt < t1; ++tt, rpar ^= 1) {
             const int z = tt / ntr, rt = tt % ntr;
             const int64_t k0 = (int64_t)z * kFwdKS;
             const int64_t row0 = (int64_t)rt * kStRows + rl;
@@ -293,77 +329,150 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
                 if (ok1) step1 = __ldg(sc.step + (((row0 + 8) * nbr + z * kStBlocks) >> 8));
             }
             if (z != prev_z) {                         // stage x[:M, k0 : k0 + 1024]
-                asm volatile("bar.sync 1, %0;\n" ::"n"(kGemvWarps * 32));
-                for (int j = threadIdx.x; j < M * (kFwdKS / 8); j += kGemvWarps * 32) {
-                    const int m = j / (kFwdKS / 8), kc = (j % (kFwdKS / 8)) * 8;
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (k0 + kc < Din) v = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)m * Din + k0 + kc));
-                    *reinterpret_cast<uint4 *>(&sx[m][kc]) = v;
+                asm volatile("bar.sync 1, %0;\n" ::"n"(kStCompute * 32));
+                for (int j = threadIdx.x; j < M * (kFwdKS / 4); j += kStCompute * 32) {
+                    const int m = j / (kFwdKS / 4), kc = (j % (kFwdKS / 4)) * 4;
+                    uint2 v = make_uint2(0u, 0u);
+                    if (k0 + kc < Din) v = __ldg(reinterpret_cast<const uint2 *>(X + (int64_t)m * Din + k0 + kc));
+                    *reinterpret_cast<uint2 *>(&sx[m][kc]) = v;
                 }
-                asm volatile("bar.sync 1, %0;\n" ::"n"(kGemvWarps * 32));
+                asm volatile("bar.sync 1, %0;\n" ::"n"(kStCompute * 32));
                 prev_z = z;
             }
-            if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (i / kStStages) & 1, abort_flag));
-            if (!ok) {
-                *abort_flag = 1;
-                continue;
-            }
-            const uint32_t st = ring + s * kStStage;
             const int nblk = (int)((Din - k0) / 64 < kStBlocks ? (Din - k0) / 64 : kStBlocks);
+            const int nh = halves(z);
             float acc[NT][4];
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
-#pragma unroll 4
-            for (int b = 0; b < kStBlocks; ++b) {
-                if (b >= nblk) break;
-                // packed: box q = b/4 holds rows x 128 B; this lane's 8 bytes of
-                // block b are 16-byte chunk 2(b%4) + t/2 (swizzled by row), half t%2
-                const uint32_t chunk = 2 * (b & 3) + (t >> 1);
-                const uint32_t boff = st + (b >> 2) * (kStRows * 128) + ((chunk ^ (rl & 7)) << 4) + 8 * (t & 1);
-                uint2 w0, w1;
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0.x), "=r"(w0.y) : "r"(boff + rl * 128) : "memory");
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w1.x), "=r"(w1.y) : "r"(boff + (rl + 8) * 128) : "memory");
-                float a0 = 0.f, a1 = 0.f;
-                if (sc.dq) {
-                    const uint8_t *cs = gbase + (st - base) + kStPacked;
-                    a0 = __fmul_rn((float)cs[rl * 16 + b], step0);
-                    a1 = __fmul_rn((float)cs[(rl + 8) * 16 + b], step1);
-                } else {
-                    const float *as = reinterpret_cast<const float *>(gbase + (st - base) + kStPacked);
-                    a0 = as[rl * 16 + b];
-                    a1 = as[(rl + 8) * 16 + b];
+            for (int h = 0; h < nh; ++h, ++hi) {
+                const int s = hi % kStStages;
+                if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (hi / kStStages) & 1, abort_flag));
+                if (!ok) {
+                    *abort_flag = 1;
+                    continue;
                 }
-                float tmp[NT][4];
+                const uint8_t *stg = gring + s * kStStage;
+                const int hb = nblk - 8 * h < 8 ? nblk - 8 * h : 8;   // blocks in this half
+                auto block = [&](int bh) {
+                    // packed: box bh/4 holds rows x 128 B; this lane's 8 bytes of
+                    // block bh are 16-byte chunk 2(bh%4) + t/2 (swizzled by row), half t%2
+                    const int chunk = 2 * (bh & 3) + (t >> 1);
+                    const uint8_t *pb = stg + (bh >> 2) * (kStRows * 128) + ((chunk ^ (rl & 7)) << 4) + 8 * (t & 1);
+                    const uint2 w0 = *reinterpret_cast<const uint2 *>(pb + rl * 128);
+                    const uint2 w1 = *reinterpret_cast<const uint2 *>(pb + (rl + 8) * 128);
+                    float a0, a1;
+                    if (sc.dq) {
+                        const uint8_t *cs = stg + kStHalf;
+                        a0 = __fmul_rn((float)cs[rl * 16 + 8 * h + bh], step0);
+                        a1 = __fmul_rn((float)cs[(rl + 8) * 16 + 8 * h + bh], step1);
+                    } else {
+                        const float *as = reinterpret_cast<const float *>(stg + kStHalf);
+                        a0 = as[rl * 8 + bh];
+                        a1 = as[(rl + 8) * 8 + bh];
+                    }
+                    float tmp[NT][4];
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
+                    for (int n = 0; n < NT; ++n)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) tmp[n][e] = 0.f;
+                        for (int e = 0; e < 4; ++e) tmp[n][e] = 0.f;
+                    const int kx = 64 * (8 * h + bh) + 16 * t;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t x0 = q < 2 ? w0.x : w0.y;
-                    const uint32_t x1 = q < 2 ? w1.x : w1.y;
-                    const int i0 = (2 * q) & 3;
-                    const uint32_t a[4] = {lookup(x0, i0), lookup(x1, i0), lookup(x0, i0 + 1),
-                                           lookup(x1, i0 + 1)};
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t x0 = q < 2 ? w0.x : w0.y;
+                        const uint32_t x1 = q < 2 ? w1.x : w1.y;
+                        const int i0 = (2 * q) & 3;
+                        const uint32_t a[4] = {lookup(x0, i0), lookup(x1, i0), lookup(x0, i0 + 1),
+                                               lookup(x1, i0 + 1)};
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kx + 4 * q]);
+                            const uint32_t bb[2] = {xv.x, xv.y};
+                            mma_bf16_16816(tmp[n], a, bb);
+                        }
+                    }
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][64 * b + 16 * t + 4 * q]);
-                        const uint32_t bb[2] = {xv.x, xv.y};
-                        mma_bf16_16816(tmp[n], a, bb);
+                        acc[n][0] = fmaf(a0, tmp[n][0], acc[n][0]);
+                        acc[n][1] = fmaf(a0, tmp[n][1], acc[n][1]);
+                        acc[n][2] = fmaf(a1, tmp[n][2], acc[n][2]);
+                        acc[n][3] = fmaf(a1, tmp[n][3], acc[n][3]);
                     }
-                }
+                };
+                // this warp's blocks of the half: bh = bpar, bpar + 2, ...
+                if (hb == 8) {
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    acc[n][0] = fmaf(a0, tmp[n][0], acc[n][0]);
-                    acc[n][1] = fmaf(a0, tmp[n][1], acc[n][1]);
-                    acc[n][2] = fmaf(a1, tmp[n][2], acc[n][2]);
-                    acc[n][3] = fmaf(a1, tmp[n][3], acc[n][3]);
+                    for (int i = 0; i < 4; ++i) block(2 * i + bpar);
+                } else {
+                    for (int bh = bpar; bh < hb; bh += 2) block(bh);
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(empty(s));
+            }
+            if (Aad && ok) {
+                // adapter down of slice z: rank tile j16 goes to tile rt = j16 * step
+                // (spread over the slice's row tiles, so over different CTAs), or
+                // with fewer row tiles than rank tiles to rt = j16 mod ntr; warp w
+                // takes block w (the 16 warps cover the slice's 16 blocks; blocks
+                // past a ragged end write zeros)
+                const int ntj = (r + 15) / 16;
+                const int step = ntr >= ntj ? ntr / ntj : 1;
+                for (int j16 = rt / step; rt % step == 0 && j16 < ntj; j16 += ntr) {
+                    const int b = warp;
+                    const int ja = 16 * j16 + g, jb = ja + 8;
+                    float ta[NT][4];
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) ta[n][e] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (b >= nblk) break;
+                        const int kk = 64 * b + 16 * t + 4 * q;    // the x fragment's inputs kk..kk+3
+                        const uint16_t *ak = Aad + (k0 + kk) * r;
+                        uint32_t v[4][2];   // [input kk + i][rank ja / jb]
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            v[i][0] = ja < r ? __ldg(ak + i * r + ja) : 0u;
+                            v[i][1] = jb < r ? __ldg(ak + i * r + jb) : 0u;
+                        }
+                        const uint32_t a[4] = {v[0][0] | (v[1][0] << 16), v[0][1] | (v[1][1] << 16),
+                                               v[2][0] | (v[3][0] << 16), v[2][1] | (v[3][1] << 16)};
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kk]);
+                            const uint32_t bb[2] = {xv.x, xv.y};
+                            mma_bf16_16816(ta[n], a, bb);
+                        }
+                    }
+                    // ta[n]: (rank ja, tokens 8n + 2t, +1) and (rank jb, same tokens)
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * n + 2 * t + (e & 1);
+                            const int j = e < 2 ? ja : jb;
+                            if (m < M && j < r)
+                                Tpart[(((int64_t)z * kStBlocks + b) * M + m) * r + j] = ta[n][e];
+                        }
                 }
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(empty(s));
+            // odd-block warps hand their sums to the even-block warps (buffer
+            // rpar; the barrier of the next tile orders its reuse)
+            float *rb = red + ((rpar * 8 + (warp & 7)) * 32 + lane) * 8;
+            if (bpar) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    *reinterpret_cast<float4 *>(rb + 4 * n) = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
+            }
+            asm volatile("bar.sync 2, %0;\n" ::"n"(kStCompute * 32));
+            if (!ok || bpar) continue;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const float4 o = *reinterpret_cast<const float4 *>(rb + 4 * n);
+                acc[n][0] += o.x, acc[n][1] += o.y, acc[n][2] += o.z, acc[n][3] += o.w;
+            }
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -377,6 +486,47 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
     if (!ok && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
     __syncwarp();
     __syncthreads();
+}
+
+// Forward finalize with the adapter-down partials of the streamed kernel:
+// T[m, j] = sum over (slice, block) of Tpart, once per CTA in a fixed order
+// (and written out by the CTAs of the first column block), then
+// y[m, n] = sum_split partial + s * sum_j T[m, j] B[j, n].  grid (ceil(Dout/256), M).
+__global__ void __launch_bounds__(256)
+k_gemv_fwd_finalize_fused(const float *__restrict__ partial, int nsplit, int M, int64_t Dout,
+                          const float *__restrict__ Tpart, int r, const uint16_t *__restrict__ Bl,
+                          float s, uint16_t *__restrict__ Y, float *__restrict__ T_out) {
+    __shared__ float Ts[QLORA_MAX_RANK];
+    __shared__ float Tg[256];
+    const int m = blockIdx.y;
+    // thread i sums the partials p = i / r, i / r + G, ... of rank i % r
+    // (G = 256 / r groups, independent loads); the G group sums are then
+    // added in group order
+    const int P = kStBlocks * nsplit;
+    const int G = r <= 256 ? 256 / r : 1;
+    const int jr = threadIdx.x % r, grp = threadIdx.x / r;
+    if (grp < G) {
+        float v = 0.f;
+#pragma unroll 8
+        for (int p = grp; p < P; p += G) v += Tpart[((int64_t)p * M + m) * r + jr];
+        Tg[threadIdx.x] = v;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < r; j += blockDim.x) {
+        float v = 0.f;
+        for (int q = 0; q < G; ++q) v += Tg[q * r + j];
+        Ts[j] = v;
+        if (blockIdx.x == 0 && T_out) T_out[(int64_t)m * r + j] = v;
+    }
+    __syncthreads();
+    const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= Dout) return;
+    float v = 0.f;
+    for (int z = 0; z < nsplit; ++z) v += partial[((int64_t)z * M + m) * Dout + n];
+    float ad = 0.f;
+    for (int j = 0; j < r; ++j)
+        ad = fmaf(Ts[j], __bfloat162float(__ushort_as_bfloat16(Bl[(int64_t)j * Dout + n])), ad);
+    Y[(int64_t)m * Dout + n] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(s, ad, v)));
 }
 
 // y[m, n] = sum_split partial + s * sum_j T[m, j] B[j, n]
@@ -543,9 +693,19 @@ static int num_sms_gemv() {
     return n;
 }
 
+size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r) {
+    const int64_t nsplit = (Din + kFwdKS - 1) / kFwdKS;
+    return (size_t)nsplit * kStBlocks * M * r;
+}
+
+// With Aad set, the streamed kernel also computes the adapter-down partials
+// (Tpart) and the fused finalize reduces them; if the streamed kernel cannot
+// run for this weight, QLORA_EUNSUPPORTED is returned before anything is
+// enqueued.  Without Aad, T is the finished adapter-down product.
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, uint32_t *d_status, cudaStream_t st) {
+                    float *partial, uint32_t *d_status, cudaStream_t st, const uint16_t *Aad,
+                    float *Tpart, float *T_out) {
     const int64_t Din = q.cols, Dout = q.rows;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
     const int64_t nsplit = (Din + kFwdKS - 1) / kFwdKS;
@@ -562,8 +722,9 @@ int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codeb
                                             Dout, nbr, 16, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         else
             stream = stream && tc::make_map(&tmC, q.absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, nbr,
-                                            Dout, nbr * 4, 16, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                                            Dout, nbr * 4, 8, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
+    if (Aad && !stream) return QLORA_EUNSUPPORTED;
     prof_begin(kProfGemv, st);
     if (stream) {
         const int ntr = (int)((Dout + kStRows - 1) / kStRows);
@@ -571,12 +732,12 @@ int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codeb
         const int grid = ntiles < num_sms_gemv() ? ntiles : num_sms_gemv();
         if (M <= 8) {
             cudaFuncSetAttribute(k_gemv_fwd_stream<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
-            k_gemv_fwd_stream<1><<<grid, kStThreads, kStSmem, st>>>(tmP, tmC, X, M, Din, Dout, sc, cb,
-                                                                     ntr, ntiles, partial, d_status);
+            k_gemv_fwd_stream<1><<<grid, kStThreads, kStSmem, st>>>(
+                tmP, tmC, X, M, Din, Dout, sc, cb, ntr, ntiles, partial, Aad, r, Tpart, d_status);
         } else {
             cudaFuncSetAttribute(k_gemv_fwd_stream<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
-            k_gemv_fwd_stream<2><<<grid, kStThreads, kStSmem, st>>>(tmP, tmC, X, M, Din, Dout, sc, cb,
-                                                                     ntr, ntiles, partial, d_status);
+            k_gemv_fwd_stream<2><<<grid, kStThreads, kStSmem, st>>>(
+                tmP, tmC, X, M, Din, Dout, sc, cb, ntr, ntiles, partial, Aad, r, Tpart, d_status);
         }
     } else {
         const size_t smem = 256 * 32 * 4 + 16 * (kFwdKS + 8) * 2;   // pair table + x slice
@@ -591,6 +752,13 @@ int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codeb
     }
     prof_end(kProfGemv, st);
     QLORA_LAUNCH_CHECK();
+    if (Aad) {
+        dim3 fg((unsigned)((Dout + 255) / 256), (unsigned)M);
+        k_gemv_fwd_finalize_fused<<<fg, 256, 0, st>>>(partial, (int)nsplit, M, Dout, Tpart, r, Bl, s, Y,
+                                                     T_out);
+        QLORA_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
     const int64_t n = (int64_t)M * Dout;
     k_gemv_fwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, (int)nsplit, M, Dout,
                                                                      T, Bl, r, s, Y);
