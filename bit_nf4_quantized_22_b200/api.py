@@ -113,6 +113,19 @@ def dequantize(q: NF4Weight, codebook: torch.Tensor | None = None,
     return out
 
 
+def merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, pool_group: int = 1,
+          codebook: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [Dout, Din] weight with the adapter folded in (qlora_merge)."""
+    r = B.shape[0]
+    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=torch.bfloat16,
+                                                  device=q.packed.device)
+    qc = q.c_struct()
+    rc = load().qlora_merge(ctypes.byref(qc), _cb_host(codebook), _ptr(A), _ptr(B), r,
+                            float(alpha), pool_group, _ptr(out), _stream())
+    _lib.check(rc, "qlora_merge")
+    return out
+
+
 def workspace_size(M: int, q: NF4Weight, r: int, pool_group: int = 1, which: int = 0) -> int:
     qc = q.c_struct()
     return int(load().qlora_workspace_size(M, ctypes.byref(qc), r, pool_group, which))

@@ -128,7 +128,7 @@ __device__ __forceinline__ void cp_async_wait() {
 
 namespace qlora {
 // Launch accounting and optional per-kernel event timing (profile.cu).
-enum ProfKind { kProfUmma = 0, kProfGemv = 1, kProfQuant = 2, kProfAdapter = 3, kProfKinds = 4 };
+enum ProfKind { kProfUmma = 0, kProfGemv = 1, kProfQuant = 2, kProfAdapter = 3, kProfMerge = 4, kProfKinds = 5 };
 void count_launch();
 void prof_begin(int kind, cudaStream_t st);
 void prof_end(int kind, cudaStream_t st);

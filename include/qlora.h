@@ -110,6 +110,22 @@ int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16]
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out,
                    void *stream);
 
+/* qlora_merge -- the weight with the adapter folded in, for deployment
+ * ("从 LoRA 到 QLoRA、QA-LoRA" section 2, W_eff = dequant(W4) + (alpha/r) A B;
+ * bitsandbytes article (CSDN) 12.10, merging before deployment):
+ *   W_out[n][k] = RN_bf16( w_hat[n][k] + (s/g) sum_j A[k/g][j] B[j][n] ),
+ * s = alpha/r, g = pool_group, w_hat the bf16 dequantized weight as
+ * nf4_dequantize writes it; the rank-r sum is accumulated in fp32.  With
+ * g = 64 every input of a group shares (A_p B)/g (the same blog, section 5),
+ * so that x . W_out^T is the pooled layer's forward.
+ *   A       device bf16 [Din/pool_group, r];  B  device bf16 [r, Dout]
+ *   W_out   device bf16 [Dout, Din], 16-byte aligned (output)
+ * No workspace.  Errors as nf4_dequantize, plus EINVAL for r outside
+ * [1, QLORA_MAX_RANK], a non-finite alpha or pool_group not 1 or 64. */
+int qlora_merge(const nf4_weight_t *q, const float codebook[16], const uint16_t *A,
+                const uint16_t *B, int32_t r, float alpha, int32_t pool_group, uint16_t *W_out,
+                void *stream);
+
 /* Scratch bytes qlora_forward (which = 0) or qlora_backward (which = 1)
  * needs for this problem.  Returns 0 when the arguments are invalid. */
 size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t pool_group,
@@ -177,7 +193,8 @@ int64_t qlora_launch_count(void);
 
 /* When enabled, each launch of the library's main kernels is bracketed by a
  * CUDA event pair recorded on its launch stream.  Kinds: 0 tensor-core GEMM
- * (tcgen05), 1 small-M GEMV kernels, 2 quantize kernel. */
+ * (tcgen05), 1 small-M GEMV kernels, 2 quantize kernel, 3 adapter products,
+ * 4 merge kernel. */
 void qlora_profile_enable(int on);
 
 /* Forget recorded events and zero the launch count (host only). */
