@@ -316,9 +316,18 @@ def run_ours(args, rank, world, dist):
                                + 2 * M * Dout * Din + 2 * M * Din * r)    # dX + adapter ext
     umma_tf = umma_flops / (umma_ms.value / 1e3) / 1e12 if umma_ms.value > 0 else None
     traffic = stored_traffic("umma_gemm.cu", "k_umma_qgemm_up_proj_4096x11008_M4096.md")
-    roof = {"bound": "tensor", "kernel": "k_umma_qgemm", "achieved": umma_tf, "peak": tf_sus,
-            "unit": "TFLOP/s", "frac": (umma_tf / tf_sus) if umma_tf else None,
-            "traffic": traffic, "peak_kind": f"bf16 dense, sustained ({peak_src})",
+    # Peak: the burst GEMM figure while the SM clock held its maximum with no
+    # power cap during the timed region (short steps do not reach the cap),
+    # else the sustained, power-capped figure.
+    csum = clk.summary()
+    capped = ("sw_power_cap" in csum.get("reasons", []) or csum.get("sm_mhz") is None
+              or (csum.get("sm_max_mhz") and csum["sm_mhz"] < 0.95 * csum["sm_max_mhz"]))
+    tf_peak = tf_sus if capped else tf_burst
+    roof = {"bound": "tensor", "kernel": "k_umma_qgemm", "achieved": umma_tf, "peak": tf_peak,
+            "unit": "TFLOP/s", "frac": (umma_tf / tf_peak) if umma_tf else None,
+            "traffic": traffic,
+            "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'} ({peak_src})",
+            "frac_of_sustained": (umma_tf / tf_sus) if umma_tf else None,
             "launches": int(umma_n.value),
             "share_of_step": umma_ms.value / sum(step_ms) if step_ms else None}
     qbytes = Din * Dout * 4 + weight_bytes(Din, Dout)
@@ -381,7 +390,7 @@ def run_ours(args, rank, world, dist):
         "quantize_roofline": quant,
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "clocks": csum,
         "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
         "decode": extras,
     }
@@ -428,18 +437,108 @@ def decode_lines(args, q, lib, torch, dev, hbm, flush):
             n, ms = ctypes.c_int64(), ctypes.c_double()
             lib.qlora_profile_read(1, ctypes.byref(n), ctypes.byref(ms))
             step = statistics.median(s.elapsed_time(e) for s, e in ev)
+            # the same forward captured once in a CUDA graph and replayed: device
+            # time without the host's per-call launch overhead
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                q.forward(x, w, A, B, spec.alpha, out=y, workspace=ws, save_T=False)
+            gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            for s_, e_ in gev:
+                flush.zero_()
+                s_.record()
+                graph.replay()
+                e_.record()
+            torch.cuda.synchronize()
+            gstep = statistics.median(s_.elapsed_time(e_) for s_, e_ in gev)
+            del graph
             wb = weight_bytes(spec.Din, spec.Dout)
             alg = wb + 2 * M * spec.Din + 2 * M * spec.Dout + 2 * spec.r * (spec.Din + spec.Dout) + 4 * M * spec.r
             kern_ms = ms.value / max(1, n.value)
+            bwd = backward_line(q, lib, torch, dev, hbm, flush, spec, cfg, lin, w, A, B, x, M)
             res[f"{spec.Din}x{spec.Dout}_M{M}"] = {
+                "backward": bwd,
                 "forward_ms": step, "weight_GBps": wb / (step / 1e3) / 1e9,
+                "forward_graph_ms": gstep, "weight_GBps_graph": wb / (gstep / 1e3) / 1e9,
                 "kernel": "k_gemv_fwd_stream", "kernel_ms": kern_ms,
                 "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
                 "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None,
                 "tflops": (2 * M * spec.Din * spec.Dout + 2 * M * spec.r * (spec.Din + spec.Dout)) / (step / 1e3) / 1e12,
             }
         del w
+    res["merge"] = merge_line(q, lib, torch, dev, hbm, flush)
     return res
+
+
+def backward_line(q, lib, torch, dev, hbm, flush, spec, cfg, lin, w, A, B, x, M):
+    """qlora_backward (dX, dA, dB) at small M: step time and the dX GEMV
+    kernel's HBM roofline fraction (weight + dY + dX bytes per launch)."""
+    import ctypes
+    dy_bits = synth.draw(spec, M, cfg, lin, which=("dY",))["dY"]
+    dy = torch.from_numpy(np.ascontiguousarray(dy_bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    _, T = q.forward(x, w, A, B, spec.alpha)
+    ws = torch.empty(max(1, q.workspace_size(M, w, spec.r, 1, 1)), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        q.backward(x, dy, w, A, B, spec.alpha, T=T, workspace=ws)
+    reps = 20
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    torch.cuda.synchronize()
+    lib.qlora_profile_reset()
+    lib.qlora_profile_enable(1)
+    for s_, e_ in ev:
+        flush.zero_()
+        s_.record()
+        q.backward(x, dy, w, A, B, spec.alpha, T=T, workspace=ws)
+        e_.record()
+    torch.cuda.synchronize()
+    lib.qlora_profile_enable(0)
+    n, ms = ctypes.c_int64(), ctypes.c_double()
+    lib.qlora_profile_read(1, ctypes.byref(n), ctypes.byref(ms))
+    step = statistics.median(s_.elapsed_time(e_) for s_, e_ in ev)
+    kern_ms = ms.value / max(1, n.value)
+    alg = (weight_bytes(spec.Din, spec.Dout) + 2 * M * spec.Dout + 2 * M * spec.Din
+           + 2 * spec.r * spec.Din + 4 * M * spec.r)
+    return {"backward_ms": step, "kernel": "k_gemv_bwd", "kernel_ms": kern_ms,
+            "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
+            "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None}
+
+
+def merge_line(q, lib, torch, dev, hbm, flush):
+    """qlora_merge on the 8192 -> 28672 weight (r = 64): the bf16 weight with
+    the adapter folded in; HBM-bound (0.52 B in, 2 B out per weight)."""
+    import ctypes
+    spec = synth.CONFIGS[5]["linears"][0]
+    base = synth.draw(spec, 1, 5, 0, which=("W", "A", "B"))
+    W = torch.from_numpy(base["W"]).to(dev)
+    w = q.quantize(W, double_quant=True)
+    del W
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    A, B = bf(base["A"]), bf(base["B"])
+    out = torch.empty(spec.Dout, spec.Din, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        q.merge(w, A, B, spec.alpha, out=out)
+    reps = 10
+    torch.cuda.synchronize()
+    lib.qlora_profile_reset()
+    lib.qlora_profile_enable(1)
+    for _ in range(reps):
+        flush.zero_()
+        q.merge(w, A, B, spec.alpha, out=out)
+    torch.cuda.synchronize()
+    lib.qlora_profile_enable(0)
+    n, ms = ctypes.c_int64(), ctypes.c_double()
+    lib.qlora_profile_read(4, ctypes.byref(n), ctypes.byref(ms))
+    kern_ms = ms.value / max(1, n.value)
+    alg = (weight_bytes(spec.Din, spec.Dout) + 2 * spec.Din * spec.Dout
+           + 2 * spec.r * (spec.Din + spec.Dout))
+    del w, out
+    return {"shape": f"{spec.Dout}x{spec.Din} r={spec.r}", "kernel": "k_merge", "kernel_ms": kern_ms,
+            "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
+            "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None}
 
 
 def main():

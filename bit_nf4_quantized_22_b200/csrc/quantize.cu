@@ -206,8 +206,10 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
 }
 
 // ------------------------------------------------------------------ fast path
-// One CTA per group of 256 blocks, brought in by four 16 KB bulk copies so
-// work starts when the first quarter lands.  A warp takes two blocks at a
+// One CTA per group of 256 blocks, brought in as four 16 KB bulk copies
+// through two buffers: quarters 0 and 1 load at once, quarter c + 2 into
+// buffer c % 2 as soon as the CTA is done with quarter c.  Five CTAs fit on
+// an SM (32 KB each), so loads stay in flight while others compute.  A warp takes two blocks at a
 // time: lanes 0-15 the first, 16-31 the second, four consecutive weights per
 // lane.  Lane j of a half also holds the exact threshold tau_j of its block
 // (lane 15: +inf).  A weight's index then costs one table lookup and one
@@ -223,15 +225,15 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
 constexpr float kBinK = 15.49f;
 constexpr float kBinC = 12582928.0f;   // 1.5 * 2^23 + 16: the low 5 bits of the sum are the bin
 constexpr int kQfThreads = 256;
-constexpr int kQfSmem = 256 * 64 * 4;
+constexpr int kQfSmem = 2 * 64 * 64 * 4;   // two 16 KB quarter buffers
 
 template <bool kExactHalf>
-__global__ void __launch_bounds__(kQfThreads, 3)
+__global__ void __launch_bounds__(kQfThreads, 5)
 k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins,
                     int zero_idx, int dq, uint8_t *__restrict__ packed,
                     float *__restrict__ absmax, uint8_t *__restrict__ codes,
                     float *__restrict__ steps, uint32_t *__restrict__ status) {
-    extern __shared__ __align__(128) float qw[];   // [256 blocks][64 weights]
+    extern __shared__ __align__(128) float qw[];   // [2 buffers][64 blocks][64 weights]
     __shared__ __align__(8) uint64_t bars[4];
     __shared__ float s_a[kQfThreads];
     __shared__ float s_cb[16];
@@ -250,7 +252,7 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
         tc::fence_proxy_async();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             const int n = nblk - 64 * c;
             if (n > 0) {
                 const uint32_t bytes = (uint32_t)(n < 64 ? n : 64) * 256u;
@@ -275,10 +277,22 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     bool ok = true;
     uint32_t bad_any = 0;
     for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(smem_u32(&bars[c]), 0, &abort_flag));
+        if (c >= 2) {
+            // quarter c - 2 is done everywhere: its buffer takes quarter c
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                const int n = nblk - 64 * c;
+                const uint32_t bytes = (uint32_t)(n < 64 ? n : 64) * 256u;
+                tc::fence_proxy_async();
+                tc::mbar_expect_tx(smem_u32(&bars[c]), bytes);
+                tc::bulk_load(smem_u32(qw) + (c & 1) * 16384u, W + (b0 + 64 * c) * 64, bytes,
+                              smem_u32(&bars[c]));
+            }
+        }
+        if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(smem_u32(&bars[c]), 0, &abort_flag));
         if (!ok) {
             abort_flag = 1;
-            break;
+            continue;   // keep meeting the CTA barriers
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -286,7 +300,7 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
             const bool valid = bl < nblk;
             float w[4] = {0.f, 0.f, 0.f, 0.f};
             if (valid) {
-                const float4 v = *reinterpret_cast<const float4 *>(qw + bl * 64 + 4 * j);
+                const float4 v = *reinterpret_cast<const float4 *>(qw + ((c & 1) * 64 + (bl & 63)) * 64 + 4 * j);
                 w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
             }
             // max |w| on the bit patterns: NaN and Inf sort above every finite value
