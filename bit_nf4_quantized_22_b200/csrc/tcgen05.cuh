@@ -10,7 +10,12 @@
 namespace qlora {
 namespace tc {
 
-constexpr uint32_t kWaitLimit = 1u << 22;   // polls before a wait gives up
+constexpr uint32_t kWaitLimit = 1u << 22;   // raw polls (no suspend) before a drain gives up
+// Bounded waits poll with a suspend-time hint: a waiting warp sleeps until
+// the phase completes or the hint elapses instead of spinning on the issue
+// slots.  Worst case kWaitPolls * kSuspendNs ~ 2 s before giving up.
+constexpr uint32_t kWaitPolls = 1u << 20;
+constexpr uint32_t kSuspendNs = 2000;
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
@@ -33,12 +38,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait on an mbarrier phase.  Gives up (returns false) after
-// kWaitLimit polls, or early when another role has already given up.
+// kWaitPolls polls, or early when another role has already given up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort_flag) return false;
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if ((i & 15u) == 15u && *abort_flag) return false;
     }
     return false;
 }
@@ -60,6 +76,17 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+
+// Tiled TMA store of a shared-memory box to global memory (bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Waits until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -152,14 +179,26 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
                                                   volatile int *abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort_flag) return false;
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (mbar_try_wait_cluster_sleep(bar, parity)) return true;
+        if ((i & 15u) == 15u && *abort_flag) return false;
     }
     return false;
 }
+
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier of the pair's first CTA (`bar0` is a shared::cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *tm, int x, int y,

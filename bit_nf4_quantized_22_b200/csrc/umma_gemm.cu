@@ -50,6 +50,7 @@ constexpr int kDqThreads = kDqWarps * 32;
 constexpr int kThreads = 64 + kDqThreads;
 static_assert(kDqThreads == 256, "one half 64-block per dequant thread");
 static_assert(kStageBytes % 1024 == 0, "stages keep 1 KB swizzle alignment");
+static_assert(kStages * kStageBytes >= 2 * 65536, "the epilogue stages a 256 x 256 bf16 tile in the ring");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 
@@ -108,7 +109,7 @@ __device__ __forceinline__ void decode_half(uint4 c, float ah, const Codebook &c
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
              const __grid_constant__ CUtensorMap tmAe, const __grid_constant__ CUtensorMap tmBe,
-             const UmmaParams p) {
+             const __grid_constant__ CUtensorMap tmY, const UmmaParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -309,32 +310,46 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         if (!ok) *abort_flag = 1;
 
         // ---------------------------------------------------------- epilogue
+        // TMEM -> registers -> bf16 -> the idle stage ring, as 128-byte-swizzled
+        // [128 rows][64 columns] boxes (half hh at hh * 64 KB, box j at + 16 KB j),
+        // then TMA stores of whole boxes: coalesced, and clipped at M and N.
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(acc_bar, 0, abort_flag));
         if (ok) {
             tc_fence_after();
             const int q = warp & 3;                       // TMEM lane quarter of this warp
             const int hh = (warp - 2) >> 2;               // accumulator (MMA half) of this warp
-            const int64_t m = m0 + 256 * hh + 128 * rank + 32 * q + lane;
+            const uint32_t L = 32 * q + lane;             // tile row = TMEM lane
+            const uint32_t stile = base + hh * 65536 + L * 128;
             for (int c = 0; c < 8; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + hh * 256 + c * 32, v);
-                if (m < p.M) {
-                    uint16_t *dst = p.Y + m * p.N + n0 + c * 32;
+                const uint32_t box = stile + (c >> 1) * 16384;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (n0 + c * 32 + 8 * i < p.N) {
-                            uint4 o;
-                            o.x = bf16x2_bits(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                            o.y = bf16x2_bits(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                            o.z = bf16x2_bits(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                            o.w = bf16x2_bits(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-                            *reinterpret_cast<uint4 *>(dst + 8 * i) = o;
-                        }
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t chunk = 4 * (c & 1) + i;
+                    sts128(box + ((chunk ^ (L & 7)) << 4),
+                           bf16x2_bits(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
+                           bf16x2_bits(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                           bf16x2_bits(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                           bf16x2_bits(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
                 }
             }
+            fence_proxy_async();                          // the writes, visible to the TMA engine
         } else {
             *abort_flag = 1;
+        }
+        asm volatile("bar.sync 1, %0;\n" ::"n"(kDqThreads));
+        if (ok && threadIdx.x == 64) {
+            for (int hh = 0; hh < 2; ++hh) {
+                const int64_t y = m0 + 256 * hh + 128 * rank;
+                if (y >= p.M) continue;
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t x = n0 + 64 * j;
+                    if (x < p.N) tma_store_2d(&tmY, base + hh * 65536 + j * 16384, (int)x, (int)y);
+                }
+            }
+            bulk_commit();
+            bulk_wait_all();
         }
     }
 
@@ -376,6 +391,10 @@ int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t
     // [128 rows][32 B] (32 B swizzle), backward [64 rows][64 B] (64 B swizzle)
     bool ok = make_map(&tA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Kmain, M, Kmain * 2, 64, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B);
+    // output boxes [128 rows][64 columns], 128-byte swizzle (the epilogue's staging layout)
+    CUtensorMap tY;
+    ok = ok && make_map(&tY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, N * 2, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (mode == 0)
         ok = ok && make_map(&tP, q.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Din / 2, Dout, Din / 2,
                             32, 128, CU_TENSOR_MAP_SWIZZLE_32B);
@@ -409,7 +428,7 @@ int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t
     // clusters of two CTAs along x: pair index = N tile of 256, rank = half
     dim3 grid((unsigned)(2 * ((N + 255) / 256)), (unsigned)((M + 511) / 512));
     prof_begin(kProfUmma, st);
-    k_umma_qgemm<<<grid, kThreads, kSmemBytes, st>>>(tA, tP, tAe, tBe, p);
+    k_umma_qgemm<<<grid, kThreads, kSmemBytes, st>>>(tA, tP, tAe, tBe, tY, p);
     prof_end(kProfUmma, st);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
