@@ -87,7 +87,8 @@ struct ReduceArgs {
     uint16_t *out_split; int64_t sp;
 };
 
-__global__ void k_reduce(ReduceArgs a) {
+// General layout (any Qp): one thread per output element.
+__global__ void k_reduce_scalar(ReduceArgs a) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= a.P * a.Qv) return;
     const int64_t p = i / a.Qv;
@@ -104,6 +105,40 @@ __global__ void k_reduce(ReduceArgs a) {
         const uint16_t h = to_bf16(v);
         a.out_split[p * 2 * a.sp + q] = h;
         a.out_split[p * 2 * a.sp + a.sp + q] = to_bf16(v - from_bf16(h));
+    }
+}
+
+// block (32, 8): thread (x, y) handles the 4 columns [4x + 128 bx, +4) of row
+// p = 8 by + y with 16-byte loads (Qp and H are multiples of 4), splits
+// unrolled 4 at a time; the sum order over z is fixed.
+__global__ void __launch_bounds__(256) k_reduce(ReduceArgs a) {
+    const int64_t p = (int64_t)blockIdx.y * 8 + threadIdx.y;
+    const int q0 = 4 * (blockIdx.x * 32 + threadIdx.x);
+    if (p >= a.P || q0 >= a.Qv) return;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *base = a.partial + p * a.Qp + q0;
+    const int64_t zs = a.P * a.Qp;
+#pragma unroll 4
+    for (int z = 0; z < a.splits; ++z) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(base + z * zs));
+        v.x += x.x, v.y += x.y, v.z += x.z, v.w += x.w;
+        if (a.H) {
+            const float4 y = __ldg(reinterpret_cast<const float4 *>(base + z * zs + a.H));
+            v.x += y.x, v.y += y.y, v.z += y.z, v.w += y.w;
+        }
+    }
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int q = q0 + e;
+        if (q >= a.Qv) break;
+        if (a.out_f32) a.out_f32[p * a.fsp + q * a.fsq] = a.f32_scale * vv[e];
+        if (a.out_bf16) a.out_bf16[p * a.bsp + q] = to_bf16(a.bf_scale * vv[e]);
+        if (a.out_split) {
+            const uint16_t h = to_bf16(vv[e]);
+            a.out_split[p * 2 * a.sp + q] = h;
+            a.out_split[p * 2 * a.sp + a.sp + q] = to_bf16(vv[e] - from_bf16(h));
+        }
     }
 }
 
@@ -143,9 +178,13 @@ int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H
                   cudaStream_t st) {
     ReduceArgs a{partial, splits, P, Qp, H, Qv, f32_scale, out_f32, fsp, fsq,
                  bf_scale, out_bf16, bsp, out_split, sp};
-    const int64_t n = P * Qv;
-    if (n == 0) return QLORA_OK;
-    k_reduce<<<blocks_for(n), 256, 0, st>>>(a);
+    if (P * Qv == 0) return QLORA_OK;
+    if (Qp % 4 != 0 || H % 4 != 0 || (reinterpret_cast<uintptr_t>(partial) & 15u) != 0) {
+        k_reduce_scalar<<<blocks_for(P * Qv), 256, 0, st>>>(a);
+    } else {
+        dim3 grid((unsigned)((Qv + 127) / 128), (unsigned)((P + 7) / 8));
+        k_reduce<<<grid, dim3(32, 8), 0, st>>>(a);
+    }
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }

@@ -652,6 +652,219 @@ k_gemv_bwd(const uint16_t *__restrict__ dY, int M, int64_t Din, int64_t Dout,
     }
 }
 
+// ------------------------------------------------------------------ backward dX, streamed
+// grid (Din / 512 slices kz, nsplit): CTA (kz, sp) reduces over its range of
+// 128-row tiles of the weight, dX[m][k] for the slice's 512 inputs k.  A
+// producer warp streams each tile -- the packed rows (two 128-byte-swizzled
+// boxes of 128 rows x 128 bytes), the rows' scale codes and dY[:, rows] (two
+// 64-column swizzled boxes of min(M, 16) token rows; the rows past M hold
+// whatever the buffer held, which only reaches output rows that are never
+// stored) -- through a three-stage ring.
+//
+// Sixteen compute warps: warp w owns the 64-block kb = w % 8 of the slice
+// and the 16-row groups q = w / 8, w / 8 + 2, ... of every tile, and keeps
+// its 16 tokens x 64 inputs accumulator in registers across the whole range
+// (warps w and w + 8 are added once at the end).  MMA m16n8k16: the tokens
+// are M, 8 inputs {8g' + i} are N (MMA i = 0..7), and the group's 16 rows are
+// K, relabelled so that lane t's K slots 2t, 2t+1, 2t+8, 2t+9 are its rows
+// 4t..4t+3.  Lane (g, t) reads one packed word (inputs 8g..8g+7) of each of
+// its four rows, decodes it with four lookups of the byte -> bf16-pair table
+// (the same table as the forward), and pairs rows with byte permutes.  The
+// weights there are the bare codebook values, so the per-row block scale is
+// moved onto dY: dY[m][n] * a_hat[n][kb], exactly, as a hi + lo pair of bf16
+// (two MMAs), so that only the codebook's own bf16 rounding remains.
+constexpr int kBsRows = 128, kBsCols = 512;
+constexpr int kBsPacked = kBsRows * kBsCols / 2;           // 32 KB
+constexpr int kBsScale = kBsRows * 8 * 4;                   // 4 KB (codes use 2 KB)
+constexpr int kBsDy = 2 * 16 * 128;                         // two [16][64] bf16 boxes
+constexpr int kBsStage = kBsPacked + kBsScale + kBsDy;      // 40 KB
+constexpr int kBsStages = 3;
+constexpr int kBsThreads = 17 * 32;
+constexpr int kBsRed = 8 * 32 * 32 * 4;                    // odd-parity warps' sums
+constexpr int kBsSmem = kStLut + kBsStages * kBsStage + kBsRed + 1024 + 256;
+static_assert(kBsStage % 1024 == 0, "stages keep 1 KB swizzle alignment");
+
+__global__ void __launch_bounds__(kBsThreads, 1)
+k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmC,
+                  const __grid_constant__ CUtensorMap tmD, int M, int Mb, int64_t Din, int64_t Dout,
+                  ScaleSrc sc, Codebook cb, int ntn, int nsplit, float *__restrict__ partial,
+                  uint32_t *__restrict__ status) {
+    extern __shared__ __align__(1024) uint8_t ssm[];
+    const uint32_t raw = smem_u32(ssm);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = ssm + (base - raw);
+    const uint8_t *lutb = gbase;                                  // [256][256 B]
+    const uint32_t ring = base + kStLut;
+    uint8_t *gring = gbase + kStLut;
+    float *red = reinterpret_cast<float *>(gring + kBsStages * kBsStage);   // [8][32][32]
+    const uint32_t bar0 = ring + kBsStages * kBsStage + kBsRed;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kBsStages + s); };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + (bar0 - base) + 64);
+    float *cbs = reinterpret_cast<float *>(gbase + (bar0 - base) + 128);
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int kz = blockIdx.x, sp = blockIdx.y;
+    const int t0 = (int)((int64_t)sp * ntn / nsplit), t1 = (int)((int64_t)(sp + 1) * ntn / nsplit);
+    const int64_t nbr = Din / 64;
+
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
+        for (int s = 0; s < kBsStages; ++s) {
+            tc::mbar_init(full(s), 1);
+            tc::mbar_init(empty(s), 16);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        tc::fence_proxy_async();
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {   // table row e: 32 copies of (c[e >> 4], c[e & 15]) in bf16
+        const int e = threadIdx.x;
+        const uint32_t v = bf16x2_bits(cbs[e >> 4], cbs[e & 15]);
+        uint4 *row = reinterpret_cast<uint4 *>(gbase + e * 256);
+        const uint4 vv = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) row[(i + lane) & 7] = vv;
+    }
+    __syncthreads();
+    bool ok = true;
+
+    if (warp == 16) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint32_t cbytes = sc.dq ? kBsRows * 16 : kBsRows * 8 * 4;
+            for (int i = 0, tt = t0; tt < t1 && ok; ++i, ++tt) {
+                const int s = i % kBsStages;
+                if (i >= kBsStages) ok = tc::mbar_wait(empty(s), ((i / kBsStages) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                const uint32_t st = ring + s * kBsStage;
+                const int n0 = tt * kBsRows;
+                tc::mbar_expect_tx(full(s), kBsPacked + cbytes + 2 * Mb * 128);
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    tc::tma_load_2d(st + q * (kBsRows * 128), &tmP, kz * (kBsCols / 2) + 128 * q, n0, full(s));
+                if (sc.dq)   // 16 codes per row from the 16-aligned start; this slice's 8 at 8 * (kz % 2)
+                    tc::tma_load_2d(st + kBsPacked, &tmC, 16 * (kz >> 1), n0, full(s));
+                else
+                    tc::tma_load_2d(st + kBsPacked, &tmC, 8 * kz, n0, full(s));
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    tc::tma_load_2d(st + kBsPacked + kBsScale + q * 2048, &tmD, n0 + 64 * q, 0, full(s));
+            }
+            if (!ok) *abort_flag = 1;
+        }
+    } else {
+        // ---------------------------------------------------------- compute warps
+        const uint32_t lanebits = 4u * lane;
+        auto lookup = [&](uint32_t word, int k) -> uint32_t {
+            const uint32_t off = __byte_perm(word, lanebits, 0x5504u | ((uint32_t)k << 4));
+            return *reinterpret_cast<const uint32_t *>(lutb + off);
+        };
+        const int kb = warp & 7, qpar = warp >> 3;
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+        for (int i = 0, tt = t0; tt < t1; ++i, ++tt) {
+            const int s = i % kBsStages;
+            if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (i / kBsStages) & 1, abort_flag));
+            if (!ok) {
+                *abort_flag = 1;
+                break;   // no CTA-wide barrier inside this loop
+            }
+            const uint8_t *stg = gring + s * kBsStage;
+            const int64_t n0 = (int64_t)tt * kBsRows;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = 2 * qq + qpar;                 // 16-row group of the tile
+                float ah[4];
+                uint32_t R[4][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int rl = 16 * q + 4 * t + j;       // tile row
+                    const int64_t n = n0 + rl;
+                    // packed word: bytes 32 kb + 4 g .. + 3 of the tile row (box kb / 4)
+                    const int chunk = 2 * (kb & 3) + (g >> 2);
+                    const uint32_t word = *reinterpret_cast<const uint32_t *>(
+                        stg + (kb >> 2) * (kBsRows * 128) + rl * 128 + ((chunk ^ (rl & 7)) << 4) + 4 * (g & 3));
+                    float a = 0.f;
+                    if (n < Dout) {
+                        if (sc.dq) {
+                            const uint8_t code = stg[kBsPacked + rl * 16 + 8 * (kz & 1) + kb];
+                            // the slice's blocks of row n lie in one double-quant group
+                            const float step = __ldg(sc.step + (((uint32_t)n * (uint32_t)nbr +
+                                                                 16u * (uint32_t)(kz >> 1)) >> 8));
+                            a = __fmul_rn((float)code, step);
+                        } else {
+                            a = reinterpret_cast<const float *>(stg + kBsPacked)[rl * 8 + kb];
+                        }
+                    }
+                    ah[j] = a;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) R[j][p] = lookup(word, p);
+                }
+                // A fragments: dY[token][row] * a_hat[row] as hi + lo bf16; rows 4t..4t+3
+                // of the group are K slots 2t, 2t+1 (reg 0/1) and 2t+8, 2t+9 (reg 2/3)
+                uint32_t ahi[4], alo[4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {            // token g (h = 0) or g + 8
+                    const int m = g + 8 * h;
+                    const int nn = 16 * q + 4 * t;          // tile row of j = 0 (column of dY)
+                    const uint8_t *dyb = stg + kBsPacked + kBsScale + (nn >> 6) * 2048 + m * 128;
+                    const int cch = (nn & 63) >> 3;         // 16-byte chunk, 4 rows = 8 bytes
+                    const uint2 dv = *reinterpret_cast<const uint2 *>(dyb + ((cch ^ (m & 7)) << 4) + 2 * (nn & 7));
+                    const float d0 = bf16_lo(dv.x) * ah[0], d1 = bf16_hi(dv.x) * ah[1];
+                    const float d2 = bf16_lo(dv.y) * ah[2], d3 = bf16_hi(dv.y) * ah[3];
+                    const uint32_t h01 = bf16x2_bits(d0, d1), h23 = bf16x2_bits(d2, d3);
+                    ahi[h] = h01;
+                    ahi[2 + h] = h23;
+                    alo[h] = bf16x2_bits(d0 - bf16_lo(h01), d1 - bf16_hi(h01));
+                    alo[2 + h] = bf16x2_bits(d2 - bf16_lo(h23), d3 - bf16_hi(h23));
+                }
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii) {
+                    const uint32_t sel = (ii & 1) ? 0x7632u : 0x5410u;
+                    const uint32_t b[2] = {__byte_perm(R[0][ii >> 1], R[1][ii >> 1], sel),
+                                           __byte_perm(R[2][ii >> 1], R[3][ii >> 1], sel)};
+                    mma_bf16_16816(acc[ii], ahi, b);
+                    mma_bf16_16816(acc[ii], alo, b);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty(s));
+        }
+        // warps w + 8 hand their sums to warps w; columns: acc[ii] holds (token g,
+        // input 16t + ii), (g, 16t + 8 + ii), (g + 8, 16t + ii), (g + 8, 16t + 8 + ii)
+        float *rb = red + (kb * 32 + lane) * 32;
+        if (qpar) {
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii)
+                *reinterpret_cast<float4 *>(rb + 4 * ii) = make_float4(acc[ii][0], acc[ii][1], acc[ii][2], acc[ii][3]);
+        }
+        asm volatile("bar.sync 1, %0;\n" ::"n"(16 * 32));
+        if (!qpar && ok) {
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) {
+                const float4 o = *reinterpret_cast<const float4 *>(rb + 4 * ii);
+                const float v[4] = {acc[ii][0] + o.x, acc[ii][1] + o.y, acc[ii][2] + o.z, acc[ii][3] + o.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int m = g + 8 * (e >> 1);
+                    const int64_t k = (int64_t)kz * kBsCols + 64 * kb + 16 * t + 8 * (e & 1) + ii;
+                    if (m < M && k < Din) partial[((int64_t)sp * M + m) * Din + k] = v[e];
+                }
+            }
+        }
+    }
+    if (!ok && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
+    __syncwarp();
+    __syncthreads();
+}
+
 __global__ void k_gemv_bwd_finalize(const float *__restrict__ partial, int nsplit, int M,
                                     int64_t Din, const float *__restrict__ G,
                                     const uint16_t *__restrict__ Al, int r, int pool, float s,
@@ -676,10 +889,23 @@ size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     return (size_t)nsplit * M * Dout * sizeof(float);
 }
 
+static int num_sms_gemv();
+
+// splits of the streamed backward: at most one CTA per SM over the slices
+// (one CTA fits on an SM; a second wave would double the time)
+static int bwd_stream_splits(int64_t Din, int64_t Dout) {
+    const int64_t nkz = (Din + kBsCols - 1) / kBsCols, ntn = (Dout + kBsRows - 1) / kBsRows;
+    int64_t ns = num_sms_gemv() / nkz;
+    if (ns > ntn) ns = ntn;
+    return (int)(ns < 1 ? 1 : ns);
+}
+
 size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     const int64_t NS = kGemvWarps * kBwdRowsPerWarp;
-    const int64_t nsplit = (Dout + NS - 1) / NS;
-    return nsplit > 1 ? (size_t)nsplit * M * Din * sizeof(float) : 0;
+    int64_t nsplit = (Dout + NS - 1) / NS;
+    const int64_t ns2 = bwd_stream_splits(Din, Dout);   // the streamed kernel always writes partials
+    if (ns2 > nsplit) nsplit = ns2;
+    return (size_t)nsplit * M * Din * sizeof(float);
 }
 
 static int num_sms_gemv() {
@@ -771,6 +997,39 @@ int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Code
                     float *partial, cudaStream_t st) {
     const int64_t Din = q.cols, Dout = q.rows;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    // streamed kernel: scale rows TMA-tileable, at least one 512-input slice and one 128-row tile
+    const int64_t nbr = Din / 64;
+    bool stream = Din >= kBsCols && Dout >= kBsRows && Dout * nbr < (int64_t(1) << 32) &&
+                  (q.double_quant ? (nbr % 16 == 0) : (nbr % 4 == 0));
+    CUtensorMap tmP, tmC, tmD;
+    const int Mb = M < 16 ? M : 16;
+    if (stream) {
+        stream = tc::make_map(&tmP, q.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Din / 2, Dout, Din / 2,
+                              128, kBsRows, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (q.double_quant)
+            stream = stream && tc::make_map(&tmC, q.absmax_code, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nbr,
+                                            Dout, nbr, 16, kBsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+        else
+            stream = stream && tc::make_map(&tmC, q.absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, nbr,
+                                            Dout, nbr * 4, 8, kBsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+        stream = stream && tc::make_map(&tmD, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dout, M, Dout * 2,
+                                        64, Mb, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (stream) {
+        const int nkz = (int)((Din + kBsCols - 1) / kBsCols), ntn = (int)((Dout + kBsRows - 1) / kBsRows);
+        const int nsplit = bwd_stream_splits(Din, Dout);
+        cudaFuncSetAttribute(k_gemv_bwd_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmem);
+        prof_begin(kProfGemv, st);
+        k_gemv_bwd_stream<<<dim3((unsigned)nkz, (unsigned)nsplit), kBsThreads, kBsSmem, st>>>(
+            tmP, tmC, tmD, M, Mb, Din, Dout, sc, cb, ntn, nsplit, partial, nullptr);
+        prof_end(kProfGemv, st);
+        QLORA_LAUNCH_CHECK();
+        const int64_t n = (int64_t)M * Din;
+        k_gemv_bwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nsplit, M, Din, G,
+                                                                         Al, r, pool, s, dX);
+        QLORA_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
     constexpr int NS = kGemvWarps * kBwdRowsPerWarp;
     const int64_t nsplit = (Dout + NS - 1) / NS;
     const size_t smem = 16 * (NS + 8) * 2 + kGemvWarps * 16 * 64 * 4;

@@ -71,6 +71,7 @@ def test_ragged_small(orc, qlib, M, dq):
     (4, 2048, 4104, True),    # more tiles than SMs
     (3, 1088, 264, True),     # Din/64 = 17: scale rows not tileable -> register GEMV
     (12, 4160, 136, False),   # Din/64 = 65 (odd): register GEMV, ragged slice
+    (5, 1280, 392, False),    # streamed backward: last 512-input slice half full
 ])
 def test_gemv_paths(orc, qlib, M, Din, Dout, dq):
     spec = LinearSpec("g", Din, Dout, 8, 16.0, dq)
