@@ -219,7 +219,7 @@ static int run_mma_gemm(MmaGemmArgs a, cudaStream_t st) {
 int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN) {
     const int64_t tiles = ((P + 127) / 128) * ((Q + BN - 1) / BN);
     const int64_t nkt = (Rtot + kMmaBK - 1) / kMmaBK;
-    int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+    int64_t s = 2 * (int64_t)num_sms() / tiles;   // one wave of two CTAs per SM
     const int64_t cap = nkt / 8 > 1 ? nkt / 8 : 1;
     if (s > cap) s = cap;
     if (s > 32) s = 32;

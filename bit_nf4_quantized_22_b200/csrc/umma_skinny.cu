@@ -236,7 +236,9 @@ int skinny_n(int64_t Q) { return Q <= 64 ? 64 : (Q <= 128 ? 128 : (Q <= 192 ? 19
 // about one CTA per SM, at least 4 k-tiles per split, no empty split.
 void skinny_splits(int64_t P, int64_t Q, int nk, int *splits, int *per) {
     const int64_t tiles = ((P + kSBM - 1) / kSBM) * ((Q + 255) / 256);
-    int64_t s = (2 * sms() + tiles - 1) / tiles;       // two resident CTAs per SM
+    // two resident CTAs per SM; round down so that the grid is one wave
+    // (a few CTAs over the slots would cost a whole second round)
+    int64_t s = 2 * sms() / tiles;
     const int64_t cap = nk / 4 > 1 ? nk / 4 : 1;
     if (s > cap) s = cap;
     if (s < 1) s = 1;
