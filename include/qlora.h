@@ -187,6 +187,14 @@ int qlora_forward_noalloc(const uint16_t *X, int64_t M, const nf4_weight_t *q,
                           int32_t r, float alpha, int32_t pool_group, uint16_t *Y, float *T_save,
                           uint32_t *d_status, void *stream);
 
+/* qlora_selftest_wait_timeout -- failure-path check (not part of the layer's
+ * computation): launches one warp that waits, with the library's bounded
+ * mbarrier wait, on a barrier nothing arrives on.  The wait gives up after
+ * its poll limit (at most about two seconds) and ORs QLORA_STATUS_TIMEOUT into
+ * *d_status (device uint32, required); nothing traps, and the stream stays
+ * usable.  Returns EINVAL for a null status pointer. */
+int qlora_selftest_wait_timeout(uint32_t *d_status, void *stream);
+
 /* ---- Benchmark support (not part of the layer's computation) ----------
  * Kernel launches made by the library since the last qlora_profile_reset(). */
 int64_t qlora_launch_count(void);
