@@ -3,6 +3,8 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "mma_gemm.cuh"
 
@@ -461,6 +463,24 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
     return launch_mma_gemm(a, 128, st);
 }
 
+// A second stream per device for the backward's adapter-gradient products,
+// which run beside the dX tensor-core GEMM and fill the SMs its last wave
+// leaves idle.  Shared by all calls on the device; each call orders its work
+// on it with its own events.
+static cudaStream_t side_stream() {
+    static std::mutex mu;
+    static std::unordered_map<int, cudaStream_t> streams;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = streams.find(dev);
+    if (it != streams.end()) return it->second;
+    cudaStream_t s = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    streams[dev] = s;
+    return s;
+}
+
 int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_weight_t *q,
                    const float codebook[16], const uint16_t *A, const uint16_t *B, int32_t r,
                    float alpha, int32_t pool_group, const float *T_saved, uint16_t *dX, float *dA,
@@ -494,12 +514,31 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     }
     if (d.g > 1 && w.ph) RC(run_pool(d, X, w.ph, w.pl, st));
 
+    // With the tensor-core dX GEMM, dA and dB go to the side stream (after
+    // G): the GEMM is enqueued first, so its CTAs are placed first and the
+    // adapter products take the SMs its last wave leaves free.
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    if (want_dx && !d.small && !d.mma_large && (want_da || want_db)) {
+        side = side_stream();
+        if (side && (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+                     cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess ||
+                     cudaEventRecord(ev_fork, st) != cudaSuccess))
+            side = nullptr;
+    }
+    const cudaStream_t ast = side ? side : st;   // stream of the dA and dB work
+
     if (want_dx) {
         if (d.small) {
             RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st));
         } else if (!d.mma_large) {
-            RC(launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st));
-            RC(launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, w.Aext, dX, d_status, st));
+            int rcx = launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st);
+            if (rcx == QLORA_OK) rcx = launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, w.Aext, dX, d_status, st);
+            if (rcx != QLORA_OK) {
+                if (ev_fork) cudaEventDestroy(ev_fork);
+                if (ev_join) cudaEventDestroy(ev_join);
+                return rcx;
+            }
         } else {
             RC(launch_pad_rows(A, d.Din, r, d.rp, d.g, 1.f / d.g, w.Aext, st));
             RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));
@@ -517,25 +556,39 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
             RC(launch_mma_gemm(a, 128, st));
         }
     }
-    if (want_da) {
+    int rc = QLORA_OK;
+    if (side && cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess) rc = QLORA_ECUDA;
+    if (rc == QLORA_OK && want_da) {
         ProdPlan pl;
-        RC(run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), d.mma_large, w.dApart, d_status, st, &pl));
-        RC(launch_reduce(w.dApart, pl.splits, d.Da, pl.Qp, d.rp, r, s, dA, r, 1, 0.f, nullptr, 0,
-                         nullptr, 0, st));
+        rc = run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), d.mma_large, w.dApart, d_status, ast, &pl);
+        if (rc == QLORA_OK)
+            rc = launch_reduce(w.dApart, pl.splits, d.Da, pl.Qp, d.rp, r, s, dA, r, 1, 0.f, nullptr,
+                               0, nullptr, 0, ast);
     }
-    if (want_db) {
+    if (rc == QLORA_OK && want_db) {
         const float *T32 = T_saved;
         if (!T32) {
-            RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, w.T32, s, nullptr, d_status, st));
+            rc = run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, w.T32, s, nullptr, d_status,
+                                  ast);
             T32 = w.T32;
         }
-        RC(launch_split_f32(T32, M, r, d.rp, w.Tsplit, st));
+        if (rc == QLORA_OK) rc = launch_split_f32(T32, M, r, d.rp, w.Tsplit, ast);
         ProdPlan pl;
-        RC(run_prod(prod_dB(d, dY, w.Tsplit), d.mma_large, w.dBpart, d_status, st, &pl));
-        RC(launch_reduce(w.dBpart, pl.splits, d.Dout, pl.Qp, d.rp, r, s, dB, 1, d.Dout, 0.f,
-                         nullptr, 0, nullptr, 0, st));
+        if (rc == QLORA_OK)
+            rc = run_prod(prod_dB(d, dY, w.Tsplit), d.mma_large, w.dBpart, d_status, ast, &pl);
+        if (rc == QLORA_OK)
+            rc = launch_reduce(w.dBpart, pl.splits, d.Dout, pl.Qp, d.rp, r, s, dB, 1, d.Dout, 0.f,
+                               nullptr, 0, nullptr, 0, ast);
     }
-    return QLORA_OK;
+    if (side) {
+        // join: the caller's stream sees all of the backward (also on errors,
+        // so that nothing is left running unordered)
+        if (cudaEventRecord(ev_join, side) != cudaSuccess || cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess)
+            rc = rc == QLORA_OK ? QLORA_ECUDA : rc;
+    }
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+    return rc;
 }
 
 }  // extern "C"
