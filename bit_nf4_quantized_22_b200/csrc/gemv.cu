@@ -387,7 +387,10 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
                                                lookup(x1, i0 + 1)};
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kx + 4 * q]);
+                            // token rows past M are zero: skip their shared loads
+                            const uint2 xv = g + 8 * n < M
+                                                 ? *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kx + 4 * q])
+                                                 : make_uint2(0u, 0u);
                             const uint32_t bb[2] = {xv.x, xv.y};
                             mma_bf16_16816(tmp[n], a, bb);
                         }
