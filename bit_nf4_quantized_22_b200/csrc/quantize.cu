@@ -206,10 +206,11 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
 }
 
 // ------------------------------------------------------------------ fast path
-// One CTA per group of 256 blocks, brought in as four 16 KB bulk copies
-// through two buffers: quarters 0 and 1 load at once, quarter c + 2 into
-// buffer c % 2 as soon as the CTA is done with quarter c.  Five CTAs fit on
-// an SM (32 KB each), so loads stay in flight while others compute.  A warp takes two blocks at a
+// One CTA per group of 256 blocks.  Each warp reads its weights straight
+// from global memory with 16-byte streaming loads, the four passes of a
+// quarter issued together; four CTAs per SM keep enough loads in flight (in
+// measurements this beat staging the group through shared memory with bulk
+// copies).  A warp takes two blocks at a
 // time: lanes 0-15 the first, 16-31 the second, four consecutive weights per
 // lane.  Lane j of a half also holds the exact threshold tau_j of its block
 // (lane 15: +inf).  A weight's index then costs one table lookup and one
@@ -225,43 +226,24 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
 constexpr float kBinK = 15.49f;
 constexpr float kBinC = 12582928.0f;   // 1.5 * 2^23 + 16: the low 5 bits of the sum are the bin
 constexpr int kQfThreads = 256;
-constexpr int kQfSmem = 2 * 64 * 64 * 4;   // two 16 KB quarter buffers
+constexpr int kQfSmem = 0;
 
 template <bool kExactHalf>
-__global__ void __launch_bounds__(kQfThreads, 5)
+__global__ void __launch_bounds__(kQfThreads, 4)
 k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins,
                     int zero_idx, int dq, uint8_t *__restrict__ packed,
                     float *__restrict__ absmax, uint8_t *__restrict__ codes,
                     float *__restrict__ steps, uint32_t *__restrict__ status) {
-    extern __shared__ __align__(128) float qw[];   // [2 buffers][64 blocks][64 weights]
-    __shared__ __align__(8) uint64_t bars[4];
     __shared__ float s_a[kQfThreads];
     __shared__ float s_cb[16];
     __shared__ double s_half[16];
     __shared__ uint32_t s_lut[32];
     __shared__ float warp_max[kQfThreads / 32];
-    __shared__ int abort_flag;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t b0 = (int64_t)blockIdx.x * 256;
     const int nblk = (int)(nb - b0 < 256 ? nb - b0 : 256);
     s_a[threadIdx.x] = 0.f;
     if (threadIdx.x == 0) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::mbar_init(smem_u32(&bars[c]), 1);
-        abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        tc::fence_proxy_async();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int n = nblk - 64 * c;
-            if (n > 0) {
-                const uint32_t bytes = (uint32_t)(n < 64 ? n : 64) * 256u;
-                tc::mbar_expect_tx(smem_u32(&bars[c]), bytes);
-                tc::bulk_load(smem_u32(qw) + c * 16384u, W + (b0 + 64 * c) * 64, bytes, smem_u32(&bars[c]));
-            }
-        }
-        // parameter arrays are copied with constant indices only (a
-        // lane-dependent index would put the whole parameter on the stack)
 #pragma unroll
         for (int j = 0; j < 16; ++j) s_cb[j] = cb.c[j];
 #pragma unroll
@@ -274,35 +256,20 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     const float c_lo = s_cb[j < 15 ? j : 14], c_hi = s_cb[j < 15 ? j + 1 : 15];
     const double hk = s_half[j < 15 ? j : 14];
     const uint32_t lut = s_lut[lane];
-    bool ok = true;
     uint32_t bad_any = 0;
     for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
-        if (c >= 2) {
-            // quarter c - 2 is done everywhere: its buffer takes quarter c
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                const int n = nblk - 64 * c;
-                const uint32_t bytes = (uint32_t)(n < 64 ? n : 64) * 256u;
-                tc::fence_proxy_async();
-                tc::mbar_expect_tx(smem_u32(&bars[c]), bytes);
-                tc::bulk_load(smem_u32(qw) + (c & 1) * 16384u, W + (b0 + 64 * c) * 64, bytes,
-                              smem_u32(&bars[c]));
-            }
-        }
-        if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(smem_u32(&bars[c]), 0, &abort_flag));
-        if (!ok) {
-            abort_flag = 1;
-            continue;   // keep meeting the CTA barriers
+        float4 pre[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int bl = 64 * c + 2 * (warp + 8 * i) + half;
+            pre[i] = bl < nblk ? __ldcs(reinterpret_cast<const float4 *>(W + (b0 + bl) * 64 + 4 * j))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int bl = 64 * c + 2 * (warp + 8 * i) + half;   // block within the group
             const bool valid = bl < nblk;
-            float w[4] = {0.f, 0.f, 0.f, 0.f};
-            if (valid) {
-                const float4 v = *reinterpret_cast<const float4 *>(qw + ((c & 1) * 64 + (bl & 63)) * 64 + 4 * j);
-                w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
-            }
+            float w[4] = {pre[i].x, pre[i].y, pre[i].z, pre[i].w};
             // max |w| on the bit patterns: NaN and Inf sort above every finite value
             uint32_t m = 0;
 #pragma unroll
@@ -350,8 +317,6 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
         }
     }
     if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
-    if (!ok && lane == 0 && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
-
     if (dq) {
         __syncthreads();
         const bool valid = threadIdx.x < nblk;
