@@ -340,9 +340,14 @@ Codebook to_cb(const float *c) {
 int run_adapter_down(const Dims &d, const uint16_t *X, const uint16_t *A, uint16_t *Apad,
                      const uint16_t *ph, const uint16_t *pl, float *Tpart, float *T32, float s,
                      uint16_t *sT, uint32_t *status, cudaStream_t st) {
-    RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st));
+    // A already has the padded row length (r a multiple of 16): use it in place
+    const uint16_t *Ause = A;
+    if (d.r != d.rp || !aligned16(A)) {
+        RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st));
+        Ause = Apad;
+    }
     ProdPlan plan;
-    RC(run_prod(prod_T(d, X, Apad, ph, pl), d.mma_large, Tpart, status, st, &plan));
+    RC(run_prod(prod_T(d, X, Ause, ph, pl), d.mma_large, Tpart, status, st, &plan));
     if (sT && cudaMemsetAsync(sT, 0, d.M * d.rp64 * sizeof(uint16_t), st) != cudaSuccess)
         return QLORA_ECUDA;
     return launch_reduce(Tpart, plan.splits, d.M, plan.Qp, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
@@ -532,8 +537,11 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
         if (d.small) {
             RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st));
         } else if (!d.mma_large) {
-            int rcx = launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st);
-            if (rcx == QLORA_OK) rcx = launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, w.Aext, dX, d_status, st);
+            // the extension operand is A itself when no padding, pooling or scaling applies
+            const bool direct = d.g == 1 && r == d.rp64 && aligned16(A);
+            int rcx = direct ? QLORA_OK : launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st);
+            if (rcx == QLORA_OK)
+                rcx = launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, direct ? A : w.Aext, dX, d_status, st);
             if (rcx != QLORA_OK) {
                 if (ev_fork) cudaEventDestroy(ev_fork);
                 if (ev_join) cudaEventDestroy(ev_join);
