@@ -9,151 +9,240 @@
 // w_hat = RN_bf16(RN32(a_hat c_q)) is the dequantized weight; the rank-r sum
 // is an fp32 MMA.  HBM-bound: 0.52 bytes in and 2 bytes out per weight.
 //
-// grid (ceil(Dout/256), ceil(Din/256)), 16 warps.  Warp w owns rows
-// [256 bx + 16 w, +16) and walks the CTA's 256 columns one 64-block at a
-// time.  256 x 256 tiles keep the staged operands small next to the
-// output (B^T once per CTA, A once per block of 64 columns).  MMA m16n8k16
-// with the 16 rows as M, 8 columns as N and 16 ranks as K: the A operand is
-// B^T, staged transposed in shared memory once per CTA; the B operand is the
-// adapter A, whose 64 rows for the current block are staged (one row when
-// pooled: the block shares it) with cp.async into one of two buffers while
-// the previous block computes.  Row pitches of ceil64(r) + 8 elements
-// (= 16 mod 128 bytes) keep the 32-bit fragment loads on distinct banks.  The accumulator fragment of lane
-// (g, t) holds columns 8nt + 2t, +1 of rows g and g+8: byte 4nt + t of each
-// row's 32 packed bytes, i.e. byte t of word nt, decoded in place.
+// Persistent: one CTA of 16 warps per SM walks a contiguous range of units,
+// a unit being 256 output rows x one 64-input block, row tile by row tile.
+// Warp w owns rows [256 rt + 16 w, +16) of row tile rt.  MMA m16n8k16 with
+// the 16 rows as M, 8 inputs as N and 16 ranks as K.
+//  - The A operand is B^T: the tile's B rows (ranks x 256 outputs) are staged
+//    as they lie in memory, once per row tile, and read with ldmatrix.trans.
+//  - The B operand is the adapter A: the 64 rows of each unit (one row when
+//    pooled: the block shares it) go by cp.async into a ring of three buffers
+//    (two when the rank is too large for three), two units ahead of use, so
+//    one barrier per unit both publishes a buffer and frees the oldest.
+//  - The inputs of a block are permuted among the 8 MMA tiles so that lane
+//    (g, t) of tile nt holds inputs 16t + 2nt and +1: each lane owns 16
+//    consecutive inputs of its two rows, i.e. 8 consecutive packed bytes (one
+//    8-byte load per row) and 32 consecutive output bytes (two 16-byte
+//    stores).  Staged row 8nt + n holds adapter row 16(n/2) + 2nt + n%2, so
+//    each tile's 8 rows are adjacent for ldmatrix.
+//  - The next unit's packed bytes and scales are loaded one unit ahead.
+// Row pitches of (ranks + 8) and (256 + 8) elements are odd multiples of 16
+// bytes, which keeps ldmatrix's eight 16-byte rows on distinct banks.
 #include "common.cuh"
 
 namespace qlora {
 namespace {
 
-constexpr int kMgRows = 256, kMgCols = 256, kMgThreads = 512;
+constexpr size_t kMgSmemMax = 227 * 1024 - 1024;    // opt-in limit less the static part
+constexpr int kMgRows = 256, kMgThreads = 512, kMgBPitch = kMgRows + 8;
 
-__device__ __forceinline__ int mg_pitch(int r) { return (r + 63) / 64 * 64 + 8; }
+__host__ __device__ __forceinline__ int mg_rp(int r) { return (r + 15) / 16 * 16; }
+__host__ __device__ __forceinline__ size_t mg_smem(int r, int nbuf) {
+    return ((size_t)mg_rp(r) * kMgBPitch + (size_t)nbuf * 64 * (mg_rp(r) + 8)) * 2;
+}
+
+// Adapter row k of a block -> its staged row (tile (k/2) % 8, column 2(k/16) + k%2).
+__device__ __forceinline__ int mg_slot(int k) { return 8 * ((k >> 1) & 7) + 2 * (k >> 4) + (k & 1); }
+
+// Packed bytes and raw scale of one row of one unit: a_hat = RN32(code * f)
+// (code = 1, f = absmax without double quantization; both exact as before).
+struct MgRow {
+    uint2 p;
+    uint32_t code;
+    float f;
+};
+
+__device__ __forceinline__ MgRow mg_load(const uint8_t *__restrict__ packed, const ScaleSrc &sc,
+                                         int64_t row, int64_t Dout, int64_t Din, int64_t kc, int t) {
+    MgRow m{make_uint2(0u, 0u), 0u, 0.f};
+    if (row < Dout) {
+        m.p = __ldg(reinterpret_cast<const uint2 *>(packed + row * (Din / 2) + kc / 2) + t);
+        const int64_t b = row * (Din / 64) + kc / 64;
+        if (sc.dq) {
+            m.code = __ldg(sc.code + b);
+            m.f = __ldg(sc.step + (b >> 8));
+        } else {
+            m.code = 1u;
+            m.f = __ldg(sc.absmax + b);
+        }
+    }
+    return m;
+}
+
+// B rows 0 .. rp-1 of row tile rt into sB (zeros past r and past Dout).
+__device__ __forceinline__ void mg_stage_b(uint16_t *sB, const uint16_t *__restrict__ B, int rt, int r,
+                                           int rp, int64_t Dout, bool bvec, int tid) {
+    const int64_t n0 = (int64_t)rt * kMgRows;
+    if (bvec) {   // Dout % 8 == 0 and B 16-byte aligned: whole 16-byte pieces are in or out
+        for (int i = tid; i < rp * (kMgRows / 8); i += kMgThreads) {
+            const int j = i / (kMgRows / 8), v = i % (kMgRows / 8);
+            const bool ok = j < r && n0 + 8 * v < Dout;
+            cp_async16(sB + j * kMgBPitch + 8 * v, ok ? B + (int64_t)j * Dout + n0 + 8 * v : B, ok);
+        }
+    } else {
+        for (int i = tid; i < rp * kMgRows; i += kMgThreads) {
+            const int j = i / kMgRows, n = i % kMgRows;
+            sB[j * kMgBPitch + n] = (j < r && n0 + n < Dout) ? B[(int64_t)j * Dout + n0 + n] : 0;
+        }
+    }
+    cp_async_commit();
+}
+
+// Adapter rows of unit u into buffer buf, in staged-row order (one group
+// committed even when u is past the CTA's range, to keep the group count).
+__device__ __forceinline__ void mg_stage_a(uint16_t *sA, const uint16_t *__restrict__ A, int u, int u1,
+                                           int buf, int nblk, int r, int gp, int pitch, bool avec,
+                                           int tid) {
+    if (u < u1) {
+        const int arows = gp == 1 ? 64 : 1;
+        const int64_t arow0 = (int64_t)(u % nblk) * 64 / gp;
+        uint16_t *dst = sA + buf * 64 * pitch;
+        if (avec) {   // r % 8 == 0 and A 16-byte aligned
+            const int nv = r / 8;
+            for (int i = tid; i < arows * nv; i += kMgThreads) {
+                const int k = i / nv, v = i - k * nv;
+                cp_async16(dst + (gp == 1 ? mg_slot(k) : 0) * pitch + 8 * v, A + (arow0 + k) * r + 8 * v,
+                           true);
+            }
+        } else {
+            for (int i = tid; i < arows * r; i += kMgThreads) {
+                const int k = i / r, j = i - k * r;
+                dst[(gp == 1 ? mg_slot(k) : 0) * pitch + j] = A[(arow0 + k) * r + j];
+            }
+        }
+    }
+    cp_async_commit();
+}
 
 __global__ void __launch_bounds__(kMgThreads, 1)
 k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
         const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, int r, int gp, float sg,
-        int64_t Dout, int64_t Din, uint16_t *__restrict__ W_out) {
+        int64_t Dout, int64_t Din, int nbuf, uint16_t *__restrict__ W_out) {
     extern __shared__ __align__(16) uint16_t msm[];
-    const int pitch = mg_pitch(r);
-    uint16_t *sBt = msm;                         // [64 rows][pitch]: B^T
-    uint16_t *sA2 = msm + kMgRows * pitch;       // [2][64 inputs][pitch]: A rows of a block
     __shared__ float cbs[16];
-    const int rp = (r + 15) / 16 * 16;
-    const int64_t nb0 = (int64_t)blockIdx.x * kMgRows;
-    if (threadIdx.x == 0) {
+    const int rp = mg_rp(r), pitch = rp + 8;
+    uint16_t *sB = msm;                              // [rp ranks][kMgBPitch]: B of the row tile
+    uint16_t *sA = msm + rp * kMgBPitch;             // [nbuf][64][pitch]: adapter rows of a unit
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    if (tid == 0) {   // constant indices: a dynamic index into the parameter would copy it to the stack
 #pragma unroll
         for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
     }
-    for (int i = threadIdx.x; i < rp * kMgRows; i += blockDim.x) {
-        const int j = i / kMgRows, n = i % kMgRows;     // consecutive threads: consecutive n
-        uint16_t v = 0;
-        if (j < r && nb0 + n < Dout) v = B[(int64_t)j * Dout + nb0 + n];
-        sBt[n * pitch + j] = v;
+
+    const int nblk = (int)(Din / 64);
+    const int64_t units = (Dout + kMgRows - 1) / kMgRows * nblk;
+    const int u0 = (int)(units * blockIdx.x / gridDim.x), u1 = (int)(units * (blockIdx.x + 1) / gridDim.x);
+    if (u0 >= u1) return;
+
+    const bool bvec = (Dout & 7) == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0;
+    const bool avec = (r & 7) == 0 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0;
+
+    // ranks r .. rp-1 of every adapter buffer stay zero (no copy reaches them)
+    for (int i = tid; i < nbuf * 64 * (rp - r); i += kMgThreads) {
+        const int row = i / (rp - r), j = r + i % (rp - r);
+        sA[row * pitch + j] = 0;
     }
+    const int ahead = nbuf - 1;                      // units staged ahead of use
+    int cur_rt = u0 / nblk;
+    mg_stage_b(sB, B, cur_rt, r, rp, Dout, bvec, tid);
+    for (int d = 0; d < ahead; ++d) mg_stage_a(sA, A, u0 + d, u1, d, nblk, r, gp, pitch, avec, tid);
 
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int64_t ra = nb0 + 16 * warp + g, rb = ra + 8;   // this lane's two rows
-    const bool vec = (r & 7) == 0 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0;
-    // ranks r .. rp-1 of the staged A rows stay zero (the copies never reach them)
-    for (int row = warp; row < 2 * 64; row += 16)
-        for (int j = r + lane; j < rp; j += 32) sA2[row * pitch + j] = 0;
-    const int64_t nbr = Din / 64;
-    const uint16_t *bt0 = sBt + (16 * warp + g) * pitch + 2 * t;
-    const uint16_t *bt1 = bt0 + 8 * pitch;
-    const int arows = gp == 1 ? 64 : 1;              // staged A rows per block
-    const int astep = gp == 1 ? 8 * pitch : 0;       // next n tile: 8 inputs on
-    // A rows of block c into buffer c % 2: cp.async 16-byte pieces (r % 8 == 0,
-    // A 16-byte aligned), else plain loads
-    auto stage = [&](int c) {
-        const int64_t kc = (int64_t)blockIdx.y * kMgCols + 64 * c;
-        uint16_t *sA = sA2 + (c & 1) * 64 * pitch;
-        const int64_t arow0 = kc / gp;
-        if (vec) {
-            const int nv = r / 8;
-            for (int i = threadIdx.x; i < arows * nv; i += kMgThreads) {
-                const int row = i / nv, v = i % nv;
-                cp_async16(sA + row * pitch + 8 * v, A + (arow0 + row) * r + 8 * v, true);
-            }
-            cp_async_commit();
-        } else {
-            for (int row = warp; row < arows; row += 16)
-                for (int j = lane; j < r; j += 32) sA[row * pitch + j] = A[(arow0 + row) * r + j];
-        }
-    };
-    stage(0);
+    // ldmatrix row addresses of this lane (element offsets; ks and the tile pair added later)
+    const int lda = (((lane >> 4) << 3) + (lane & 7)) * kMgBPitch + 16 * warp + 8 * ((lane >> 3) & 1);
+    const int ldb = (gp == 1 ? (8 * (lane >> 4) + (lane & 7)) * pitch : 0) + 8 * ((lane >> 3) & 1);
+    const int ldb_np = gp == 1 ? 16 * pitch : 0;
 
-    for (int c = 0; c < kMgCols / 64; ++c) {
-        const int64_t kc = (int64_t)blockIdx.y * kMgCols + 64 * c;   // this 64-block's first input
-        if (kc >= Din) break;
-        const bool next = c + 1 < kMgCols / 64 && kc + 64 < Din;
-        if (c) __syncthreads();                      // block c-1's reads of buffer (c+1) % 2 done
-        if (next) stage(c + 1);
-        const uint16_t *sa = sA2 + (c & 1) * 64 * pitch + (gp == 1 ? g : 0) * pitch + 2 * t;
-        // this lane's packed words: rows ra, rb, 32 bytes each
-        uint32_t pw[2][8];
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int64_t row = hr ? rb : ra;
-            uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-            if (row < Dout) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(packed + row * (Din / 2) + kc / 2);
-                lo = __ldg(src);
-                hi = __ldg(src + 1);
-            }
-            pw[hr][0] = lo.x, pw[hr][1] = lo.y, pw[hr][2] = lo.z, pw[hr][3] = lo.w;
-            pw[hr][4] = hi.x, pw[hr][5] = hi.y, pw[hr][6] = hi.z, pw[hr][7] = hi.w;
+    int rt = cur_rt, cblk = u0 - cur_rt * nblk;
+    MgRow nxt0, nxt1;
+    {
+        const int64_t ra = (int64_t)rt * kMgRows + 16 * warp + g;
+        nxt0 = mg_load(packed, sc, ra, Dout, Din, 64 * (int64_t)cblk, t);
+        nxt1 = mg_load(packed, sc, ra + 8, Dout, Din, 64 * (int64_t)cblk, t);
+    }
+    int buf = 0;
+    for (int u = u0; u < u1; ++u) {
+        const int64_t kc = 64 * (int64_t)cblk;
+        const int64_t ra = (int64_t)rt * kMgRows + 16 * warp + g;
+        const MgRow cur0 = nxt0, cur1 = nxt1;
+        int nrt = rt, ncb = cblk + 1;                // the next unit
+        if (ncb == nblk) ncb = 0, ++nrt;
+        if (u + 1 < u1) {
+            const int64_t na = (int64_t)nrt * kMgRows + 16 * warp + g;
+            nxt0 = mg_load(packed, sc, na, Dout, Din, 64 * (int64_t)ncb, t);
+            nxt1 = mg_load(packed, sc, na + 8, Dout, Din, 64 * (int64_t)ncb, t);
         }
-        const float aha = ra < Dout ? load_scale(sc, ra * nbr + kc / 64) : 0.f;
-        const float ahb = rb < Dout ? load_scale(sc, rb * nbr + kc / 64) : 0.f;
-        if (vec) {
-            if (next) cp_async_wait<1>();            // block c's copies landed, c+1's may fly
-            else cp_async_wait<0>();
+        if (rt != cur_rt) {                          // new row tile: restage B
+            __syncthreads();                         // every warp is past its last read of sB
+            mg_stage_b(sB, B, rt, r, rp, Dout, bvec, tid);
+            cp_async_wait<0>();
+            cur_rt = rt;
         }
-        __syncthreads();                             // sA of block c (and, first time, sBt) ready
+        if (ahead == 2) cp_async_wait<1>();          // this unit's rows landed; the next may fly
+        else cp_async_wait<0>();
+        __syncthreads();                             // ... for every thread; buffer (buf-1) is free
+        mg_stage_a(sA, A, u + ahead, u1, buf == 0 ? nbuf - 1 : buf - 1, nblk, r, gp, pitch, avec, tid);
+
+        const uint16_t *sAc = sA + buf * 64 * pitch;
         float acc[8][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
         for (int ks = 0; ks < rp; ks += 16) {
-            const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(bt0 + ks),
-                                   *reinterpret_cast<const uint32_t *>(bt1 + ks),
-                                   *reinterpret_cast<const uint32_t *>(bt0 + ks + 8),
-                                   *reinterpret_cast<const uint32_t *>(bt1 + ks + 8)};
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, sB + lda + ks * kMgBPitch);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b4[4];
+                ldmatrix_x4(b4, sAc + ldb + np * ldb_np + ks);
+                const uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
+                mma_bf16_16816(acc[2 * np], a, b0);
+                mma_bf16_16816(acc[2 * np + 1], a, b1);
+            }
+        }
+        // epilogue: row ra (hr 0) / ra + 8 (hr 1), inputs kc + 16t + 2nt, +1 = byte 8t + nt
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int64_t row = ra + 8 * hr;
+            if (row >= Dout) continue;
+            const MgRow m = hr ? cur1 : cur0;
+            const float ah = __fmul_rn((float)m.code, m.f);
+            uint32_t o[8];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
-                // B operand: ranks ks + 2t, +1 (and +8, +9) of input kc + 8nt + g
-                const uint16_t *ar = sa + nt * astep + ks;
-                const uint32_t bb[2] = {*reinterpret_cast<const uint32_t *>(ar),
-                                        *reinterpret_cast<const uint32_t *>(ar + 8)};
-                mma_bf16_16816(acc[nt], a, bb);
-            }
-        }
-        // epilogue: rows ra / rb, inputs kc + 8nt + 2t and +1 (byte t of word nt)
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int64_t col = kc + 8 * nt + 2 * t;
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int64_t row = hr ? rb : ra;
-                if (row >= Dout) continue;
-                const float ah = hr ? ahb : aha;
-                const uint32_t byte = (pw[hr][nt] >> (8 * t)) & 0xffu;
+                const uint32_t byte = ((nt < 4 ? m.p.x : m.p.y) >> (8 * (nt & 3))) & 0xffu;
                 const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(ah, cbs[byte >> 4])));
                 const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(ah, cbs[byte & 15])));
-                const float v0 = fmaf(sg, acc[nt][2 * hr], w0);
-                const float v1 = fmaf(sg, acc[nt][2 * hr + 1], w1);
-                *reinterpret_cast<uint32_t *>(W_out + row * Din + col) = bf16x2_bits(v0, v1);
+                o[nt] = bf16x2_bits(fmaf(sg, acc[nt][2 * hr], w0), fmaf(sg, acc[nt][2 * hr + 1], w1));
             }
+            uint4 *dst = reinterpret_cast<uint4 *>(W_out + row * Din + kc + 16 * t);
+            __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
         }
+        rt = nrt, cblk = ncb;
+        buf = buf + 1 == nbuf ? 0 : buf + 1;
     }
+    cp_async_wait<0>();                              // no copy outlives the CTA
+}
+
+int mg_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
 }
 
 }  // namespace
 
-size_t merge_smem_bytes(int r) { return (size_t)(kMgRows + 2 * 64) * ((r + 63) / 64 * 64 + 8) * 2; }
+size_t merge_smem_bytes(int r) {
+    const size_t three = mg_smem(r, 3);
+    return three <= kMgSmemMax ? three : mg_smem(r, 2);
+}
 
 int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, const uint16_t *B,
                  int r, int gp, float s, uint16_t *W_out, cudaStream_t st) {
@@ -161,10 +250,13 @@ int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, c
     if (Dout * Din == 0) return QLORA_OK;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
     const size_t smem = merge_smem_bytes(r);
+    const int nbuf = smem == mg_smem(r, 3) ? 3 : 2;
     cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dim3 grid((unsigned)((Dout + kMgRows - 1) / kMgRows), (unsigned)((Din + kMgCols - 1) / kMgCols));
+    const int64_t units = (Dout + kMgRows - 1) / kMgRows * (Din / 64);
+    const unsigned grid = (unsigned)(units < mg_sms() ? units : mg_sms());
     prof_begin(kProfMerge, st);
-    k_merge<<<grid, kMgThreads, smem, st>>>(q.packed, sc, cb, A, B, r, gp, s / (float)gp, Dout, Din, W_out);
+    k_merge<<<grid, kMgThreads, smem, st>>>(q.packed, sc, cb, A, B, r, gp, s / (float)gp, Dout, Din,
+                                            nbuf, W_out);
     prof_end(kProfMerge, st);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;

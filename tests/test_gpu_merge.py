@@ -33,6 +33,9 @@ def _case(orc, qlib, spec, cfg, lin=0):
     (1024, 136, 100, True, 1),    # rank past 64 (two 64-wide B^T pitches)
     (512, 136, 8, True, 64),      # pooled adapter
     (4096, 4096, 16, True, 1),
+    (192, 204, 24, False, 1),     # Dout % 8 != 0: B staged element by element
+    (4096, 1024, 256, True, 1),   # largest rank: two adapter buffers; several units per CTA
+    (4096, 2048, 64, True, 64),   # pooled, several units and row tiles per CTA
 ])
 def test_merge_matches_oracle(orc, qlib, Din, Dout, r, dq, pool):
     spec = LinearSpec("m", Din, Dout, r, 2.0 * r, dq, pool_group=pool)
