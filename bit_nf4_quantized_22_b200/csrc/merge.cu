@@ -88,26 +88,34 @@ __device__ __forceinline__ void mg_stage_b(uint16_t *sB, const uint16_t *__restr
     cp_async_commit();
 }
 
-// Adapter rows of unit u into buffer buf, in staged-row order (one group
-// committed even when u is past the CTA's range, to keep the group count).
-__device__ __forceinline__ void mg_stage_a(uint16_t *sA, const uint16_t *__restrict__ A, int u, int u1,
-                                           int buf, int nblk, int r, int gp, int pitch, bool avec,
-                                           int tid) {
-    if (u < u1) {
+// Adapter rows of 64-input block blk into buffer buf, in staged-row order.
+// One group is committed even when there is no unit to stage, which keeps
+// the group count.  With one 16-byte piece per thread at most (the common
+// case, r <= 64), every thread moves the same piece of every unit, located
+// once at the start (dst, src: element offsets; dst < 0: no piece).
+struct MgCopy {
+    int dst, src;
+};
+
+__device__ __forceinline__ void mg_stage_a(uint16_t *sA, const uint16_t *__restrict__ A, bool valid, int blk,
+                                           int buf, int r, int gp, int pitch, bool avec, bool one,
+                                           MgCopy cp, int tid) {
+    if (valid) {
         const int arows = gp == 1 ? 64 : 1;
-        const int64_t arow0 = (int64_t)(u % nblk) * 64 / gp;
+        const uint16_t *src = A + (int64_t)blk * 64 / gp * r;
         uint16_t *dst = sA + buf * 64 * pitch;
-        if (avec) {   // r % 8 == 0 and A 16-byte aligned
+        if (one) {
+            if (cp.dst >= 0) cp_async16(dst + cp.dst, src + cp.src, true);
+        } else if (avec) {   // r % 8 == 0 and A 16-byte aligned
             const int nv = r / 8;
             for (int i = tid; i < arows * nv; i += kMgThreads) {
                 const int k = i / nv, v = i - k * nv;
-                cp_async16(dst + (gp == 1 ? mg_slot(k) : 0) * pitch + 8 * v, A + (arow0 + k) * r + 8 * v,
-                           true);
+                cp_async16(dst + (gp == 1 ? mg_slot(k) : 0) * pitch + 8 * v, src + k * r + 8 * v, true);
             }
         } else {
             for (int i = tid; i < arows * r; i += kMgThreads) {
                 const int k = i / r, j = i - k * r;
-                dst[(gp == 1 ? mg_slot(k) : 0) * pitch + j] = A[(arow0 + k) * r + j];
+                dst[(gp == 1 ? mg_slot(k) : 0) * pitch + j] = src[k * r + j];
             }
         }
     }
@@ -145,8 +153,19 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
     }
     const int ahead = nbuf - 1;                      // units staged ahead of use
     int cur_rt = u0 / nblk;
+    const int arows = gp == 1 ? 64 : 1;
+    const bool one = avec && arows * (r / 8) <= kMgThreads;
+    MgCopy cp{-1, 0};
+    if (one && tid < arows * (r / 8)) {
+        const int k = tid / (r / 8), v = tid - k * (r / 8);
+        cp = MgCopy{(gp == 1 ? mg_slot(k) : 0) * pitch + 8 * v, k * r + 8 * v};
+    }
     mg_stage_b(sB, B, cur_rt, r, rp, Dout, bvec, tid);
-    for (int d = 0; d < ahead; ++d) mg_stage_a(sA, A, u0 + d, u1, d, nblk, r, gp, pitch, avec, tid);
+    int sblk = u0 - cur_rt * nblk;                   // block of the next unit to stage
+    for (int d = 0; d < ahead; ++d) {
+        mg_stage_a(sA, A, u0 + d < u1, sblk, d, r, gp, pitch, avec, one, cp, tid);
+        if (++sblk == nblk) sblk = 0;
+    }
 
     // ldmatrix row addresses of this lane (element offsets; ks and the tile pair added later)
     const int lda = (((lane >> 4) << 3) + (lane & 7)) * kMgBPitch + 16 * warp + 8 * ((lane >> 3) & 1);
@@ -181,7 +200,9 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
         if (ahead == 2) cp_async_wait<1>();          // this unit's rows landed; the next may fly
         else cp_async_wait<0>();
         __syncthreads();                             // ... for every thread; buffer (buf-1) is free
-        mg_stage_a(sA, A, u + ahead, u1, buf == 0 ? nbuf - 1 : buf - 1, nblk, r, gp, pitch, avec, tid);
+        mg_stage_a(sA, A, u + ahead < u1, sblk, buf == 0 ? nbuf - 1 : buf - 1, r, gp, pitch, avec, one, cp,
+                   tid);
+        if (++sblk == nblk) sblk = 0;
 
         const uint16_t *sAc = sA + buf * 64 * pitch;
         float acc[8][4];
@@ -212,9 +233,9 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const uint32_t byte = ((nt < 4 ? m.p.x : m.p.y) >> (8 * (nt & 3))) & 0xffu;
-                const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(ah, cbs[byte >> 4])));
-                const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(ah, cbs[byte & 15])));
-                o[nt] = bf16x2_bits(fmaf(sg, acc[nt][2 * hr], w0), fmaf(sg, acc[nt][2 * hr + 1], w1));
+                // both weights rounded to bf16 by one paired conversion
+                const uint32_t w = bf16x2_bits(__fmul_rn(ah, cbs[byte >> 4]), __fmul_rn(ah, cbs[byte & 15]));
+                o[nt] = bf16x2_bits(fmaf(sg, acc[nt][2 * hr], bf16_lo(w)), fmaf(sg, acc[nt][2 * hr + 1], bf16_hi(w)));
             }
             uint4 *dst = reinterpret_cast<uint4 *>(W_out + row * Din + kc + 16 * t);
             __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
