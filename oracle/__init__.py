@@ -58,9 +58,11 @@ def _L():
         lib.orc_nf4_codebook.restype = None
         lib.orc_nf4_codebook.argtypes = [ctypes.c_double, P]
         lib.orc_quantize.restype = ctypes.c_int
-        lib.orc_quantize.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        lib.orc_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
+                                     P]
         lib.orc_dequantize.restype = None
-        lib.orc_dequantize.argtypes = [i64, i64, P, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
+        lib.orc_dequantize.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
+                                       P, P]
         lib.orc_adapter_down.restype = None
         lib.orc_adapter_down.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, P]
         lib.orc_forward.restype = None
@@ -118,6 +120,7 @@ class QuantizedWeight:
     codes: np.ndarray | None      # uint8 [nb]
     steps: np.ndarray | None      # float32 [ceil(nb/256)]
     status: int
+    block: int = BLOCK            # weights per first-level scale
 
     @property
     def nbytes(self) -> int:
@@ -129,27 +132,27 @@ class QuantizedWeight:
 
 
 def quantize(W: np.ndarray, codebook: np.ndarray, double_quant: bool,
-             dq_group: int = DQ_GROUP) -> QuantizedWeight:
+             dq_group: int = DQ_GROUP, block: int = BLOCK) -> QuantizedWeight:
     W = _c(W, np.float32)
     rows, cols = W.shape
-    assert (rows * cols) % BLOCK == 0
+    assert block % 2 == 0 and cols % block == 0
     cb = _c(codebook, np.float32)
-    nb = rows * cols // BLOCK
+    nb = rows * cols // block
     packed = np.zeros(rows * cols // 2, dtype=np.uint8)
     absmax = None if double_quant else np.zeros(nb, dtype=np.float32)
     codes = np.zeros(nb, dtype=np.uint8) if double_quant else None
     ng = (nb + dq_group - 1) // dq_group
     steps = np.zeros(ng, dtype=np.float32) if double_quant else None
-    st = _L().orc_quantize(_p(W), rows, cols, _p(cb), int(double_quant), dq_group,
+    st = _L().orc_quantize(_p(W), rows, cols, block, _p(cb), int(double_quant), dq_group,
                            _p(packed), _p(absmax), _p(codes), _p(steps))
-    return QuantizedWeight(rows, cols, double_quant, packed, absmax, codes, steps, int(st))
+    return QuantizedWeight(rows, cols, double_quant, packed, absmax, codes, steps, int(st), block)
 
 
 def dequantize(q: QuantizedWeight, codebook: np.ndarray, dq_group: int = DQ_GROUP) -> np.ndarray:
     """bf16 bit patterns [rows, cols]."""
     cb = _c(codebook, np.float32)
     out = np.zeros((q.rows, q.cols), dtype=np.uint16)
-    _L().orc_dequantize(q.rows, q.cols, _p(cb), int(q.double_quant), dq_group, _p(q.packed),
+    _L().orc_dequantize(q.rows, q.cols, q.block, _p(cb), int(q.double_quant), dq_group, _p(q.packed),
                         _p(q.absmax), _p(q.codes), _p(q.steps), _p(out))
     return out
 

@@ -179,7 +179,10 @@ static int nearest_level(float w, float a, const float cb[16], int zero_idx) {
     return best;
 }
 
-/* Quantize Wt:[rows, cols] (fp32, row-major; rows*cols a multiple of 64).
+/* Quantize Wt:[rows, cols] (fp32, row-major) in blocks of `block` weights
+ * (64 by default; 32, 128 or 256 trade scale resolution against metadata,
+ * [CSDN] 5.1).  The row-major flattening is cut into consecutive blocks; cols
+ * is a multiple of block, so every block lies inside one row.
  *   packed  [rows*cols/2]        two indices per byte, high nibble first
  *   absmax  [nb]                 fp32 block absmax (used when dq == 0)
  *   codes   [nb], steps [ceil(nb/dq_group)]   (used when dq != 0)
@@ -196,29 +199,29 @@ static int nearest_level(float w, float a, const float cb[16], int zero_idx) {
  * [0,255] (f = 0 gives code 0).  The weights themselves are encoded once,
  * with the true a_b ([CSDN] 7: the second pass quantizes the scales, not
  * the weights). */
-int orc_quantize(const float *W, int64_t rows, int64_t cols, const float cb[16],
+int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const float cb[16],
                  int dq, int dq_group, uint8_t *packed, float *absmax,
                  uint8_t *codes, float *steps) {
     const int64_t n = rows * cols;
-    const int64_t nb = n / 64;
+    const int64_t nb = n / block;
     const int zero_idx = zero_level_index(cb);
     int status = 0;
     float *a_all = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
 #pragma omp parallel for schedule(static) reduction(| : status)
     for (int64_t b = 0; b < nb; ++b) {
-        const float *wb = W + b * 64;
+        const float *wb = W + b * block;
         double a = 0.0;
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < block; ++i) {
             if (!isfinite(wb[i])) status |= ORC_STATUS_NONFINITE;
             double m = fabs((double)wb[i]);
             if (m > a) a = m;
         }
         float af = (float)a; /* exact: a is the magnitude of an fp32 value */
         a_all[b] = af;
-        for (int i = 0; i < 64; i += 2) {
+        for (int i = 0; i < block; i += 2) {
             int q0 = nearest_level(wb[i], af, cb, zero_idx);
             int q1 = nearest_level(wb[i + 1], af, cb, zero_idx);
-            packed[(b * 64 + i) / 2] = (uint8_t)((q0 << 4) | q1);
+            packed[(b * block + i) / 2] = (uint8_t)((q0 << 4) | q1);
         }
         if (!dq) absmax[b] = af;
     }
@@ -264,15 +267,15 @@ static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
 }
 
 /* Dequantize ([CSDN] 5.2 w_hat = a * c_q; 8.6 the result is in the compute
- * dtype, bf16 here): w_hat = RN_bf16(RN_fp32(a_hat * c_q)).  Output is bf16
- * bit patterns, [rows, cols]. */
-void orc_dequantize(int64_t rows, int64_t cols, const float cb[16], int dq,
+ * dtype, bf16 here): w_hat = RN_bf16(RN_fp32(a_hat * c_q)), element e taking
+ * the scale of block e / block.  Output is bf16 bit patterns, [rows, cols]. */
+void orc_dequantize(int64_t rows, int64_t cols, int block, const float cb[16], int dq,
                     int dq_group, const uint8_t *packed, const float *absmax,
                     const uint8_t *codes, const float *steps, uint16_t *out) {
     const int64_t n = rows * cols;
 #pragma omp parallel for schedule(static)
     for (int64_t e = 0; e < n; ++e) {
-        int64_t b = e / 64;
+        int64_t b = e / block;
         uint8_t byte = packed[e / 2];
         int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
         float ah = block_scale(b, dq, dq_group, absmax, codes, steps);

@@ -305,3 +305,97 @@ def test_dq_overhead_partial_group(orc):
     W = np.ones((3, 64 * 100), dtype=np.float32)       # nb = 300
     q = orc.quantize(W, cb, double_quant=True)
     assert q.codes.size == 300 and q.steps.size == 2
+
+
+# ---------------------------------------------------------------- other block sizes
+# The article names 64 as the common default and weighs smaller blocks (finer
+# scales, more metadata) against larger ones (less metadata, outliers reach
+# further) in section 5.1; sizes 32, 128 and 256 are pinned here the same way.
+
+@pytest.mark.parametrize("block", [32, 128, 256])
+def test_block_sizes_bruteforce(orc, block):
+    """Every block of `block` consecutive weights of a row takes its own absmax
+    and exact nearest levels (brute force in rationals)."""
+    rng = np.random.default_rng(100 + block)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_normal((3, 2 * 256)) * 0.02).astype(np.float32)
+    W[1, block:2 * block] = rng.standard_t(3, block).astype(np.float32)   # one heavy block
+    W[2, :block] = 0.0                                                    # an all-zero block
+    q = orc.quantize(W, cb, double_quant=False, block=block)
+    assert q.status == 0 and q.block == block
+    flat = W.reshape(-1)
+    assert q.absmax.size == flat.size // block
+    idx = unpack(q.packed, flat.size)
+    for b in range(flat.size // block):
+        blk = flat[b * block:(b + 1) * block]
+        a = np.float32(np.max(np.abs(blk)))
+        assert q.absmax[b] == a, b
+        for i in range(0, block, 7):   # a stride through every block, both nibbles
+            assert idx[b * block + i] == exact_argmin(blk[i], a, cb), (b, i)
+        assert idx[b * block + block - 1] == exact_argmin(blk[-1], a, cb)
+
+
+def test_block_size_changes_only_the_scales(orc):
+    """When every 32-weight sub-block of a 256-block holds the 256-block's
+    absmax, all block sizes give the same indices; when the sub-blocks' maxima
+    differ, the smaller blocks resolve the small-valued ones more finely."""
+    rng = np.random.default_rng(11)
+    cb = orc.nf4_codebook()
+    W = (rng.uniform(-0.9, 0.9, (4, 1024)) * 0.05).astype(np.float32)
+    W.reshape(-1, 32)[:, 5] = np.float32(0.05)          # the same absmax in every sub-block
+    qs = {b: orc.quantize(W, cb, double_quant=False, block=b) for b in (32, 64, 128, 256)}
+    for b in (64, 128, 256):
+        assert np.array_equal(qs[b].packed, qs[32].packed), b
+        assert np.all(qs[b].absmax == np.float32(0.05))
+    V = W.copy()
+    V.reshape(-1, 32)[1::2] *= np.float32(0.01)          # every other sub-block tiny
+    V.reshape(-1, 32)[1::2, 5] = np.float32(0.0005)
+    err = {}
+    for b in (32, 256):
+        q = orc.quantize(V, cb, double_quant=False, block=b)
+        rec = np.repeat(q.absmax.astype(np.float64), b) * cb.astype(np.float64)[unpack(q.packed, V.size)]
+        err[b] = np.abs(rec - V.reshape(-1)).reshape(-1, 32)[1::2].max()
+    # 32-blocks: within half the widest level gap of their own absmax 0.0005;
+    # 256-blocks: the tiny values fall to the zero level, a full 0.0005 off
+    gap = np.max(np.diff(cb.astype(np.float64))) / 2
+    assert err[32] <= 0.0005 * gap * (1 + 1e-6)
+    assert err[256] >= 0.0005 * 0.99
+
+
+@pytest.mark.parametrize("block", [32, 128, 256])
+def test_block_sizes_dequant_roundtrip_and_dq(orc, block):
+    """Weights that are exactly RN32(a_b * c_j) with a_b reached in each block
+    quantize to j and dequantize to RN_bf16 of themselves: a scale taken from
+    a wrong block would break it (the blocks' absmax differ by powers of two).
+    With double quantization the codes follow the brute-force rule over groups
+    of 256 blocks of this size."""
+    cb = orc.nf4_codebook()
+    rng = np.random.default_rng(200 + block)
+    nb = 2 * 256 + 16                                   # two full double-quant groups + a partial one
+    a = np.float32(2.0) ** rng.integers(-12, -2, nb).astype(np.float32)
+    j = rng.integers(0, 16, (nb, block))
+    j[:, 0] = 15                                        # the absmax itself (c_15 = 1)
+    W = np.array([[rn32(Fr(float(a[b])) * Fr(float(cb[jj]))) for jj in j[b]] for b in range(nb)],
+                 dtype=np.float32).reshape(-1, 8 * block)
+    nb_used = W.size // block
+    assert nb_used == nb
+    q = orc.quantize(W, cb, double_quant=False, block=block)
+    assert np.array_equal(q.absmax, a)
+    assert np.array_equal(unpack(q.packed, W.size), j.reshape(-1))
+    assert np.array_equal(orc.dequantize(q, cb).reshape(-1), bf16_of_f32(W.reshape(-1)))
+    qd = orc.quantize(W, cb, double_quant=True, block=block)
+    codes, steps = _expected_dq(list(a))
+    assert np.array_equal(qd.codes, codes) and np.array_equal(qd.steps, steps)
+    assert np.array_equal(qd.packed, q.packed)
+    # decoded scales RN32(code * f) of each block scale that block's levels
+    ahat = np.array([rn32(Fr(int(c)) * Fr(float(steps[i // 256]))) for i, c in enumerate(codes)],
+                    dtype=np.float32)
+    jf = j.reshape(-1)
+
+    def scaled(e):   # RN32(a_hat * c), with the IEEE sign of a zero product (+0 * negative = -0)
+        v = rn32(Fr(float(ahat[e // block])) * Fr(float(cb[jf[e]])))
+        return np.float32(-0.0) if v == 0 and cb[jf[e]] < 0 else v
+
+    expect = np.array([scaled(e) for e in range(0, jf.size, 97)], dtype=np.float32)
+    got = orc.dequantize(qd, cb).reshape(-1)[::97]
+    assert np.array_equal(got, bf16_of_f32(expect))
