@@ -467,7 +467,55 @@ def decode_lines(args, q, lib, torch, dev, hbm, flush):
             }
         del w
     res["merge"] = merge_line(q, lib, torch, dev, hbm, flush)
+    res["block_sizes"] = block_size_lines(q, lib, torch, dev, hbm, flush)
     return res
+
+
+def block_size_lines(q, lib, torch, dev, hbm, flush):
+    """nf4_quantize (double quantization) and nf4_dequantize of the 4096 x
+    11008 weight in blocks of 32, 64, 128 and 256: kernel time (library
+    events) and HBM fraction of the algorithmic bytes, L2 flushed before each
+    launch."""
+    import ctypes
+    spec = synth.CONFIGS[3]["linears"][0]
+    W = torch.from_numpy(synth.draw(spec, 1, 3, 0, which=("W",))["W"]).to(dev)
+    n = W.numel()
+    out = {}
+    for blk in (32, 64, 128, 256):
+        w = q.quantize(W, double_quant=True, block=blk)
+        deq = torch.empty(W.shape, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            q.quantize(W, double_quant=True, block=blk, out=w)
+            q.dequantize(w, out=deq)
+        reps = 10
+        torch.cuda.synchronize()
+        lib.qlora_profile_reset()
+        lib.qlora_profile_enable(1)
+        for _ in range(reps):
+            flush.zero_()
+            q.quantize(W, double_quant=True, block=blk, out=w)
+        torch.cuda.synchronize()
+        lib.qlora_profile_enable(0)
+        cnt, ms = ctypes.c_int64(), ctypes.c_double()
+        lib.qlora_profile_read(2, ctypes.byref(cnt), ctypes.byref(ms))
+        qms = ms.value / max(1, cnt.value)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record()
+            q.dequantize(w, out=deq)
+            e1.record()
+        torch.cuda.synchronize()
+        dms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[reps // 2]
+        meta = w.nbytes - n // 2
+        qbytes, dbytes = 4 * n + n // 2 + meta, n // 2 + meta + 2 * n
+        out[str(blk)] = {
+            "quantize_ms": qms, "quantize_frac_hbm": qbytes / (qms / 1e3) / 1e9 / hbm if qms > 0 else None,
+            "dequantize_ms": dms, "dequantize_frac_hbm": dbytes / (dms / 1e3) / 1e9 / hbm,
+            "metadata_bytes_per_weight": meta / n,
+            "kernel": "k_nf4_quantize_fast" if blk == 64 else "k_nf4_quantize_blk"}
+        del w, deq
+    return out
 
 
 def backward_line(q, lib, torch, dev, hbm, flush, spec, cfg, lin, w, A, B, x, M):

@@ -52,22 +52,23 @@ class NF4Weight:
     absmax: torch.Tensor | None = None     # fp32 [nb]
     codes: torch.Tensor | None = None      # uint8 [nb]
     steps: torch.Tensor | None = None      # fp32 [ceil(nb/256)]
+    block: int = BLOCK                     # weights per first-level scale (32, 64, 128, 256)
 
     @staticmethod
-    def empty(rows: int, cols: int, double_quant: bool, device="cuda") -> "NF4Weight":
-        nb = rows * cols // BLOCK
+    def empty(rows: int, cols: int, double_quant: bool, device="cuda", block: int = BLOCK) -> "NF4Weight":
+        nb = rows * cols // block
         packed = torch.empty(rows * cols // 2, dtype=torch.uint8, device=device)
         if double_quant:
             ng = (nb + DQ_GROUP - 1) // DQ_GROUP
             return NF4Weight(rows, cols, True, packed,
                              codes=torch.empty(nb, dtype=torch.uint8, device=device),
-                             steps=torch.empty(ng, dtype=torch.float32, device=device))
+                             steps=torch.empty(ng, dtype=torch.float32, device=device), block=block)
         return NF4Weight(rows, cols, False, packed,
-                         absmax=torch.empty(nb, dtype=torch.float32, device=device))
+                         absmax=torch.empty(nb, dtype=torch.float32, device=device), block=block)
 
     def c_struct(self) -> _lib.NF4WeightC:
         return _lib.NF4WeightC(
-            self.rows, self.cols, BLOCK, int(self.double_quant), DQ_GROUP, 0,
+            self.rows, self.cols, self.block, int(self.double_quant), DQ_GROUP, 0,
             self.packed.data_ptr(),
             self.absmax.data_ptr() if self.absmax is not None else None,
             self.codes.data_ptr() if self.codes is not None else None,
@@ -92,11 +93,13 @@ def check_codebook(codebook: torch.Tensor) -> int:
 
 
 def quantize(W: torch.Tensor, double_quant: bool = True, codebook: torch.Tensor | None = None,
-             status: torch.Tensor | None = None, out: NF4Weight | None = None) -> NF4Weight:
-    """nf4_quantize on W (fp32 [Dout, Din], CUDA)."""
+             status: torch.Tensor | None = None, out: NF4Weight | None = None,
+             block: int = BLOCK) -> NF4Weight:
+    """nf4_quantize on W (fp32 [Dout, Din], CUDA) in blocks of `block` weights
+    (32, 64, 128 or 256; the layer calls need 64)."""
     _need(W, torch.float32, "W", 2)
     rows, cols = W.shape
-    q = out if out is not None else NF4Weight.empty(rows, cols, double_quant, W.device)
+    q = out if out is not None else NF4Weight.empty(rows, cols, double_quant, W.device, block)
     qc = q.c_struct()
     rc = load().nf4_quantize(_ptr(W), ctypes.byref(qc), _cb_host(codebook), _ptr(status), _stream())
     _lib.check(rc, "nf4_quantize")

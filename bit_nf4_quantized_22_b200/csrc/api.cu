@@ -79,12 +79,20 @@ int check_codebook(const float *cb, int *zero_idx) {
     return QLORA_OK;
 }
 
-int check_weight(const nf4_weight_t *q, bool need_rows) {
+// codec: nf4_quantize / nf4_dequantize, which also take blocks of 32, 128
+// and 256 weights (cols a multiple of the block); every other call needs 64.
+int check_weight(const nf4_weight_t *q, bool need_rows, bool codec = false) {
     if (!q) return QLORA_EINVAL;
     if (q->rows < 0 || q->cols < 0) return QLORA_EINVAL;
     if (need_rows && q->rows < 1) return QLORA_EINVAL;
-    if (q->cols % 64 != 0) return QLORA_EINVAL;
-    if (q->block != 64) return QLORA_EUNSUPPORTED;
+    if (codec) {
+        if (q->block != 32 && q->block != 64 && q->block != 128 && q->block != 256)
+            return QLORA_EUNSUPPORTED;
+        if (q->cols % q->block != 0) return QLORA_EINVAL;
+    } else {
+        if (q->cols % 64 != 0) return QLORA_EINVAL;
+        if (q->block != 64) return QLORA_EUNSUPPORTED;
+    }
     if (q->double_quant != 0 && q->double_quant != 1) return QLORA_EINVAL;
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!q->packed || !aligned16(q->packed)) return QLORA_EINVAL;
@@ -383,7 +391,7 @@ int qlora_check_codebook(const float codebook[16]) { return check_codebook(codeb
 int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16],
                  uint32_t *d_status, void *stream) {
     int zi = 0;
-    RC(check_weight(q, false));
+    RC(check_weight(q, false, true));
     RC(check_codebook(codebook, &zi));
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!W || !aligned16(W)) return QLORA_EINVAL;
@@ -391,7 +399,7 @@ int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16]
 }
 
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out, void *stream) {
-    RC(check_weight(q, false));
+    RC(check_weight(q, false, true));
     RC(check_codebook(codebook, nullptr));
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!W_out || !aligned16(W_out)) return QLORA_EINVAL;

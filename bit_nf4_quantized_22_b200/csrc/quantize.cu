@@ -337,6 +337,165 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     }
 }
 
+// ------------------------------------------------------------------ other block sizes
+// Blocks of B = 32 V weights (V = 1, 4, 8: blocks of 32, 128, 256; the
+// article's section 5.1 trade of scale resolution against metadata).  One
+// CTA per double-quant group of 256 blocks; warp w takes blocks w, w + 8, ...
+// of the group, one whole block per warp with V weights per lane, four
+// blocks' loads issued together.  The decision per weight is the fast
+// kernel's (bin table, one exact compare against tau_j held by lane j) when
+// the table is usable and a lies in [2^-100, 2^100], else the branch-free
+// search; packing, absmax and double quantization as in the other kernels.
+//   V = 1: lane l holds weight l; bytes are paired across lanes by shuffles.
+//   V = 4: lane l holds weights 4l .. 4l+3 (bytes 2l, 2l+1).
+//   V = 8: lane l holds weights 4l .. 4l+3 and 128 + 4l .. 131 + 4l.
+constexpr int kQbThreads = 256, kQbUnroll = 4;
+
+template <int V, bool kExactHalf>
+__global__ void __launch_bounds__(kQbThreads)
+k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins, bool use_bins,
+                   int zero_idx, int dq, uint8_t *__restrict__ packed, float *__restrict__ absmax,
+                   uint8_t *__restrict__ codes, float *__restrict__ steps,
+                   uint32_t *__restrict__ status) {
+    constexpr int B = 32 * V;
+    __shared__ float s_a[kQbThreads];
+    __shared__ float s_cb[16];
+    __shared__ double s_half[16];
+    __shared__ uint32_t s_lut[32];
+    __shared__ float warp_max[kQbThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t b0 = (int64_t)blockIdx.x * 256;
+    const int nblk = (int)(nb - b0 < 256 ? nb - b0 : 256);
+    s_a[threadIdx.x] = 0.f;
+    if (threadIdx.x == 0) {   // constant indices keep the parameters out of local memory
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s_cb[j] = cb.c[j];
+#pragma unroll
+        for (int j = 0; j < 15; ++j) s_half[j] = bins.half[j];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s_lut[i] = (bins.nib[i >> 3] >> (4 * (i & 7))) & 15u;
+    }
+    __syncthreads();
+    const int j = lane < 15 ? lane : 14;
+    const float c_lo = s_cb[j], c_hi = s_cb[j + 1];
+    const double hk = s_half[j];
+    const uint32_t lut = s_lut[lane];
+    uint32_t bad_any = 0;
+    for (int c = 0; 8 * kQbUnroll * c < nblk; ++c) {
+        float w[kQbUnroll][V];
+#pragma unroll
+        for (int i = 0; i < kQbUnroll; ++i) {
+            const int bl = 8 * (kQbUnroll * c + i) + warp;
+            const float *src = W + (b0 + bl) * B;
+            if (bl < nblk) {
+                if (V == 1) {
+                    w[i][0] = __ldcs(src + lane);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < V / 4; ++h) {
+                        const float4 v = __ldcs(reinterpret_cast<const float4 *>(src + 128 * h) + lane);
+                        w[i][4 * h] = v.x, w[i][4 * h + 1] = v.y, w[i][4 * h + 2] = v.z, w[i][4 * h + 3] = v.w;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < V; ++k) w[i][k] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kQbUnroll; ++i) {
+            const int bl = 8 * (kQbUnroll * c + i) + warp;
+            if (bl >= nblk) break;                           // warp-uniform
+            // max |w| on the bit patterns: NaN and Inf sort above every finite value
+            uint32_t m = 0;
+#pragma unroll
+            for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[i][k]) & 0x7fffffffu);
+            const uint32_t ab = __reduce_max_sync(0xffffffffu, m);
+            const float a = __uint_as_float(ab);
+            float tau = kExactHalf ? next_up(__double2float_rd(__dmul_rn(hk, (double)a)))
+                                   : exact_threshold(c_lo, c_hi, a);
+            if (lane >= 15) tau = __uint_as_float(0x7f800000u);
+            const bool fast = use_bins && ab >= 0x0d800000u && ab <= 0x71800000u;   // warp-uniform
+            uint32_t qv[V];
+            if (fast) {
+                const float kr = __fmul_rn(kBinK, rcp_approx(a));
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    const float y = fmaf(w[i][k], kr, kBinC);
+                    const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
+                    const float t = __shfl_sync(0xffffffffu, tau, (int)jt);
+                    qv[k] = jt + (w[i][k] >= t ? 1u : 0u);
+                }
+            } else {
+                float t[15];
+#pragma unroll
+                for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k);
+#pragma unroll
+                for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[i][k], t);
+            }
+            uint8_t *dst = packed + (b0 + bl) * (B / 2);
+            if (V == 1) {
+                // even lane 2i: byte i = (q_2i << 4) | q_2i+1; lane 8k gathers bytes 4k .. 4k+3
+                const uint32_t nx = __shfl_down_sync(0xffffffffu, qv[0], 1);
+                const uint32_t byte = ((qv[0] << 4) | nx) & 0xffu;
+                const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 2);
+                const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 4);
+                const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 6);
+                if ((lane & 7) == 0)
+                    *reinterpret_cast<uint32_t *>(dst + lane / 2) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            } else {
+#pragma unroll
+                for (int h = 0; h < V / 4; ++h) {
+                    const uint32_t v = qv[4 * h + 1] | (qv[4 * h] << 4) | (qv[4 * h + 3] << 8) | (qv[4 * h + 2] << 12);
+                    *reinterpret_cast<uint16_t *>(dst + 64 * h + 2 * lane) = (uint16_t)v;
+                }
+            }
+            if (lane == 0) {
+                s_a[bl] = a;
+                if (!dq) absmax[b0 + bl] = a;
+                bad_any |= ab >= 0x7f800000u;
+            }
+        }
+    }
+    if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
+    if (dq) {
+        __syncthreads();
+        const float a = s_a[threadIdx.x];
+        float mx = a;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) warp_max[warp] = mx;
+        __syncthreads();
+        float gm = warp_max[0];
+#pragma unroll
+        for (int i = 1; i < kQbThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
+        const float f = __fdiv_rn(gm, 255.f);
+        if (threadIdx.x == 0) steps[blockIdx.x] = f;
+        if (threadIdx.x < nblk) codes[b0 + threadIdx.x] = (uint8_t)dq_code(a, f);
+    }
+}
+
+// Dequantize blocks of any supported size: a thread decodes 16 consecutive
+// elements (two packed words, always inside one block) through the per-block
+// product table; grid-stride over the weight.
+__global__ void __launch_bounds__(256)
+k_nf4_dequantize_blk(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t n16, int log2_b16,
+                     Codebook cb, uint16_t *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float ah = load_scale(sc, i >> log2_b16);
+        ProdTable tab;
+        build_table(ah, cb, tab);
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(packed) + i);
+        uint32_t o0[4], o1[4];
+        decode8(w.x, tab, o0);
+        decode8(w.y, tab, o1);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * i);
+        dst[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+        dst[1] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    }
+}
+
 // Dequantize: 4 threads per block; thread i of the 4 owns packed bytes
 // [4i, 4i+4) and [16+4i, 16+4i+4) of its block, i.e. output elements
 // [8i, 8i+8) and [32+8i, 32+8i+8), so each group of 4 threads reads 16
@@ -414,8 +573,36 @@ bool make_exact_halves(const Codebook &cb, QuantBins *bins) {
     return ok;
 }
 
+namespace {
+
+template <int V>
+void launch_quantize_blk(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
+                         uint32_t *d_status, cudaStream_t st) {
+    const int64_t nb = q.rows * q.cols / (32 * V);
+    QuantBins bins{};
+    const bool use_bins = make_quant_bins(cb, &bins);
+    const bool exact_half = make_exact_halves(cb, &bins);
+    auto kern = exact_half ? k_nf4_quantize_blk<V, true> : k_nf4_quantize_blk<V, false>;
+    prof_begin(kProfQuant, st);
+    kern<<<(unsigned)((nb + 255) / 256), kQbThreads, 0, st>>>(W, nb, cb, bins, use_bins, zero_idx,
+                                                              q.double_quant, q.packed, q.absmax,
+                                                              q.absmax_code, q.dq_step, d_status);
+    prof_end(kProfQuant, st);
+}
+
+}  // namespace
+
 int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
                         uint32_t *d_status, cudaStream_t st) {
+    if (q.block != 64) {
+        if (q.rows * q.cols == 0) return QLORA_OK;
+        if (q.block == 32) launch_quantize_blk<1>(W, q, cb, zero_idx, d_status, st);
+        else if (q.block == 128) launch_quantize_blk<4>(W, q, cb, zero_idx, d_status, st);
+        else if (q.block == 256) launch_quantize_blk<8>(W, q, cb, zero_idx, d_status, st);
+        else return QLORA_EUNSUPPORTED;
+        QLORA_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
     QuantBins bins;
@@ -449,6 +636,22 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
 
 int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *out,
                           cudaStream_t st) {
+    if (q.block != 64) {
+        const int64_t n16 = q.rows * q.cols / 16;
+        if (n16 == 0) return QLORA_OK;
+        int lg = 0;
+        while ((16 << lg) < q.block) ++lg;
+        if ((16 << lg) != q.block) return QLORA_EUNSUPPORTED;
+        ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t need = (n16 + 255) / 256, cap = (int64_t)sms * 8;
+        k_nf4_dequantize_blk<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(q.packed, sc, n16, lg,
+                                                                               cb, out);
+        QLORA_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};

@@ -26,6 +26,11 @@
  *   - The frozen weight is stored transposed, Wt:[Dout, Din] (the
  *     nn.Linear layout).  Flattened row-major it is cut into blocks of 64
  *     consecutive weights, each inside one row; Din must be a multiple of 64.
+ *     nf4_quantize and nf4_dequantize also take blocks of 32, 128 or 256
+ *     (q->block; Din a multiple of it; the article's section 5.1 weighs
+ *     smaller blocks' finer scales against their metadata); the layer calls
+ *     and qlora_merge read one scale per 64 inputs and return
+ *     QLORA_EUNSUPPORTED for any other block.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; no call synchronizes the host.
  *   - Return value: QLORA_OK, or an error code.  Arguments are validated on
@@ -59,7 +64,7 @@ extern "C" {
 #define QLORA_DQ_GROUP 256
 #define QLORA_MAX_RANK 256
 
-/* One quantized weight Wt:[rows = Dout, cols = Din]; nb = rows*cols/64.
+/* One quantized weight Wt:[rows = Dout, cols = Din]; nb = rows*cols/block.
  *   packed      [rows*cols/2] uint8   two 4-bit codebook indices per byte;
  *                                     element 2i in the HIGH nibble of byte i
  *   absmax      [nb] fp32             block absmax (double_quant == 0)
@@ -71,7 +76,7 @@ extern "C" {
 typedef struct {
     int64_t rows;
     int64_t cols;
-    int32_t block;          /* must be 64 */
+    int32_t block;          /* 64; the codec calls also take 32, 128, 256 */
     int32_t double_quant;   /* 0 or 1 */
     int32_t dq_group;       /* must be 256 when double_quant == 1 */
     int32_t reserved;
@@ -101,12 +106,18 @@ int qlora_check_codebook(const float codebook[16]);
  * Per block: a = max|w|; index = argmin_j |w - c_j a| in exact arithmetic,
  * ties to the lower index; an all-zero block maps to the exact-zero level.
  * A NaN/Inf weight sets QLORA_STATUS_NONFINITE; that block's outputs are
- * unspecified.  Reads 4 bytes and writes ~0.52 bytes per weight. */
+ * unspecified.  Reads 4 bytes and writes 0.5 + 1/block (+ 4/(256 block)
+ * with double quantization) bytes per weight: ~0.52 at block 64.
+ * Errors: EINVAL for a NULL or unaligned W or buffer, cols not a multiple of
+ * the block, a bad codebook; EUNSUPPORTED for a block outside {32, 64, 128,
+ * 256} or dq_group != 256. */
 int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16],
                  uint32_t *d_status, void *stream);
 
 /* nf4_dequantize -- W_out[rows, cols] (bf16) = RN_bf16(RN32(a_hat * c_q))
- * (section 5.2, w_hat = a c_q, in the bf16 compute dtype of section 8.3). */
+ * (section 5.2, w_hat = a c_q, in the bf16 compute dtype of section 8.3);
+ * element e takes the scale of block e / q->block.  W_out 16-byte aligned.
+ * Errors as nf4_quantize. */
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out,
                    void *stream);
 

@@ -68,7 +68,11 @@ def test_quantize_rejects_bad_arguments(lib):
     W = ctypes.c_void_p(1 << 20)
     E = _lib
     assert lib.nf4_quantize(W, ctypes.byref(_wc(cols=100)), cb, None, None) == E.QLORA_EINVAL
-    assert lib.nf4_quantize(W, ctypes.byref(_wc(block=32)), cb, None, None) == E.QLORA_EUNSUPPORTED
+    for blk in (16, 48, 512):
+        assert lib.nf4_quantize(W, ctypes.byref(_wc(block=blk)), cb, None, None) == E.QLORA_EUNSUPPORTED
+    assert lib.nf4_quantize(W, ctypes.byref(_wc(block=128, cols=192)), cb, None, None) == E.QLORA_EINVAL
+    assert lib.nf4_dequantize(ctypes.byref(_wc(block=256, cols=128)), cb, W, None) == E.QLORA_EINVAL
+    assert lib.nf4_dequantize(ctypes.byref(_wc(block=96)), cb, W, None) == E.QLORA_EUNSUPPORTED
     assert lib.nf4_quantize(W, ctypes.byref(_wc(group=128)), cb, None, None) == E.QLORA_EUNSUPPORTED
     assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=2)), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_quantize(W, ctypes.byref(_wc(ptrs=False)), cb, None, None) == E.QLORA_EINVAL
@@ -100,6 +104,10 @@ def test_layer_rejects_bad_arguments(lib):
     assert fwd(Y=ctypes.c_void_p((1 << 20) + 2)) == E.QLORA_EINVAL
     assert fwd(wc=_wc(rows=60)) == E.QLORA_EUNSUPPORTED          # Dout % 8
     assert fwd(wc=_wc(rows=0)) == E.QLORA_EINVAL
+    for blk in (32, 128, 256):                       # the layer needs blocks of 64
+        assert fwd(wc=_wc(block=blk, cols=256)) == E.QLORA_EUNSUPPORTED
+        assert lib.qlora_merge(ctypes.byref(_wc(block=blk, cols=256)), cb, P, P, 8, 16.0, 1, P,
+                               None) == E.QLORA_EUNSUPPORTED
     assert fwd(nbytes=16) == E.QLORA_EWORKSPACE
     assert fwd(ws=None) == E.QLORA_EWORKSPACE
     assert fwd(M=0) == E.QLORA_OK                                 # empty batch: no-op

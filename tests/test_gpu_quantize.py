@@ -11,18 +11,19 @@ from bit_nf4_quantized_22_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-def _gpu_quant(qlib, W, dq, cb=None):
+def _gpu_quant(qlib, W, dq, cb=None, block=64):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    w = qlib.quantize(torch.from_numpy(W).cuda(), double_quant=dq, codebook=cb, status=status)
+    w = qlib.quantize(torch.from_numpy(W).cuda(), double_quant=dq, codebook=cb, status=status,
+                      block=block)
     torch.cuda.synchronize()
     return w, int(status.item())
 
 
-def _check_same(orc, qlib, W, dq, cb_np=None):
+def _check_same(orc, qlib, W, dq, cb_np=None, block=64):
     cb_np = orc.nf4_codebook() if cb_np is None else cb_np
     cb_t = torch.from_numpy(cb_np.copy())
-    ref = orc.quantize(W, cb_np, dq)
-    w, st = _gpu_quant(qlib, W, dq, cb_t)
+    ref = orc.quantize(W, cb_np, dq, block=block)
+    w, st = _gpu_quant(qlib, W, dq, cb_t, block)
     assert st == ref.status
     gp = w.packed.cpu().numpy()
     if not np.array_equal(gp, ref.packed):
@@ -55,11 +56,10 @@ def test_ragged_shapes(orc, qlib, shape, dq):
     _check_same(orc, qlib, W, dq)
 
 
-def test_adversarial_thresholds(orc, qlib):
-    """Weights at and within a few ulps of every decision threshold, for
-    several absmax magnitudes (incl. subnormal-range scales)."""
+def _adversarial_W(cb, block=64):
+    """Blocks holding +-a and values at and within a few ulps of every decision
+    threshold, for several absmax magnitudes (incl. subnormal-range scales)."""
     from fractions import Fraction as Fr
-    cb = orc.nf4_codebook()
     rows = []
     for a in (1.0, 0.0371, 3.1e-3, 2.0 ** -120, 1.7e30, 6.1e-39):
         a = np.float32(a)
@@ -73,13 +73,17 @@ def test_adversarial_thresholds(orc, qlib):
                     y = np.nextafter(y, np.float32(np.inf if k > 0 else -np.inf))
                 vals.append(y)
         vals = np.array(vals, dtype=np.float32)
-        for s in range(0, vals.size, 62):
-            blk = np.zeros(64, np.float32)
+        for s in range(0, vals.size, block - 2):
+            blk = np.zeros(block, np.float32)
             blk[0], blk[1] = a, -a
-            chunk = vals[s:s + 62]
+            chunk = vals[s:s + block - 2]
             blk[2:2 + chunk.size] = chunk
             rows.append(blk)
-    W = np.stack(rows).reshape(-1, 64)
+    return np.stack(rows).reshape(-1, block)
+
+
+def test_adversarial_thresholds(orc, qlib):
+    W = _adversarial_W(orc.nf4_codebook())
     _check_same(orc, qlib, W, False)
     _check_same(orc, qlib, W, True)
 
@@ -168,3 +172,79 @@ def test_full_size_quantize_70b(orc, qlib):
     spec = synth.CONFIGS[5]["linears"][0]
     W = synth.draw(spec, 1, 5, 0, which=("W",))["W"]
     _check_same(orc, qlib, W, True)
+
+
+# ------------------------------------------------------------ other block sizes
+
+BLOCKS = [32, 128, 256]
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+@pytest.mark.parametrize("shape,dq", [((3, 256), False), ((37, 512), True), ((129, 1280), True),
+                                      ((129, 1280), False)])
+def test_block_sizes_ragged(orc, qlib, block, shape, dq):
+    """Blocks of 32, 128 and 256 weights: partial CTAs and partial double-quant
+    groups, bit-exact indices, scales and dequantized weights."""
+    rng = np.random.default_rng(block * 1000 + shape[0])
+    W = (rng.standard_t(4, size=shape) * 0.02).astype(np.float32)
+    w = _check_same(orc, qlib, W, dq, block=block)
+    nb = W.size // block
+    assert (w.codes if dq else w.absmax).numel() == nb
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+def test_block_sizes_adversarial_and_special(orc, qlib, block):
+    cb = orc.nf4_codebook()
+    W = _adversarial_W(cb, block)
+    _check_same(orc, qlib, W, False, block=block)
+    _check_same(orc, qlib, W, True, block=block)
+    rng = np.random.default_rng(block)
+    S = (rng.standard_normal((6, 2 * 256)) * 0.05).astype(np.float32)
+    S[0, :block] = 0.0                                  # all-zero block
+    S[1, :block] = -0.0
+    S[2, block:2 * block] = 1e-42                       # subnormal block
+    S[3, :block] *= np.float32(2.0 ** 110)              # scales outside [2^-100, 2^100]: the search path
+    S[4, block:2 * block] *= np.float32(2.0 ** -110)
+    S[5, :block] *= np.float32(2.0 ** -96)
+    _check_same(orc, qlib, S, False, block=block)
+    _check_same(orc, qlib, S, True, block=block)
+    S[0, 3] = np.nan
+    assert _gpu_quant(qlib, S, True, block=block)[1] == 1
+
+
+@pytest.mark.parametrize("block", [32, 256])
+def test_block_sizes_custom_codebooks(orc, qlib, block):
+    """A codebook too dense for the bin table (the search path throughout) and
+    one the table serves, with exact ties on their own midpoints."""
+    rng = np.random.default_rng(19 + block)
+    W = (rng.standard_normal((16, 512)) * 0.05).astype(np.float32)
+    tiny = np.array([-1, -.9, -.8, -.7, -.6, -.5, -2.0 ** -60, 0, .5, .6, .7, .75, .8, .85, .9, 1],
+                    dtype=np.float32)
+    wide = np.array([-1, -.85, -.7, -.55, -.4, -.25, -.1, 0, .1, .25, .4, .55, .7, .8, .9, 1],
+                    dtype=np.float32)
+    for cb in (tiny, wide):
+        W2 = W.copy()
+        W2[1, :16] = (np.concatenate([[1.0], (cb[:-1] + cb[1:]) / 2])).astype(np.float32)
+        W2[1, 16:31] = np.nextafter(W2[1, 1:16], np.float32(-np.inf))
+        _check_same(orc, qlib, W2, True, cb, block=block)
+
+
+def test_block_size_full_size_up_proj(orc, qlib):
+    """The 4096 x 11008 weight in blocks of 128 with double quantization."""
+    spec = synth.CONFIGS[3]["linears"][0]
+    W = synth.draw(spec, 1, 3, 0, which=("W",))["W"]
+    _check_same(orc, qlib, W, True, block=128)
+
+
+def test_block_size_layer_calls_refused(qlib):
+    """The layer kernels read one scale per 64 inputs: other sizes are refused
+    loudly rather than misread."""
+    W = torch.zeros(64, 256, device="cuda")
+    w = qlib.quantize(W, block=32)
+    x = torch.zeros(4, 256, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros(256, 8, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError):
+        qlib.forward(x, w, A, B, 16.0)
+    with pytest.raises(RuntimeError):
+        qlib.merge(w, A, B, 16.0)
