@@ -513,7 +513,7 @@ def block_size_lines(q, lib, torch, dev, hbm, flush):
             "quantize_ms": qms, "quantize_frac_hbm": qbytes / (qms / 1e3) / 1e9 / hbm if qms > 0 else None,
             "dequantize_ms": dms, "dequantize_frac_hbm": dbytes / (dms / 1e3) / 1e9 / hbm,
             "metadata_bytes_per_weight": meta / n,
-            "kernel": "k_nf4_quantize_fast" if blk == 64 else "k_nf4_quantize_blk"}
+            "kernel": "k_nf4_quantize_fast" if blk in (32, 64) else "k_nf4_quantize_blk"}
         del w, deq
     return out
 

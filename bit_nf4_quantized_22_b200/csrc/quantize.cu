@@ -211,8 +211,8 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
 // quarter issued together; four CTAs per SM keep enough loads in flight (in
 // measurements this beat staging the group through shared memory with bulk
 // copies).  A warp takes two blocks at a
-// time: lanes 0-15 the first, 16-31 the second, four consecutive weights per
-// lane.  Lane j of a half also holds the exact threshold tau_j of its block
+// time: lanes 0-15 the first, 16-31 the second, V consecutive weights per
+// lane (V = 4 for blocks of 64, 2 for blocks of 32).  Lane j of a half also holds the exact threshold tau_j of its block
 // (lane 15: +inf).  A weight's index then costs one table lookup and one
 // exact compare instead of a four-level search:
 //   bin = RN(K * (w * RN(1/a)) + 16)          (approximate)
@@ -228,7 +228,8 @@ constexpr float kBinC = 12582928.0f;   // 1.5 * 2^23 + 16: the low 5 bits of the
 constexpr int kQfThreads = 256;
 constexpr int kQfSmem = 0;
 
-template <bool kExactHalf>
+// V weights per lane: 4 for blocks of 64, 2 for blocks of 32 (16 lanes per block either way).
+template <bool kExactHalf, int V>
 __global__ void __launch_bounds__(kQfThreads, 4)
 k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins,
                     int zero_idx, int dq, uint8_t *__restrict__ packed,
@@ -258,22 +259,32 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
     for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
-        float4 pre[4];
+        float pre[4][V];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int bl = 64 * c + 2 * (warp + 8 * i) + half;
-            pre[i] = bl < nblk ? __ldcs(reinterpret_cast<const float4 *>(W + (b0 + bl) * 64 + 4 * j))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float *src = W + (b0 + bl) * (16 * V) + V * j;
+            if (V == 4) {
+                const float4 v = bl < nblk ? __ldcs(reinterpret_cast<const float4 *>(src))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                pre[i][0] = v.x, pre[i][1] = v.y, pre[i][2] = v.z, pre[i][3] = v.w;
+            } else {
+                const float2 v = bl < nblk ? __ldcs(reinterpret_cast<const float2 *>(src))
+                                           : make_float2(0.f, 0.f);
+                pre[i][0] = v.x, pre[i][1] = v.y;
+            }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int bl = 64 * c + 2 * (warp + 8 * i) + half;   // block within the group
             const bool valid = bl < nblk;
-            float w[4] = {pre[i].x, pre[i].y, pre[i].z, pre[i].w};
+            float w[V];
+#pragma unroll
+            for (int k = 0; k < V; ++k) w[k] = pre[i][k];
             // max |w| on the bit patterns: NaN and Inf sort above every finite value
             uint32_t m = 0;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) m = max(m, __float_as_uint(w[k]) & 0x7fffffffu);
+            for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[k]) & 0x7fffffffu);
             const uint32_t m0 = __reduce_max_sync(0xffffffffu, half ? 0u : m);
             const uint32_t m1 = __reduce_max_sync(0xffffffffu, half ? m : 0u);
             const uint32_t ab = half ? m1 : m0;
@@ -287,11 +298,11 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
                 tau = exact_threshold(c_lo, c_hi, a);
             if (j == 15) tau = __uint_as_float(0x7f800000u);
             const bool fast = ab >= 0x0d800000u && ab <= 0x71800000u;   // 2^-100 <= a <= 2^100
-            uint32_t qv[4];
+            uint32_t qv[V];
             if (__all_sync(0xffffffffu, fast || !valid)) {
                 const float kr = __fmul_rn(kBinK, rcp_approx(a));   // K / a, relative error < 2^-22
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < V; ++k) {
                     const float y = fmaf(w[k], kr, kBinC);
                     const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
                     const float t = __shfl_sync(0xffffffffu, tau, (int)jt, 16);
@@ -302,12 +313,16 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
 #pragma unroll
                 for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k, 16);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[k], t);
+                for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[k], t);
             }
             if (valid) {
-                // weights 4j..4j+3 -> bytes 2j, 2j+1; element 2i in the high nibble
-                const uint32_t v = qv[1] | (qv[0] << 4) | (qv[3] << 8) | (qv[2] << 12);
-                *reinterpret_cast<uint16_t *>(packed + (b0 + bl) * 32 + 2 * j) = (uint16_t)v;
+                // weights V j .. V j + V-1 -> bytes (V/2) j ..; element 2i in the high nibble
+                if (V == 4) {
+                    const uint32_t v = qv[1] | (qv[0] << 4) | (qv[3 % V] << 8) | (qv[2 % V] << 12);
+                    *reinterpret_cast<uint16_t *>(packed + (b0 + bl) * 32 + 2 * j) = (uint16_t)v;
+                } else {
+                    packed[(b0 + bl) * 16 + j] = (uint8_t)(qv[1] | (qv[0] << 4));
+                }
                 if (j == 0) {
                     s_a[bl] = a;
                     if (!dq) absmax[b0 + bl] = a;
@@ -596,7 +611,17 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
                         uint32_t *d_status, cudaStream_t st) {
     if (q.block != 64) {
         if (q.rows * q.cols == 0) return QLORA_OK;
-        if (q.block == 32) launch_quantize_blk<1>(W, q, cb, zero_idx, d_status, st);
+        QuantBins bins32;
+        if (q.block == 32 && make_quant_bins(cb, &bins32)) {   // two blocks per warp, as at 64
+            const int64_t nb = q.rows * q.cols / 32;
+            auto kern = make_exact_halves(cb, &bins32) ? k_nf4_quantize_fast<true, 2>
+                                                       : k_nf4_quantize_fast<false, 2>;
+            prof_begin(kProfQuant, st);
+            kern<<<(unsigned)((nb + 255) / 256), kQfThreads, kQfSmem, st>>>(
+                W, nb, cb, bins32, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code,
+                q.dq_step, d_status);
+            prof_end(kProfQuant, st);
+        } else if (q.block == 32) launch_quantize_blk<1>(W, q, cb, zero_idx, d_status, st);
         else if (q.block == 128) launch_quantize_blk<4>(W, q, cb, zero_idx, d_status, st);
         else if (q.block == 256) launch_quantize_blk<8>(W, q, cb, zero_idx, d_status, st);
         else return QLORA_EUNSUPPORTED;
@@ -608,7 +633,7 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
     QuantBins bins;
     if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && make_quant_bins(cb, &bins)) {
         const bool exact_half = make_exact_halves(cb, &bins);
-        auto kern = exact_half ? k_nf4_quantize_fast<true> : k_nf4_quantize_fast<false>;
+        auto kern = exact_half ? k_nf4_quantize_fast<true, 4> : k_nf4_quantize_fast<false, 4>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQfSmem);
         prof_begin(kProfQuant, st);
         kern<<<(unsigned)((nb + 255) / 256), kQfThreads, kQfSmem, st>>>(
