@@ -63,6 +63,11 @@ def _L():
         lib.orc_dequantize.restype = None
         lib.orc_dequantize.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
                                        P, P]
+        lib.orc_dequantize_dt.restype = None
+        lib.orc_dequantize_dt.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P,
+                                          P, P, ctypes.c_int, P]
+        lib.orc_fp16_bits.restype = None
+        lib.orc_fp16_bits.argtypes = [P, i64, P]
         lib.orc_adapter_down.restype = None
         lib.orc_adapter_down.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, P]
         lib.orc_forward.restype = None
@@ -154,6 +159,28 @@ def dequantize(q: QuantizedWeight, codebook: np.ndarray, dq_group: int = DQ_GROU
     out = np.zeros((q.rows, q.cols), dtype=np.uint16)
     _L().orc_dequantize(q.rows, q.cols, q.block, _p(cb), int(q.double_quant), dq_group, _p(q.packed),
                         _p(q.absmax), _p(q.codes), _p(q.steps), _p(out))
+    return out
+
+
+DTYPES = {"bf16": 0, "fp16": 1, "fp32": 2}
+
+
+def dequantize_dt(q: QuantizedWeight, codebook: np.ndarray, dtype: str,
+                  dq_group: int = DQ_GROUP) -> np.ndarray:
+    """[rows, cols] in the compute dtype: uint16 bit patterns for bf16 and
+    fp16, float32 values for fp32."""
+    cb = _c(codebook, np.float32)
+    out = np.zeros((q.rows, q.cols), dtype=np.float32 if dtype == "fp32" else np.uint16)
+    _L().orc_dequantize_dt(q.rows, q.cols, q.block, _p(cb), int(q.double_quant), dq_group,
+                           _p(q.packed), _p(q.absmax), _p(q.codes), _p(q.steps), DTYPES[dtype],
+                           _p(out))
+    return out
+
+
+def fp16_bits(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32).reshape(-1)
+    out = np.zeros(x.size, dtype=np.uint16)
+    _L().orc_fp16_bits(_p(x), x.size, _p(out))
     return out
 
 

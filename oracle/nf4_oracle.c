@@ -284,6 +284,61 @@ void orc_dequantize(int64_t rows, int64_t cols, int block, const float cb[16], i
     }
 }
 
+/* Round a finite or infinite fp32 value to IEEE binary16, round to nearest
+ * even, as bits.  binary16 keeps 11 significant bits; below 2^-14 its
+ * spacing is fixed at 2^-24 (subnormals).  x is scaled so that the kept bits
+ * are the integer part, rounded by rint (the default mode is to nearest
+ * even) and scaled back, all exact in fp64; magnitudes past 65504 after
+ * rounding are infinite. */
+static uint16_t float_to_fp16_rne(float f) {
+    double x = (double)f;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    if (isnan(x)) return (uint16_t)(sign | 0x7e00u);
+    x = fabs(x);
+    if (isinf(x)) return (uint16_t)(sign | 0x7c00u);
+    if (x == 0.0) return sign;
+    int e;
+    frexp(x, &e);                        /* x = m 2^e, m in [0.5, 1): leading bit 2^(e-1) */
+    int q = e - 11;                      /* exponent of the last kept bit */
+    if (q < -24) q = -24;                /* the subnormal spacing */
+    double r = ldexp(rint(ldexp(x, -q)), q);
+    if (r > 65504.0) return (uint16_t)(sign | 0x7c00u);
+    if (r < ldexp(1.0, -14))             /* subnormal (or zero): mantissa in units of 2^-24 */
+        return (uint16_t)(sign | (uint16_t)ldexp(r, 24));
+    int er;
+    double mr = frexp(r, &er);           /* r = mr 2^er; biased exponent er - 1 + 15 */
+    uint16_t mant = (uint16_t)(ldexp(mr, 11) - 1024.0);
+    return (uint16_t)(sign | (uint16_t)((er - 1 + 15) << 10) | mant);
+}
+
+/* Dequantize into a chosen compute dtype ([CSDN] 8.3: the dequantized
+ * weights and the arithmetic are FP32, BF16 or FP16): w_hat =
+ * RN_dtype(RN_fp32(a_hat * c_q)).  dtype 0 = bf16, 1 = fp16 (16-bit patterns
+ * in out), 2 = fp32 (out holds fp32 values). */
+void orc_dequantize_dt(int64_t rows, int64_t cols, int block, const float cb[16], int dq,
+                       int dq_group, const uint8_t *packed, const float *absmax,
+                       const uint8_t *codes, const float *steps, int dtype, void *out) {
+    const int64_t n = rows * cols;
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n; ++e) {
+        uint8_t byte = packed[e / 2];
+        int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
+        float ah = block_scale(e / block, dq, dq_group, absmax, codes, steps);
+        float w = (float)((double)ah * (double)cb[q]);
+        if (dtype == 2)
+            ((float *)out)[e] = w;
+        else if (dtype == 1)
+            ((uint16_t *)out)[e] = float_to_fp16_rne(w);
+        else
+            ((uint16_t *)out)[e] = float_to_bf16_rne(w);
+    }
+}
+
+/* fp32 -> binary16 bits, exported so tests can pin the conversion alone. */
+void orc_fp16_bits(const float *x, int64_t n, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = float_to_fp16_rne(x[i]);
+}
+
 /* ------------------------------------------------------------------------ */
 /* The layer: forward and backward in fp64                                   */
 /* ------------------------------------------------------------------------ */

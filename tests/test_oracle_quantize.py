@@ -399,3 +399,55 @@ def test_block_sizes_dequant_roundtrip_and_dq(orc, block):
     expect = np.array([scaled(e) for e in range(0, jf.size, 97)], dtype=np.float32)
     got = orc.dequantize(qd, cb).reshape(-1)[::97]
     assert np.array_equal(got, bf16_of_f32(expect))
+
+
+# ---------------------------------------------------------------- compute dtypes
+# The article's section 8.3: the dequantized weights and the arithmetic are in
+# the compute dtype, FP32, BF16 or FP16.
+
+def test_fp16_rounding_matches_ieee(orc):
+    """The oracle's binary16 rounding against numpy's IEEE conversion on
+    normal, subnormal, tie, overflow and special values."""
+    rng = np.random.default_rng(23)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(5000) * 1e-5).astype(np.float32),          # fp16 subnormals
+        (rng.standard_normal(2000) * 1e-8).astype(np.float32),          # below half the least subnormal
+        np.array([65504, 65519.99, 65520, 70000, -65520, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                  2.0 ** -14, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 0.0, -0.0, np.inf, -np.inf],
+                 dtype=np.float32)])
+    got = orc.fp16_bits(x)
+    with np.errstate(over="ignore"):                    # the overflow to infinity is intended
+        want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:5]
+    assert orc.fp16_bits(np.array([np.nan], np.float32))[0] & 0x7c00 == 0x7c00
+
+
+@pytest.mark.parametrize("block", [32, 64, 256])
+def test_dequantize_compute_dtypes(orc, block):
+    """fp32 output is RN32(a_hat c_q) itself; bf16 and fp16 are that value
+    rounded once, so they equal numpy's rounding of the fp32 output, and the
+    bf16 case equals the bf16 dequantize."""
+    rng = np.random.default_rng(31 + block)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_t(4, (16, 512)) * 0.5).astype(np.float32)
+    W[3] *= np.float32(1e5)                             # scales that overflow fp16
+    W[5] *= np.float32(1e-6)                            # and ones in its subnormal range
+    for dq in (False, True):
+        q = orc.quantize(W, cb, dq, block=block)
+        f32 = orc.dequantize_dt(q, cb, "fp32")
+        idx = unpack(q.packed, W.size)
+        if not dq:
+            ahat = np.repeat(q.absmax, block)
+        else:
+            ahat = (q.codes.astype(np.float64) * np.repeat(q.steps.astype(np.float64), 256)[:q.codes.size]
+                    ).astype(np.float32)
+            ahat = np.repeat(ahat, block)
+        # a product of two fp32 values is exact in fp64: one rounding to fp32
+        expect = (ahat.astype(np.float64) * cb.astype(np.float64)[idx]).astype(np.float32)
+        assert np.array_equal(f32.reshape(-1).view(np.uint32), expect.view(np.uint32))
+        with np.errstate(over="ignore"):
+            f16 = f32.reshape(-1).astype(np.float16).view(np.uint16)
+        assert np.array_equal(orc.dequantize_dt(q, cb, "fp16").reshape(-1), f16)
+        assert np.array_equal(orc.dequantize_dt(q, cb, "bf16"), orc.dequantize(q, cb))
+        assert np.array_equal(orc.dequantize(q, cb).reshape(-1), bf16_of_f32(f32.reshape(-1)))
