@@ -514,6 +514,23 @@ def block_size_lines(q, lib, torch, dev, hbm, flush):
             "dequantize_ms": dms, "dequantize_frac_hbm": dbytes / (dms / 1e3) / 1e9 / hbm,
             "metadata_bytes_per_weight": meta / n,
             "kernel": "k_nf4_quantize_fast" if blk in (32, 64) else "k_nf4_quantize_blk"}
+        if blk == 64:   # the other compute dtypes (fp16: 2 B out per weight, fp32: 4 B)
+            for name, dt, ob in (("fp16", torch.float16, 2), ("fp32", torch.float32, 4)):
+                o = torch.empty(W.shape, dtype=dt, device=dev)
+                for _ in range(3):
+                    q.dequantize(w, out=o, dtype=dt)
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(reps)]
+                for e0, e1 in ev:
+                    flush.zero_()
+                    e0.record()
+                    q.dequantize(w, out=o, dtype=dt)
+                    e1.record()
+                torch.cuda.synchronize()
+                t = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[reps // 2]
+                out[str(blk)][f"dequantize_{name}_ms"] = t
+                out[str(blk)][f"dequantize_{name}_frac_hbm"] = (n // 2 + meta + ob * n) / (t / 1e3) / 1e9 / hbm
+                del o
         del w, deq
     return out
 

@@ -20,7 +20,7 @@ EXPORTS = (
     "qlora_strerror", "qlora_version", "qlora_check_codebook", "nf4_quantize",
     "nf4_dequantize", "qlora_workspace_size", "qlora_forward", "qlora_backward",
     "qlora_launch_count", "qlora_profile_enable", "qlora_profile_reset", "qlora_profile_read",
-    "qlora_forward_noalloc", "qlora_merge", "qlora_selftest_wait_timeout",
+    "qlora_forward_noalloc", "qlora_merge", "qlora_selftest_wait_timeout", "nf4_dequantize_dtype",
 )
 
 
@@ -72,6 +72,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.nf4_quantize.argtypes = [P, W, P, P, P]
     lib.nf4_dequantize.restype = ctypes.c_int
     lib.nf4_dequantize.argtypes = [W, P, P, P]
+    lib.nf4_dequantize_dtype.restype = ctypes.c_int
+    lib.nf4_dequantize_dtype.argtypes = [W, P, i32, P, P]
     lib.qlora_workspace_size.restype = sz
     lib.qlora_workspace_size.argtypes = [i64, W, i32, i32, i32]
     lib.qlora_forward.restype = ctypes.c_int

@@ -106,12 +106,24 @@ def quantize(W: torch.Tensor, double_quant: bool = True, codebook: torch.Tensor 
     return q
 
 
+_DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+
+
 def dequantize(q: NF4Weight, codebook: torch.Tensor | None = None,
-               out: torch.Tensor | None = None) -> torch.Tensor:
-    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=torch.bfloat16,
+               out: torch.Tensor | None = None, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """The dequantized weight [rows, cols] in the compute dtype (bf16, fp16 or fp32)."""
+    if dtype not in _DTYPE_CODES:
+        raise TypeError(f"dtype: one of {list(_DTYPE_CODES)}")
+    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=dtype,
                                                   device=q.packed.device)
+    if out.dtype != dtype:
+        raise TypeError("out: dtype does not match")
     qc = q.c_struct()
-    rc = load().nf4_dequantize(ctypes.byref(qc), _cb_host(codebook), _ptr(out), _stream())
+    if dtype == torch.bfloat16:
+        rc = load().nf4_dequantize(ctypes.byref(qc), _cb_host(codebook), _ptr(out), _stream())
+    else:
+        rc = load().nf4_dequantize_dtype(ctypes.byref(qc), _cb_host(codebook), _DTYPE_CODES[dtype],
+                                         _ptr(out), _stream())
     _lib.check(rc, "nf4_dequantize")
     return out
 

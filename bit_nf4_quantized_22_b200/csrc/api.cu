@@ -13,6 +13,8 @@ namespace qlora {
 int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
                         uint32_t *d_status, cudaStream_t st);
 int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *out, cudaStream_t st);
+int launch_nf4_dequantize_dtype(const nf4_weight_t &q, const Codebook &cb, int dtype, void *out,
+                                cudaStream_t st);
 // merge.cu
 int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, const uint16_t *B,
                  int r, int gp, float s, uint16_t *W_out, cudaStream_t st);
@@ -396,6 +398,20 @@ int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16]
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!W || !aligned16(W)) return QLORA_EINVAL;
     return launch_nf4_quantize(W, *q, to_cb(codebook), zi, d_status, (cudaStream_t)stream);
+}
+
+int nf4_dequantize_dtype(const nf4_weight_t *q, const float codebook[16], int32_t dtype,
+                         void *W_out, void *stream) {
+    if (dtype != QLORA_DTYPE_BF16 && dtype != QLORA_DTYPE_FP16 && dtype != QLORA_DTYPE_FP32)
+        return QLORA_EINVAL;
+    RC(check_weight(q, false, true));
+    RC(check_codebook(codebook, nullptr));
+    if (q->rows * q->cols == 0) return QLORA_OK;
+    if (!W_out || !aligned16(W_out)) return QLORA_EINVAL;
+    if (dtype == QLORA_DTYPE_BF16)
+        return launch_nf4_dequantize(*q, to_cb(codebook), static_cast<uint16_t *>(W_out),
+                                     (cudaStream_t)stream);
+    return launch_nf4_dequantize_dtype(*q, to_cb(codebook), dtype, W_out, (cudaStream_t)stream);
 }
 
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out, void *stream) {

@@ -511,6 +511,65 @@ k_nf4_dequantize_blk(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t n1
     }
 }
 
+// Dequantize into fp16: the per-block product table of binary16 patterns
+// RN_fp16(RN32(a_hat * c_j)) (IEEE rounding of each half, subnormals kept),
+// decoded by the same byte permutes as the bf16 table; 16 elements a thread.
+__global__ void __launch_bounds__(256)
+k_nf4_dequantize_f16(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t n16, int log2_b16,
+                     Codebook cb, uint16_t *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float ah = load_scale(sc, i >> log2_b16);
+        uint32_t p[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const __half2 h = __floats2half2_rn(__fmul_rn(ah, cb.c[2 * k]), __fmul_rn(ah, cb.c[2 * k + 1]));
+            p[k] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        ProdTable tab;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            tab.lo[k] = __byte_perm(p[2 * k], p[2 * k + 1], 0x6420);
+            tab.hi[k] = __byte_perm(p[2 * k], p[2 * k + 1], 0x7531);
+        }
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(packed) + i);
+        uint32_t o0[4], o1[4];
+        decode8(w.x, tab, o0);
+        decode8(w.y, tab, o1);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * i);
+        dst[0] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+        dst[1] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    }
+}
+
+// Dequantize into fp32: RN32(a_hat * c_q) itself; 8 elements (one packed
+// word) a thread, the codebook in shared memory.
+__global__ void __launch_bounds__(256)
+k_nf4_dequantize_f32(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t n8, int log2_b8,
+                     Codebook cb, float *__restrict__ out) {
+    __shared__ float cbs[16];
+    if (threadIdx.x == 0) {   // constant indices keep the parameter out of local memory
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
+    }
+    __syncthreads();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float ah = load_scale(sc, i >> log2_b8);
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(packed) + i);
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // byte k: element 2k in the high nibble
+            const uint32_t byte = (w >> (8 * k)) & 0xffu;
+            v[2 * k] = __fmul_rn(ah, cbs[byte >> 4]);
+            v[2 * k + 1] = __fmul_rn(ah, cbs[byte & 15]);
+        }
+        float4 *dst = reinterpret_cast<float4 *>(out + 8 * i);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
 // Dequantize: 4 threads per block; thread i of the 4 owns packed bytes
 // [4i, 4i+4) and [16+4i, 16+4i+4) of its block, i.e. output elements
 // [8i, 8i+8) and [32+8i, 32+8i+8), so each group of 4 threads reads 16
@@ -683,6 +742,33 @@ int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *o
     const int64_t threads = nb * 4;
     const int64_t grid = (threads + 255) / 256;
     k_nf4_dequantize<<<(unsigned)grid, 256, 0, st>>>(q.packed, sc, nb, cb, out);
+    QLORA_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+int launch_nf4_dequantize_dtype(const nf4_weight_t &q, const Codebook &cb, int dtype, void *out,
+                                cudaStream_t st) {
+    const int64_t n = q.rows * q.cols;
+    if (n == 0) return QLORA_OK;
+    int lg = 0;                                   // block = 8 << lg
+    while ((8 << lg) < q.block) ++lg;
+    if ((8 << lg) != q.block) return QLORA_EUNSUPPORTED;
+    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * 8;
+    if (dtype == QLORA_DTYPE_FP16) {
+        const int64_t n16 = n / 16, need = (n16 + 255) / 256;
+        k_nf4_dequantize_f16<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(
+            q.packed, sc, n16, lg - 1, cb, static_cast<uint16_t *>(out));
+    } else if (dtype == QLORA_DTYPE_FP32) {
+        const int64_t n8 = n / 8, need = (n8 + 255) / 256;
+        k_nf4_dequantize_f32<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(
+            q.packed, sc, n8, lg, cb, static_cast<float *>(out));
+    } else {
+        return QLORA_EINVAL;
+    }
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }

@@ -121,6 +121,23 @@ int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16]
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out,
                    void *stream);
 
+/* Compute dtypes of nf4_dequantize_dtype (section 8.3: FP32, BF16 or FP16). */
+#define QLORA_DTYPE_BF16 0
+#define QLORA_DTYPE_FP16 1
+#define QLORA_DTYPE_FP32 2
+
+/* nf4_dequantize_dtype -- as nf4_dequantize, into the compute dtype `dtype`
+ * (bitsandbytes article (CSDN) section 8.3: the dequantized weights and the
+ * arithmetic are FP32, BF16 or FP16; 8.5 on FP16's narrower range):
+ *   W_out[e] = RN_dtype(RN32(a_hat * c_q)), one rounding of the fp32
+ *   product; fp16 follows IEEE binary16 (subnormals kept, magnitudes past
+ *   65504 after rounding become infinite); fp32 is the product itself.
+ *   W_out   device [rows, cols] of 16-bit patterns (bf16, fp16) or fp32,
+ *           16-byte aligned.
+ * Errors as nf4_dequantize, plus EINVAL for an unknown dtype. */
+int nf4_dequantize_dtype(const nf4_weight_t *q, const float codebook[16], int32_t dtype,
+                         void *W_out, void *stream);
+
 /* qlora_merge -- the weight with the adapter folded in, for deployment
  * ("从 LoRA 到 QLoRA、QA-LoRA" section 2, W_eff = dequant(W4) + (alpha/r) A B;
  * bitsandbytes article (CSDN) 12.10, merging before deployment):

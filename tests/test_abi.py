@@ -73,6 +73,11 @@ def test_quantize_rejects_bad_arguments(lib):
     assert lib.nf4_quantize(W, ctypes.byref(_wc(block=128, cols=192)), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_dequantize(ctypes.byref(_wc(block=256, cols=128)), cb, W, None) == E.QLORA_EINVAL
     assert lib.nf4_dequantize(ctypes.byref(_wc(block=96)), cb, W, None) == E.QLORA_EUNSUPPORTED
+    for bad_dtype in (-1, 3):
+        assert lib.nf4_dequantize_dtype(ctypes.byref(_wc()), cb, bad_dtype, W, None) == E.QLORA_EINVAL
+    assert lib.nf4_dequantize_dtype(ctypes.byref(_wc()), cb, 1, ctypes.c_void_p((1 << 20) + 8),
+                                    None) == E.QLORA_EINVAL
+    assert lib.nf4_dequantize_dtype(ctypes.byref(_wc(rows=0)), cb, 2, W, None) == E.QLORA_OK
     assert lib.nf4_quantize(W, ctypes.byref(_wc(group=128)), cb, None, None) == E.QLORA_EUNSUPPORTED
     assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=2)), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_quantize(W, ctypes.byref(_wc(ptrs=False)), cb, None, None) == E.QLORA_EINVAL

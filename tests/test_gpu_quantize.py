@@ -248,3 +248,26 @@ def test_block_size_layer_calls_refused(qlib):
         qlib.forward(x, w, A, B, 16.0)
     with pytest.raises(RuntimeError):
         qlib.merge(w, A, B, 16.0)
+
+
+# ------------------------------------------------------------ compute dtypes
+
+@pytest.mark.parametrize("block", [32, 64, 256])
+@pytest.mark.parametrize("dq", [False, True])
+def test_dequantize_compute_dtypes(orc, qlib, block, dq):
+    """fp16 and fp32 outputs bit-exact against the oracle, including scales
+    whose products overflow fp16 and ones in its subnormal range."""
+    rng = np.random.default_rng(41 + block)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_t(4, (37, 1024)) * 0.5).astype(np.float32)
+    W[3] *= np.float32(1e5)
+    W[5] *= np.float32(1e-6)
+    W[7, :block] = 0.0
+    ref = orc.quantize(W, cb, dq, block=block)
+    w, _ = _gpu_quant(qlib, W, dq, block=block)
+    for name, dt in (("fp16", torch.float16), ("fp32", torch.float32), ("bf16", torch.bfloat16)):
+        got = qlib.dequantize(w, dtype=dt)
+        torch.cuda.synchronize()
+        want = orc.dequantize_dt(ref, cb, name)
+        g = got.cpu().view(torch.int32 if dt == torch.float32 else torch.int16).numpy()
+        assert np.array_equal(g.view(want.dtype), want), name
