@@ -191,17 +191,6 @@ int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H
 
 // ---------------------------------------------------------------- GEMM launcher
 
-static int num_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    return sms;
-}
-
 template <int BM, int BN>
 static int run_mma_gemm(MmaGemmArgs a, cudaStream_t st) {
     using S = MmaSmem<BM, BN>;
@@ -219,7 +208,7 @@ static int run_mma_gemm(MmaGemmArgs a, cudaStream_t st) {
 int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN) {
     const int64_t tiles = ((P + 127) / 128) * ((Q + BN - 1) / BN);
     const int64_t nkt = (Rtot + kMmaBK - 1) / kMmaBK;
-    int64_t s = 2 * (int64_t)num_sms() / tiles;   // one wave of two CTAs per SM
+    int64_t s = 2 * (int64_t)device_sms() / tiles;   // one wave of two CTAs per SM
     const int64_t cap = nkt / 8 > 1 ? nkt / 8 : 1;
     if (s > cap) s = cap;
     if (s > 32) s = 32;

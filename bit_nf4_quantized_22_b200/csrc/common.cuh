@@ -132,6 +132,9 @@ enum ProfKind { kProfUmma = 0, kProfGemv = 1, kProfQuant = 2, kProfAdapter = 3, 
 void count_launch();
 void prof_begin(int kind, cudaStream_t st);
 void prof_end(int kind, cudaStream_t st);
+// Streaming multiprocessors of the current device (cached per device; 148
+// if the query fails), for grids sized to whole waves.
+int device_sms();
 }  // namespace qlora
 
 // Host-side launch check used after every kernel launch.

@@ -892,13 +892,11 @@ size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     return (size_t)nsplit * M * Dout * sizeof(float);
 }
 
-static int num_sms_gemv();
-
 // splits of the streamed backward: at most one CTA per SM over the slices
 // (one CTA fits on an SM; a second wave would double the time)
 static int bwd_stream_splits(int64_t Din, int64_t Dout) {
     const int64_t nkz = (Din + kBsCols - 1) / kBsCols, ntn = (Dout + kBsRows - 1) / kBsRows;
-    int64_t ns = num_sms_gemv() / nkz;
+    int64_t ns = device_sms() / nkz;
     if (ns > ntn) ns = ntn;
     return (int)(ns < 1 ? 1 : ns);
 }
@@ -909,17 +907,6 @@ size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     const int64_t ns2 = bwd_stream_splits(Din, Dout);   // the streamed kernel always writes partials
     if (ns2 > nsplit) nsplit = ns2;
     return (size_t)nsplit * M * Din * sizeof(float);
-}
-
-static int num_sms_gemv() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
 }
 
 size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r) {
@@ -958,7 +945,7 @@ int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codeb
     if (stream) {
         const int ntr = (int)((Dout + kStRows - 1) / kStRows);
         const int ntiles = (int)(ntr * nsplit);
-        const int grid = ntiles < num_sms_gemv() ? ntiles : num_sms_gemv();
+        const int grid = ntiles < device_sms() ? ntiles : device_sms();
         if (M <= 8) {
             cudaFuncSetAttribute(k_gemv_fwd_stream<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
             k_gemv_fwd_stream<1><<<grid, kStThreads, kStSmem, st>>>(

@@ -247,17 +247,6 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
     cp_async_wait<0>();                              // no copy outlives the CTA
 }
 
-int mg_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 }  // namespace
 
 size_t merge_smem_bytes(int r) {
@@ -274,7 +263,7 @@ int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, c
     const int nbuf = smem == mg_smem(r, 3) ? 3 : 2;
     cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int64_t units = (Dout + kMgRows - 1) / kMgRows * (Din / 64);
-    const unsigned grid = (unsigned)(units < mg_sms() ? units : mg_sms());
+    const unsigned grid = (unsigned)(units < device_sms() ? units : device_sms());
     prof_begin(kProfMerge, st);
     k_merge<<<grid, kMgThreads, smem, st>>>(q.packed, sc, cb, A, B, r, gp, s / (float)gp, Dout, Din,
                                             nbuf, W_out);

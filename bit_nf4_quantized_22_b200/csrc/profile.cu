@@ -22,6 +22,20 @@ Pairs g_pairs[kProfKinds];
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int device_sms() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+    std::atomic<int> &slot = cache[dev < 64 ? dev : 63];
+    int n = slot.load(std::memory_order_relaxed);
+    if (n <= 0 || dev >= 64) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        if (dev < 64) slot.store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
 void prof_begin(int kind, cudaStream_t st) {
     if (!g_on.load(std::memory_order_relaxed)) return;
     std::lock_guard<std::mutex> lk(g_mu);

@@ -727,10 +727,7 @@ int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *o
         while ((16 << lg) < q.block) ++lg;
         if ((16 << lg) != q.block) return QLORA_EUNSUPPORTED;
         ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t need = (n16 + 255) / 256, cap = (int64_t)sms * 8;
+        const int64_t need = (n16 + 255) / 256, cap = (int64_t)device_sms() * 8;
         k_nf4_dequantize_blk<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(q.packed, sc, n16, lg,
                                                                                cb, out);
         QLORA_LAUNCH_CHECK();
@@ -754,10 +751,7 @@ int launch_nf4_dequantize_dtype(const nf4_weight_t &q, const Codebook &cb, int d
     while ((8 << lg) < q.block) ++lg;
     if ((8 << lg) != q.block) return QLORA_EUNSUPPORTED;
     ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 8;
+    const int64_t cap = (int64_t)device_sms() * 8;
     if (dtype == QLORA_DTYPE_FP16) {
         const int64_t n16 = n / 16, need = (n16 + 255) / 256;
         k_nf4_dequantize_f16<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(

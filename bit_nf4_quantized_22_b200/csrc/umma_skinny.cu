@@ -217,17 +217,6 @@ bool make_operand_map(CUtensorMap *m, const uint16_t *ptr, int64_t ld, int kmajo
                     (uint64_t)ld * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 }  // namespace
 
 int skinny_n(int64_t Q) { return Q <= 64 ? 64 : (Q <= 128 ? 128 : (Q <= 192 ? 192 : 256)); }
@@ -238,7 +227,7 @@ void skinny_splits(int64_t P, int64_t Q, int nk, int *splits, int *per) {
     const int64_t tiles = ((P + kSBM - 1) / kSBM) * ((Q + 255) / 256);
     // two resident CTAs per SM; round down so that the grid is one wave
     // (a few CTAs over the slots would cost a whole second round)
-    int64_t s = 2 * sms() / tiles;
+    int64_t s = 2 * device_sms() / tiles;
     const int64_t cap = nk / 4 > 1 ? nk / 4 : 1;
     if (s > cap) s = cap;
     if (s < 1) s = 1;
