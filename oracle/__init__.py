@@ -69,20 +69,23 @@ def _L():
         lib.orc_fp16_bits.restype = None
         lib.orc_fp16_bits.argtypes = [P, i64, P]
         lib.orc_adapter_down.restype = None
-        lib.orc_adapter_down.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, P]
+        lib.orc_adapter_down.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+        lib.orc_fp16_decode.restype = None
+        lib.orc_fp16_decode.argtypes = [P, i64, P]
         lib.orc_forward.restype = None
         lib.orc_forward.argtypes = [P, i64, i64, i64, P, P, P, ctypes.c_int, ctypes.c_double,
-                                    ctypes.c_int, P, P]
+                                    ctypes.c_int, P, P, ctypes.c_int]
         lib.orc_merge.restype = None
-        lib.orc_merge.argtypes = [i64, i64, P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_int, P]
+        lib.orc_merge.argtypes = [i64, i64, P, P, P, ctypes.c_int, ctypes.c_double, ctypes.c_int, P,
+                                  ctypes.c_int]
         lib.orc_grad_G.restype = None
-        lib.orc_grad_G.argtypes = [P, i64, i64, P, ctypes.c_int, P]
+        lib.orc_grad_G.argtypes = [P, i64, i64, P, ctypes.c_int, P, ctypes.c_int]
         lib.orc_backward_dx.restype = None
         lib.orc_backward_dx.argtypes = [P, i64, i64, i64, P, P, P, ctypes.c_int, ctypes.c_double,
-                                        ctypes.c_int, P]
+                                        ctypes.c_int, P, ctypes.c_int]
         lib.orc_backward_dadb.restype = None
         lib.orc_backward_dadb.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_double,
-                                          ctypes.c_int, P, P]
+                                          ctypes.c_int, P, P, ctypes.c_int]
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_num_threads.argtypes = []
         _lib = lib
@@ -184,17 +187,29 @@ def fp16_bits(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def adapter_down(X, A, r: int, pool_group: int = 1) -> np.ndarray:
+# 16-bit element formats of the layer's arrays (the compute dtype)
+FMT16 = {"bf16": 0, "fp16": 1}
+
+
+def fp16_decode(h: np.ndarray) -> np.ndarray:
+    h = _c(h, np.uint16).reshape(-1)
+    out = np.zeros(h.size, dtype=np.float64)
+    _L().orc_fp16_decode(_p(h), h.size, _p(out))
+    return out
+
+
+def adapter_down(X, A, r: int, pool_group: int = 1, dtype: str = "bf16") -> np.ndarray:
     X = _c(X, np.uint16)
     A = _c(A, np.uint16)
     M, Din = X.shape
     T = np.zeros((M, r), dtype=np.float64)
-    _L().orc_adapter_down(_p(X), M, Din, _p(A), r, pool_group, _p(T))
+    _L().orc_adapter_down(_p(X), M, Din, _p(A), r, pool_group, _p(T), FMT16[dtype])
     return T
 
 
-def forward(X, Wt, A, B, r: int, alpha: float, pool_group: int = 1):
-    """Returns (y fp64 [M, Dout], T fp64 [M, r])."""
+def forward(X, Wt, A, B, r: int, alpha: float, pool_group: int = 1, dtype: str = "bf16"):
+    """Returns (y fp64 [M, Dout], T fp64 [M, r]).  X, Wt, A, B hold bf16 or
+    fp16 bit patterns (dtype)."""
     X = _c(X, np.uint16)
     Wt = _c(Wt, np.uint16)
     A = _c(A, np.uint16)
@@ -204,11 +219,11 @@ def forward(X, Wt, A, B, r: int, alpha: float, pool_group: int = 1):
     Y = np.zeros((M, Dout), dtype=np.float64)
     T = np.zeros((M, r), dtype=np.float64)
     _L().orc_forward(_p(X), M, Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha), pool_group,
-                     _p(Y), _p(T))
+                     _p(Y), _p(T), FMT16[dtype])
     return Y, T
 
 
-def merge(Wt, A, B, r: int, alpha: float, pool_group: int = 1) -> np.ndarray:
+def merge(Wt, A, B, r: int, alpha: float, pool_group: int = 1, dtype: str = "bf16") -> np.ndarray:
     """W_eff fp64 [Dout, Din] = dequantized Wt + (alpha/r) (A B) in the stored
     orientation; pooled: (alpha/r)/g (A_p B) shared by each group's inputs."""
     Wt = _c(Wt, np.uint16)
@@ -216,20 +231,21 @@ def merge(Wt, A, B, r: int, alpha: float, pool_group: int = 1) -> np.ndarray:
     B = _c(B, np.uint16)
     Dout, Din = Wt.shape
     out = np.zeros((Dout, Din), dtype=np.float64)
-    _L().orc_merge(Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha), pool_group, _p(out))
+    _L().orc_merge(Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha), pool_group, _p(out), FMT16[dtype])
     return out
 
 
-def grad_G(dY, B, r: int) -> np.ndarray:
+def grad_G(dY, B, r: int, dtype: str = "bf16") -> np.ndarray:
     dY = _c(dY, np.uint16)
     B = _c(B, np.uint16)
     M, Dout = dY.shape
     G = np.zeros((M, r), dtype=np.float64)
-    _L().orc_grad_G(_p(dY), M, Dout, _p(B), r, _p(G))
+    _L().orc_grad_G(_p(dY), M, Dout, _p(B), r, _p(G), FMT16[dtype])
     return G
 
 
-def backward_dx(dY, Wt, A, B, r: int, alpha: float, pool_group: int = 1) -> np.ndarray:
+def backward_dx(dY, Wt, A, B, r: int, alpha: float, pool_group: int = 1,
+                dtype: str = "bf16") -> np.ndarray:
     dY = _c(dY, np.uint16)
     Wt = _c(Wt, np.uint16)
     A = _c(A, np.uint16)
@@ -238,12 +254,12 @@ def backward_dx(dY, Wt, A, B, r: int, alpha: float, pool_group: int = 1) -> np.n
     Din = Wt.shape[1]
     dX = np.zeros((M, Din), dtype=np.float64)
     _L().orc_backward_dx(_p(dY), M, Din, Dout, _p(Wt), _p(A), _p(B), r, float(alpha),
-                         pool_group, _p(dX))
+                         pool_group, _p(dX), FMT16[dtype])
     return dX
 
 
 def backward_dadb(X, dY, A, B, r: int, alpha: float, pool_group: int = 1,
-                  want_dA: bool = True, want_dB: bool = True):
+                  want_dA: bool = True, want_dB: bool = True, dtype: str = "bf16"):
     X = _c(X, np.uint16)
     dY = _c(dY, np.uint16)
     A = _c(A, np.uint16)
@@ -253,12 +269,12 @@ def backward_dadb(X, dY, A, B, r: int, alpha: float, pool_group: int = 1,
     dA = np.zeros((Din // pool_group, r), dtype=np.float64) if want_dA else None
     dB = np.zeros((r, Dout), dtype=np.float64) if want_dB else None
     _L().orc_backward_dadb(_p(X), _p(dY), M, Din, Dout, _p(A), _p(B), r, float(alpha),
-                           pool_group, _p(dA), _p(dB))
+                           pool_group, _p(dA), _p(dB), FMT16[dtype])
     return dA, dB
 
 
-def backward(X, dY, Wt, A, B, r: int, alpha: float, pool_group: int = 1):
+def backward(X, dY, Wt, A, B, r: int, alpha: float, pool_group: int = 1, dtype: str = "bf16"):
     """Returns (dX, dA, dB), all fp64."""
-    dX = backward_dx(dY, Wt, A, B, r, alpha, pool_group)
-    dA, dB = backward_dadb(X, dY, A, B, r, alpha, pool_group)
+    dX = backward_dx(dY, Wt, A, B, r, alpha, pool_group, dtype)
+    dA, dB = backward_dadb(X, dY, A, B, r, alpha, pool_group, dtype=dtype)
     return dX, dA, dB

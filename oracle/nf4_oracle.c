@@ -45,6 +45,24 @@ static double bf16_to_double(uint16_t h) {
     return (double)f;
 }
 
+/* IEEE binary16 bits -> double (exact): 1 sign, 5 exponent (bias 15) and 10
+ * fraction bits; exponent 0 holds the subnormals f * 2^-24. */
+static double fp16_to_double(uint16_t h) {
+    const int sign = h >> 15, ex = (h >> 10) & 31, fr = h & 1023;
+    double v;
+    if (ex == 0)
+        v = ldexp((double)fr, -24);
+    else if (ex == 31)
+        v = fr ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + fr), ex - 25);
+    return sign ? -v : v;
+}
+
+/* A 16-bit activation or weight element in the layer's compute dtype
+ * ([CSDN] 8.3): dt 0 = bf16, 1 = fp16. */
+static double dec16(uint16_t h, int dt) { return dt ? fp16_to_double(h) : bf16_to_double(h); }
+
 /* Round an fp32 value to bf16, round-to-nearest-even on the bit pattern. */
 static uint16_t float_to_bf16_rne(float f) {
     uint32_t u;
@@ -334,6 +352,11 @@ void orc_dequantize_dt(int64_t rows, int64_t cols, int block, const float cb[16]
     }
 }
 
+/* binary16 bits -> double, exported so tests can pin the decoding alone. */
+void orc_fp16_decode(const uint16_t *h, int64_t n, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = fp16_to_double(h[i]);
+}
+
 /* fp32 -> binary16 bits, exported so tests can pin the conversion alone. */
 void orc_fp16_bits(const float *x, int64_t n, uint16_t *out) {
     for (int64_t i = 0; i < n; ++i) out[i] = float_to_fp16_rne(x[i]);
@@ -346,23 +369,23 @@ void orc_fp16_bits(const float *x, int64_t n, uint16_t *out) {
 /* Adapter input: x itself, or with pooling ([BLOG] sections 3-4) the mean of
  * each run of g consecutive input features: p[m,k'] = (1/g) sum_i x[m,k'g+i]. */
 static double adapter_in(const uint16_t *X, int64_t Din, int64_t m, int64_t kp,
-                         int g) {
-    if (g == 1) return bf16_to_double(X[m * Din + kp]);
+                         int g, int dt) {
+    if (g == 1) return dec16(X[m * Din + kp], dt);
     double s = 0.0;
-    for (int i = 0; i < g; ++i) s += bf16_to_double(X[m * Din + kp * g + i]);
+    for (int i = 0; i < g; ++i) s += dec16(X[m * Din + kp * g + i], dt);
     return s / (double)g;
 }
 
 /* T = adapter_in(x) . A   ->  T:[M, r]   ([BLOG] section 2; [CSDN] 12.2) */
 void orc_adapter_down(const uint16_t *X, int64_t M, int64_t Din,
-                      const uint16_t *A, int r, int g, double *T) {
+                      const uint16_t *A, int r, int g, double *T, int dt) {
     const int64_t Da = Din / g;
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int j = 0; j < r; ++j) {
             double s = 0.0;
             for (int64_t k = 0; k < Da; ++k)
-                s += adapter_in(X, Din, m, k, g) * bf16_to_double(A[k * r + j]);
+                s += adapter_in(X, Din, m, k, g, dt) * dec16(A[k * r + j], dt);
             T[m * r + j] = s;
         }
 }
@@ -370,21 +393,24 @@ void orc_adapter_down(const uint16_t *X, int64_t M, int64_t Din,
 /* Forward ([BLOG] section 2 W_eff = dequant(W4) + (alpha/r) A B;
  * [CSDN] 12.4 Y = X W_hat + s X A B with s = lora_alpha / r):
  *   y[m,n] = sum_k x[m,k] Wt[n,k] + s * sum_j T[m,j] B[j,n].
- * Wt is the dequantized weight (bf16 bits, [Dout, Din]).  T may be NULL. */
+ * Wt is the dequantized weight ([Dout, Din]).  T may be NULL.  In every layer
+ * function the 16-bit arrays (x, dY, Wt, A, B) hold bf16 (dt = 0) or fp16
+ * (dt = 1) bit patterns, the compute dtype of [CSDN] 8.3; all arithmetic is
+ * fp64 either way. */
 void orc_forward(const uint16_t *X, int64_t M, int64_t Din, int64_t Dout,
                  const uint16_t *Wt, const uint16_t *A, const uint16_t *B,
-                 int r, double alpha, int g, double *Y, double *T_out) {
+                 int r, double alpha, int g, double *Y, double *T_out, int dt) {
     const double s = alpha / (double)r;
     double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
-    orc_adapter_down(X, M, Din, A, r, g, T);
+    orc_adapter_down(X, M, Din, A, r, g, T, dt);
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < Dout; ++n) {
             double base = 0.0;
             for (int64_t k = 0; k < Din; ++k)
-                base += bf16_to_double(X[m * Din + k]) * bf16_to_double(Wt[n * Din + k]);
+                base += dec16(X[m * Din + k], dt) * dec16(Wt[n * Din + k], dt);
             double ad = 0.0;
-            for (int j = 0; j < r; ++j) ad += T[m * r + j] * bf16_to_double(B[(int64_t)j * Dout + n]);
+            for (int j = 0; j < r; ++j) ad += T[m * r + j] * dec16(B[(int64_t)j * Dout + n], dt);
             Y[m * Dout + n] = base + s * ad;
         }
     if (T_out) memcpy(T_out, T, sizeof(double) * (size_t)(M * r));
@@ -393,13 +419,13 @@ void orc_forward(const uint16_t *X, int64_t M, int64_t Din, int64_t Dout,
 
 /* G = dY . B^T  ->  G:[M, r] */
 void orc_grad_G(const uint16_t *dY, int64_t M, int64_t Dout, const uint16_t *B,
-                int r, double *G) {
+                int r, double *G, int dt) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int j = 0; j < r; ++j) {
             double s = 0.0;
             for (int64_t n = 0; n < Dout; ++n)
-                s += bf16_to_double(dY[m * Dout + n]) * bf16_to_double(B[(int64_t)j * Dout + n]);
+                s += dec16(dY[m * Dout + n], dt) * dec16(B[(int64_t)j * Dout + n], dt);
             G[m * r + j] = s;
         }
 }
@@ -409,10 +435,10 @@ void orc_grad_G(const uint16_t *dY, int64_t M, int64_t Dout, const uint16_t *B,
  *   dX[m,k] = sum_n dY[m,n] Wt[n,k] + (s/g) sum_j G[m,j] A[k/g, j]. */
 void orc_backward_dx(const uint16_t *dY, int64_t M, int64_t Din, int64_t Dout,
                      const uint16_t *Wt, const uint16_t *A, const uint16_t *B,
-                     int r, double alpha, int g, double *dX) {
+                     int r, double alpha, int g, double *dX, int dt) {
     const double s = alpha / (double)r;
     double *G = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
-    orc_grad_G(dY, M, Dout, B, r, G);
+    orc_grad_G(dY, M, Dout, B, r, G, dt);
     /* Each output dX[m,k] sums n = 0..Dout-1 in ascending order; the loops
      * run n outside k only so that Wt is read row by row. */
     const int64_t KC = 256;
@@ -424,14 +450,14 @@ void orc_backward_dx(const uint16_t *dY, int64_t M, int64_t Din, int64_t Dout,
             const int64_t k0 = c * KC, k1 = k0 + KC < Din ? k0 + KC : Din;
             for (int64_t k = k0; k < k1; ++k) acc[k - k0] = 0.0;
             for (int64_t n = 0; n < Dout; ++n) {
-                const double dy = bf16_to_double(dY[m * Dout + n]);
+                const double dy = dec16(dY[m * Dout + n], dt);
                 for (int64_t k = k0; k < k1; ++k)
-                    acc[k - k0] += dy * bf16_to_double(Wt[n * Din + k]);
+                    acc[k - k0] += dy * dec16(Wt[n * Din + k], dt);
             }
             for (int64_t k = k0; k < k1; ++k) {
                 double ad = 0.0;
                 for (int j = 0; j < r; ++j)
-                    ad += G[m * r + j] * bf16_to_double(A[(k / g) * r + j]);
+                    ad += G[m * r + j] * dec16(A[(k / g) * r + j], dt);
                 dX[m * Din + k] = acc[k - k0] + s * ad / (double)g;
             }
         }
@@ -444,13 +470,13 @@ void orc_backward_dx(const uint16_t *dY, int64_t M, int64_t Din, int64_t Dout,
 void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
                        int64_t Din, int64_t Dout, const uint16_t *A,
                        const uint16_t *B, int r, double alpha, int g,
-                       double *dA, double *dB) {
+                       double *dA, double *dB, int dt) {
     const double s = alpha / (double)r;
     const int64_t Da = Din / g;
     double *G = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
     double *T = (double *)malloc(sizeof(double) * (size_t)(M * r > 0 ? M * r : 1));
-    orc_grad_G(dY, M, Dout, B, r, G);
-    orc_adapter_down(X, M, Din, A, r, g, T);
+    orc_grad_G(dY, M, Dout, B, r, G, dt);
+    orc_adapter_down(X, M, Din, A, r, g, T, dt);
     /* Each output sums m = 0..M-1 in ascending order; the loops run m
      * outside the output column so that x, dY are read row by row. */
     if (dA) {
@@ -463,7 +489,7 @@ void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
                 for (int j = 0; j < r; ++j) dA[k * r + j] = 0.0;
             for (int64_t m = 0; m < M; ++m)
                 for (int64_t k = k0; k < k1; ++k) {
-                    const double u = adapter_in(X, Din, m, k, g);
+                    const double u = adapter_in(X, Din, m, k, g, dt);
                     for (int j = 0; j < r; ++j) dA[k * r + j] += u * G[m * r + j];
                 }
             for (int64_t k = k0; k < k1; ++k)
@@ -481,7 +507,7 @@ void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
                 for (int64_t n = n0; n < n1; ++n) row[n] = 0.0;
                 for (int64_t m = 0; m < M; ++m) {
                     const double t = T[m * r + j];
-                    for (int64_t n = n0; n < n1; ++n) row[n] += t * bf16_to_double(dY[m * Dout + n]);
+                    for (int64_t n = n0; n < n1; ++n) row[n] += t * dec16(dY[m * Dout + n], dt);
                 }
                 for (int64_t n = n0; n < n1; ++n) row[n] *= s;
             }
@@ -501,15 +527,15 @@ void orc_backward_dadb(const uint16_t *X, const uint16_t *dY, int64_t M,
  * x . W_eff^T equals the layer's forward, since pool(x) averages a group.
  * Wt is the bf16 dequantized weight; the result is exact fp64 arithmetic on it. */
 void orc_merge(int64_t Din, int64_t Dout, const uint16_t *Wt, const uint16_t *A,
-               const uint16_t *B, int r, double alpha, int g, double *out) {
+               const uint16_t *B, int r, double alpha, int g, double *out, int dt) {
     const double s = alpha / (double)r;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < Dout; ++n)
         for (int64_t k = 0; k < Din; ++k) {
             double ad = 0.0;
             for (int j = 0; j < r; ++j)
-                ad += bf16_to_double(A[(k / g) * r + j]) * bf16_to_double(B[(int64_t)j * Dout + n]);
-            out[n * Din + k] = bf16_to_double(Wt[n * Din + k]) + (s / (double)g) * ad;
+                ad += dec16(A[(k / g) * r + j], dt) * dec16(B[(int64_t)j * Dout + n], dt);
+            out[n * Din + k] = dec16(Wt[n * Din + k], dt) + (s / (double)g) * ad;
         }
 }
 

@@ -192,3 +192,69 @@ def test_no_weight_gradient_and_shapes(orc):
     out = orc.backward(X, dY, Wt, A, B, 1, 1.0)
     assert len(out) == 3
     assert out[0].shape == (2, 64) and out[1].shape == (64, 1) and out[2].shape == (1, 4)
+
+
+# ---------------------------------------------------------------- fp16 compute dtype
+# The article's section 8.3 lets the layer's arithmetic run in FP16 as well as
+# BF16; the oracle's layer functions read either format (fp64 arithmetic).
+
+def test_fp16_decode_exhaustive(orc):
+    """Every one of the 65536 binary16 patterns decodes to numpy's value."""
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = orc.fp16_decode(h)
+    want = h.view(np.float16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+
+
+def _both_formats(rng, shape, scale):
+    """Values with at most 8 significant bits inside fp16's normal range: the
+    same numbers in bf16 and in fp16 bit patterns."""
+    mant = rng.integers(128, 256, shape) * rng.choice([-1, 1], shape)
+    ex = rng.integers(-14, -6, shape)
+    v = (mant * np.exp2(ex - 7.0) * scale).astype(np.float32)
+    return v.view(np.uint32).astype(np.uint64) >> 16, v.astype(np.float16).view(np.uint16)
+
+
+@pytest.mark.parametrize("g", [1, 64])
+def test_fp16_layer_equals_bf16_on_shared_values(orc, g):
+    """On values both formats hold exactly, the fp16 layer equals the bf16
+    layer bit for bit (same fp64 sums in the same order), for every output:
+    y, T, dX, dA, dB and the merge; and it matches a float64 matmul."""
+    rng = np.random.default_rng(3 + g)
+    M, Din, Dout, r, alpha = 5, 128, 72, 8, 16.0
+    xb, xh = _both_formats(rng, (M, Din), 1.0)
+    wb, wh = _both_formats(rng, (Dout, Din), 1.0)
+    ab, ah = _both_formats(rng, (Din // g, r), 1.0)
+    bb, bh = _both_formats(rng, (r, Dout), 1.0)
+    db, dh = _both_formats(rng, (M, Dout), 1.0)
+    xb, wb, ab, bb, db = (a.astype(np.uint16) for a in (xb, wb, ab, bb, db))
+    yb, Tb = orc.forward(xb, wb, ab, bb, r, alpha, g)
+    yh, Th = orc.forward(xh, wh, ah, bh, r, alpha, g, dtype="fp16")
+    assert np.array_equal(yb, yh) and np.array_equal(Tb, Th)
+    for fb, fh in zip(orc.backward(xb, db, wb, ab, bb, r, alpha, g),
+                      orc.backward(xh, dh, wh, ah, bh, r, alpha, g, dtype="fp16")):
+        assert np.array_equal(fb, fh)
+    assert np.array_equal(orc.merge(wb, ab, bb, r, alpha, g), orc.merge(wh, ah, bh, r, alpha, g, "fp16"))
+    f = lambda h: h.view(np.float16).astype(np.float64)
+    u = f(xh) if g == 1 else f(xh).reshape(M, Din // g, g).mean(axis=2)
+    ref = f(xh) @ f(wh).T + (alpha / r) * (u @ f(ah)) @ f(bh)
+    assert np.allclose(yh, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp16_layer_reads_fp16_values(orc):
+    """Values bf16 cannot hold (11 significant bits): the fp16 forward matches
+    a float64 matmul of the decoded fp16 inputs, and differs from reading the
+    same bits as bf16."""
+    rng = np.random.default_rng(9)
+    M, Din, Dout, r, alpha = 3, 64, 40, 4, 8.0
+    h = lambda shape: rng.standard_normal(shape).astype(np.float16).view(np.uint16)
+    x, w, a, b = h((M, Din)), h((Dout, Din)), h((Din, r)), h((r, Dout))
+    y, _ = orc.forward(x, w, a, b, r, alpha, dtype="fp16")
+    f = lambda v: v.view(np.float16).astype(np.float64)
+    ref = f(x) @ f(w).T + (alpha / r) * (f(x) @ f(a)) @ f(b)
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    yb, _ = orc.forward(x, w, a, b, r, alpha)
+    assert not np.allclose(yb, y)
