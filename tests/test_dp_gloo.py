@@ -69,3 +69,46 @@ def test_two_rank_adapter_grad_allreduce():
     for r in range(2):
         np.testing.assert_allclose(res[r][0], dA, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(res[r][1], dB, rtol=1e-12, atol=1e-12)
+
+
+def _leaving_worker(rank, world, port, out):
+    """Rank 1 completes one exchange, then leaves between steps without its
+    second collective; rank 0's second exchange must end in an error within the
+    process group's short timeout rather than wait for ever."""
+    import datetime
+    import time
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    dA, dB = torch.ones(4, 2, dtype=torch.float64), torch.ones(2, 3, dtype=torch.float64)
+    allreduce_adapter_grads(dA, dB)
+    out[f"step1_{rank}"] = float(dA.sum())
+    if rank == 1:
+        os._exit(0)                              # leaves between steps, nothing in flight
+    t0 = time.monotonic()
+    try:
+        allreduce_adapter_grads(dA, dB)
+        out["error"] = None
+    except Exception as e:                       # the backend's timeout or connection error
+        out["error"] = type(e).__name__
+    out["waited_s"] = time.monotonic() - t0
+    os._exit(0)
+
+
+def test_rank_leaving_surfaces_as_error():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        res = dict(out)
+    assert res["step1_0"] == res["step1_1"] == 16.0      # the first exchange summed both ranks
+    assert res["error"] is not None, "the surviving rank's collective returned without its peer"
+    assert res["waited_s"] < 60
