@@ -147,3 +147,26 @@ def test_binding_requires_cuda_tensors(lib):
     W = torch.zeros(64, 64)
     with pytest.raises(TypeError):
         q.quantize(W)
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/qlora.h is a C ABI: it compiles as strict C99 (and as C++),
+    with no torch, CUDA or C++ types in its signatures."""
+    import shutil
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text('#include "qlora.h"\n'
+                   "int main(void) { nf4_weight_t w = {0}; (void)w;\n"
+                   "  return qlora_version() > 0 ? 0 : 1; }\n")
+    inc = os.path.join(ROOT, "include")
+    for cc, flags in (("gcc", ["-std=c99", "-pedantic-errors", "-Wall", "-Werror"]),
+                      ("g++", ["-std=c++17", "-Wall", "-Werror", "-x", "c++"])):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not installed")
+        r = subprocess.run([cc, *flags, "-I", inc, "-fsyntax-only", str(src)],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+    text = open(os.path.join(inc, "qlora.h")).read()
+    code = re.sub(r"//[^\n]*", "", re.sub(r"/\*.*?\*/", "", text, flags=re.S))   # comments may name them
+    for word in ("torch", "at::", "cudaStream_t", "__nv_bfloat16", "std::"):
+        assert word not in code, word
