@@ -258,3 +258,77 @@ def test_fp16_layer_reads_fp16_values(orc):
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
     yb, _ = orc.forward(x, w, a, b, r, alpha)
     assert not np.allclose(yb, y)
+
+
+# ---------------------------------------------------------------- backward over several column chunks
+
+@pytest.mark.parametrize("pool_group", [1, 64])
+def test_backward_multichunk(orc, pool_group):
+    """Din = 640 and Dout = 2112 run the backward's dX over three input
+    chunks (the last one ragged) and dB over three output chunks (ragged), at
+    M = 3.  Three facts from the chain rule ("大模型量化从0到1（十）" 12.4) pin
+    every entry:
+
+    - finite differences at each chunk's first and last column;
+    - Euler's identity: L = sum(dY * y) is linear and homogeneous in x, so
+      L = <dX, x> exactly;
+    - the adapter part of L is linear and homogeneous in A and in B, so
+      L - L(B = 0) = <dA, A> = <dB, B>.
+
+    A wrong chunk bound leaves some entries unwritten or summed twice, which
+    breaks one of them."""
+    rng = np.random.default_rng(41 + pool_group)
+    M, Din, Dout, r, alpha = 3, 640, 2112, 3, 7.0
+    W, X, A, B, dY = _problem(rng, M, Din, Dout, r)
+    if pool_group > 1:
+        A = bf16(rng.standard_normal((Din // pool_group, r)))
+    cb = orc.nf4_codebook()
+    Wt = orc.dequantize(orc.quantize(W, cb, True), cb)
+    dX, dA, dB = orc.backward(X, dY, Wt, A, B, r, alpha, pool_group)
+    dyf = f64(dY)
+
+    def loss(X_, A_, B_):
+        Y, _ = orc.forward(X_, Wt, A_, B_, r, alpha, pool_group)
+        return float(np.sum(dyf * Y))
+
+    L0 = loss(X, A, B)
+    L_base = loss(X, A, np.zeros_like(B))
+    assert L0 == pytest.approx(float(np.sum(dX * f64(X))), rel=1e-10)
+    assert L0 - L_base == pytest.approx(float(np.sum(dB * f64(B))), rel=1e-9)
+    assert L0 - L_base == pytest.approx(float(np.sum(dA * f64(A))), rel=1e-9)
+
+    def fd(arr, idx, which):
+        old = f64(arr[idx])
+        new = old + 0.5 if abs(old) < 4 else old * 1.5
+        arr2 = arr.copy()
+        arr2[idx] = bf16(new)
+        h = f64(arr2[idx]) - old
+        args = {"X": (arr2, A, B), "A": (X, arr2, B), "B": (X, A, arr2)}[which]
+        return (loss(*args) - L0) / h
+
+    for m, k in [(0, 0), (1, 255), (2, 256), (0, 511), (1, 512), (2, 639)]:
+        assert fd(X, (m, k), "X") == pytest.approx(dX[m, k], rel=1e-8, abs=1e-9)
+    a_rows = [0, A.shape[0] - 1] + ([63, 64, 600] if pool_group == 1 else [4])
+    for k in a_rows:
+        assert fd(A, (k, k % r), "A") == pytest.approx(dA[k, k % r], rel=1e-8, abs=1e-9)
+    for j, n in [(0, 0), (1, 1023), (2, 1024), (0, 2047), (1, 2048), (2, 2111)]:
+        assert fd(B, (j, n), "B") == pytest.approx(dB[j, n], rel=1e-8, abs=1e-9)
+
+
+@pytest.mark.parametrize("pool_group", [1, 64])
+def test_backward_multichunk_B_zero_is_plain_matmul(orc, pool_group):
+    """B = 0 at the multi-chunk sizes: dX = dY . dequant(W4) as numpy's matmul
+    computes it, dA = 0, and dB = s (u A)^T dY with u = x or pool(x)."""
+    rng = np.random.default_rng(51 + pool_group)
+    M, Din, Dout, r, alpha = 4, 640, 2112, 2, 6.0
+    W, X, A, B, dY = _problem(rng, M, Din, Dout, r)
+    if pool_group > 1:
+        A = bf16(rng.standard_normal((Din // pool_group, r)))
+    B[:] = 0
+    cb = orc.nf4_codebook()
+    Wt = orc.dequantize(orc.quantize(W, cb, False), cb)
+    dX, dA, dB = orc.backward(X, dY, Wt, A, B, r, alpha, pool_group)
+    np.testing.assert_allclose(dX, f64(dY) @ f64(Wt), rtol=1e-12, atol=1e-12)
+    assert np.all(dA == 0)
+    u = f64(X) if pool_group == 1 else f64(X).reshape(M, -1, pool_group).mean(axis=2)
+    np.testing.assert_allclose(dB, (alpha / r) * (u @ f64(A)).T @ f64(dY), rtol=1e-12, atol=1e-12)
