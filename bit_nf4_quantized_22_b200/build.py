@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqlora.so")
 SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "adapter.cu", "umma_gemm.cu", "profile.cu", "noalloc.cu", "umma_skinny.cu", "merge.cu", "selftest.cu"]
-HEADERS = ["common.cuh", "mma_gemm.cuh", "tcgen05.cuh"]
+HEADERS = ["common.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -5,11 +5,13 @@
 //   dA = s u^T G      dB = s T^T dY
 //
 // (LoRA/QLoRA/QA-LoRA blog sections 2-5; bitsandbytes article (CSDN) 12.2.)
-// All four are skinny GEMMs run on the warp-MMA tiled GEMM.  fp32 operands
-// (T, G, pool(x)) are carried as two bf16 terms hi + lo, hi = RN_bf16(v),
-// lo = RN_bf16(v - hi), which keeps ~16 mantissa bits; the GEMM multiplies
-// both terms and the reduce kernel adds the two halves in fp32.
-#include "mma_gemm.cuh"
+// The four products themselves run on the tcgen05 skinny GEMM (umma_skinny.cu);
+// this file holds the helpers around them: adapter padding, pooling, the
+// hi/lo split of fp32 operands and the deterministic split-K reduce.  fp32
+// operands (T, G, pool(x)) are carried as two bf16 terms hi + lo,
+// hi = RN_bf16(v), lo = RN_bf16(v - hi), which keeps ~16 mantissa bits; the
+// GEMM multiplies both terms and the reduce kernel adds the two halves in fp32.
+#include "common.cuh"
 
 namespace qlora {
 namespace {
@@ -187,38 +189,6 @@ int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H
     }
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
-}
-
-// ---------------------------------------------------------------- GEMM launcher
-
-template <int BM, int BN>
-static int run_mma_gemm(MmaGemmArgs a, cudaStream_t st) {
-    using S = MmaSmem<BM, BN>;
-    cudaFuncSetAttribute(k_mma_gemm<BM, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)S::BYTES);
-    dim3 grid((unsigned)((a.Q + BN - 1) / BN), (unsigned)((a.P + BM - 1) / BM), (unsigned)a.splits);
-    k_mma_gemm<BM, BN><<<grid, kMmaThreads, S::BYTES, st>>>(a);
-    QLORA_LAUNCH_CHECK();
-    return QLORA_OK;
-}
-
-// Number of k-splits that fills the machine for a (P, Q, R) problem, capped
-// so each split keeps >= 8 k-tiles.  The caller sizes `partial` with
-// mma_partial_floats().
-int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN) {
-    const int64_t tiles = ((P + 127) / 128) * ((Q + BN - 1) / BN);
-    const int64_t nkt = (Rtot + kMmaBK - 1) / kMmaBK;
-    int64_t s = 2 * (int64_t)device_sms() / tiles;   // one wave of two CTAs per SM
-    const int64_t cap = nkt / 8 > 1 ? nkt / 8 : 1;
-    if (s > cap) s = cap;
-    if (s > 32) s = 32;
-    return (int)(s < 1 ? 1 : s);
-}
-
-int launch_mma_gemm(MmaGemmArgs a, int bn, cudaStream_t st) {
-    if (a.P <= 0 || a.Q <= 0) return QLORA_OK;
-    if (bn == 128) return run_mma_gemm<128, 128>(a, st);
-    return run_mma_gemm<128, 64>(a, st);
 }
 
 }  // namespace qlora

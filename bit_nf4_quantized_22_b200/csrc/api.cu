@@ -1,12 +1,10 @@
 // api.cu -- the extern "C" entry points declared in include/qlora.h:
 // argument validation, workspace layout and kernel dispatch.
 #include <cmath>
-#include <cstdlib>
-#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
-#include "mma_gemm.cuh"
+#include "common.cuh"
 
 namespace qlora {
 // quantize.cu
@@ -38,8 +36,6 @@ int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *ds
 int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H, int Qv,
                   float f32_scale, float *out_f32, int64_t fsp, int64_t fsq, float bf_scale,
                   uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp, cudaStream_t st);
-int mma_choose_splits(int64_t P, int64_t Q, int64_t Rtot, int BN);
-int launch_mma_gemm(MmaGemmArgs a, int bn, cudaStream_t st);
 // umma_skinny.cu
 struct SkinnySeg {
     const uint16_t *a;
@@ -107,11 +103,6 @@ int check_weight(const nf4_weight_t *q, bool need_rows, bool codec = false) {
     return QLORA_OK;
 }
 
-bool large_path_uses_mma() {
-    const char *e = std::getenv("QLORA_LARGE_M_PATH");
-    return e && std::strcmp(e, "mma") == 0;
-}
-
 // Bump allocator over the caller's workspace (256-byte aligned pieces).
 struct Bump {
     uintptr_t base;
@@ -130,7 +121,7 @@ struct Dims {
     int64_t M, Din, Dout;
     int r, rp, rp64, g;
     int64_t Da, Dap;
-    bool small, mma_large;
+    bool small;
 };
 
 Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
@@ -145,14 +136,12 @@ Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
     d.Da = d.Din / g;
     d.Dap = round_up(d.Da, 8);
     d.small = M <= kGemvMaxM;
-    d.mma_large = !d.small && large_path_uses_mma();
     return d;
 }
 
 // ---------------------------------------------------------------- adapter products
 // C[P, Q] = sum over segments of A(p,t) B(t,q), as fp32 split-K partials
-// [splits][P][Qp]; run on the tcgen05 engine, or on the warp-MMA engine when
-// the warp-MMA path is selected.
+// [splits][P][Qp], on the tcgen05 skinny-GEMM engine.
 struct Prod {
     SkinnySeg seg[2];
     int nseg;
@@ -163,41 +152,22 @@ struct ProdPlan {
     int64_t Qp;
 };
 
-ProdPlan plan_prod(const Prod &pr, bool mma) {
+ProdPlan plan_prod(const Prod &pr) {
     ProdPlan pl;
-    if (mma) {
-        int64_t R = 0;
-        for (int i = 0; i < pr.nseg; ++i) R += pr.seg[i].R;
-        pl.splits = mma_choose_splits(pr.P, pr.Q, R, pr.Q <= 64 ? 64 : 128);
-        pl.Qp = pr.Q;
-    } else {
-        int per = 1;
-        skinny_splits(pr.P, pr.Q, skinny_k_tiles(pr.seg, pr.nseg), &pl.splits, &per);
-        pl.Qp = round_up(pr.Q, 4);
-    }
+    int per = 1;
+    skinny_splits(pr.P, pr.Q, skinny_k_tiles(pr.seg, pr.nseg), &pl.splits, &per);
+    pl.Qp = round_up(pr.Q, 4);
     return pl;
 }
 
-size_t prod_partial_floats(const Prod &pr, bool mma) {
-    const ProdPlan pl = plan_prod(pr, mma);
+size_t prod_partial_floats(const Prod &pr) {
+    const ProdPlan pl = plan_prod(pr);
     return (size_t)pl.splits * pr.P * pl.Qp;
 }
 
-int run_prod(const Prod &pr, bool mma, float *partial, uint32_t *status, cudaStream_t st,
-             ProdPlan *plan) {
-    *plan = plan_prod(pr, mma);
-    if (!mma) return launch_umma_skinny(pr.seg, pr.nseg, pr.P, pr.Q, plan->Qp, partial, status, st);
-    MmaGemmArgs a{};
-    for (int i = 0; i < pr.nseg; ++i) {
-        const SkinnySeg &g = pr.seg[i];
-        a.seg[i] = MmaSeg{MmaOperand{g.a, g.lda, g.a_kmajor}, MmaOperand{g.b, g.ldb, g.b_kmajor}, g.R};
-    }
-    a.nseg = pr.nseg;
-    a.P = pr.P;
-    a.Q = pr.Q;
-    a.splits = plan->splits;
-    a.partial = partial;
-    return launch_mma_gemm(a, pr.Q <= 64 ? 64 : 128, st);
+int run_prod(const Prod &pr, float *partial, uint32_t *status, cudaStream_t st, ProdPlan *plan) {
+    *plan = plan_prod(pr);
+    return launch_umma_skinny(pr.seg, pr.nseg, pr.P, pr.Q, plan->Qp, partial, status, st);
 }
 
 // T = u . A    (u = x [M, Din], or pooled hi/lo [M, Dap]; A padded [Da, rp])
@@ -253,11 +223,11 @@ Prod prod_dB(const Dims &d, const uint16_t *dY, const uint16_t *Tsplit) {
 
 // Workspace pieces.  The same function sizes (base == nullptr) and carves.
 struct FwdWs {
-    uint16_t *Apad, *ph, *pl, *sT, *Wdeq;
+    uint16_t *Apad, *ph, *pl, *sT;
     float *T32, *Tpart, *gemv_part, *gemv_tpart;
 };
 struct BwdWs {
-    uint16_t *Apad, *ph, *pl, *sG, *Gsplit, *Tsplit, *Aext, *Wdeq;
+    uint16_t *Apad, *ph, *pl, *sG, *Gsplit, *Tsplit, *Aext;
     float *G32, *Gpart, *T32, *Tpart, *dApart, *dBpart, *gemv_part;
 };
 
@@ -270,13 +240,12 @@ size_t layout_fwd(const Dims &d, bool have_tsave, void *base, FwdWs *w) {
         x.pl = b.take<uint16_t>(d.M * d.Dap);
     }
     if (!have_tsave) x.T32 = b.take<float>(d.M * d.r);
-    x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0), d.mma_large));
+    x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0)));
     if (d.small) {
         x.gemv_part = b.take<float>(gemv_fwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
         if (d.g == 1) x.gemv_tpart = b.take<float>(gemv_fwd_tpart_floats((int)d.M, d.Din, d.r));
     } else {
         x.sT = b.take<uint16_t>(d.M * d.rp64);
-        if (d.mma_large) x.Wdeq = b.take<uint16_t>(d.Dout * d.Din);
     }
     if (w) *w = x;
     return b.off;
@@ -287,7 +256,7 @@ size_t layout_bwd(const Dims &d, bool have_tsaved, bool want_dx, bool want_da, b
     Bump b(base);
     BwdWs x{};
     x.G32 = b.take<float>(d.M * d.r);
-    x.Gpart = b.take<float>(prod_partial_floats(prod_G(d, 0, 0), d.mma_large));
+    x.Gpart = b.take<float>(prod_partial_floats(prod_G(d, 0, 0)));
     if (want_da) x.Gsplit = b.take<uint16_t>(d.M * 2 * d.rp);
     if (d.g > 1 && (want_da || (want_db && !have_tsaved))) {
         x.ph = b.take<uint16_t>(d.M * d.Dap);
@@ -297,23 +266,18 @@ size_t layout_bwd(const Dims &d, bool have_tsaved, bool want_dx, bool want_da, b
         if (!have_tsaved) {
             x.Apad = b.take<uint16_t>(d.Da * d.rp);
             x.T32 = b.take<float>(d.M * d.r);
-            x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0), d.mma_large));
+            x.Tpart = b.take<float>(prod_partial_floats(prod_T(d, 0, 0, 0, 0)));
         }
         x.Tsplit = b.take<uint16_t>(d.M * 2 * d.rp);
-        x.dBpart = b.take<float>(prod_partial_floats(prod_dB(d, 0, 0), d.mma_large));
+        x.dBpart = b.take<float>(prod_partial_floats(prod_dB(d, 0, 0)));
     }
-    if (want_da) x.dApart = b.take<float>(prod_partial_floats(prod_dA(d, 0, 0, 0, 0), d.mma_large));
+    if (want_da) x.dApart = b.take<float>(prod_partial_floats(prod_dA(d, 0, 0, 0, 0)));
     if (want_dx) {
         if (d.small) {
             x.gemv_part = b.take<float>(gemv_bwd_partial_bytes((int)d.M, d.Din, d.Dout) / 4 + 1);
         } else {
             x.sG = b.take<uint16_t>(d.M * d.rp64);
-            if (d.mma_large) {
-                x.Aext = b.take<uint16_t>(d.Din * d.rp);
-                x.Wdeq = b.take<uint16_t>(d.Dout * d.Din);
-            } else {
-                x.Aext = b.take<uint16_t>(d.Din * d.rp64);
-            }
+            x.Aext = b.take<uint16_t>(d.Din * d.rp64);
         }
     }
     if (w) *w = x;
@@ -357,7 +321,7 @@ int run_adapter_down(const Dims &d, const uint16_t *X, const uint16_t *A, uint16
         Ause = Apad;
     }
     ProdPlan plan;
-    RC(run_prod(prod_T(d, X, Ause, ph, pl), d.mma_large, Tpart, status, st, &plan));
+    RC(run_prod(prod_T(d, X, Ause, ph, pl), Tpart, status, st, &plan));
     if (sT && cudaMemsetAsync(sT, 0, d.M * d.rp64 * sizeof(uint16_t), st) != cudaSuccess)
         return QLORA_ECUDA;
     return launch_reduce(Tpart, plan.splits, d.M, plan.Qp, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
@@ -475,21 +439,7 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
     RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT,
                         d_status, st));
     if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, d_status, st);
-    if (!d.mma_large) return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
-    // warp-MMA path: dequantize to a bf16 copy, then one two-segment GEMM
-    RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));
-    MmaGemmArgs a{};
-    a.seg[0] = MmaSeg{MmaOperand{X, d.Din, 1}, MmaOperand{w.Wdeq, d.Din, 1}, d.Din};
-    a.seg[1] = MmaSeg{MmaOperand{w.sT, d.rp64, 1}, MmaOperand{B, d.Dout, 0}, (int64_t)r};
-    a.nseg = 2;
-    a.P = M;
-    a.Q = d.Dout;
-    a.out_scale = 1.f;
-    a.out_bf16 = Y;
-    a.bf_sp = d.Dout;
-    a.bf_sq = 1;
-    a.splits = 1;
-    return launch_mma_gemm(a, 128, st);
+    return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
 }
 
 // A second stream per device for the backward's adapter-gradient products,
@@ -533,7 +483,7 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     // G = dY . B^T  (fp32), s*G (bf16, large M), hi/lo split (for dA)
     {
         ProdPlan pl;
-        RC(run_prod(prod_G(d, dY, B), d.mma_large, w.Gpart, d_status, st, &pl));
+        RC(run_prod(prod_G(d, dY, B), w.Gpart, d_status, st, &pl));
         uint16_t *sG = (want_dx && !d.small) ? w.sG : nullptr;
         if (sG && cudaMemsetAsync(sG, 0, M * d.rp64 * 2, st) != cudaSuccess) return QLORA_ECUDA;
         if (w.Gsplit && cudaMemsetAsync(w.Gsplit, 0, M * 2 * d.rp * 2, st) != cudaSuccess)
@@ -548,7 +498,7 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     // adapter products take the SMs its last wave leaves free.
     cudaStream_t side = nullptr;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-    if (want_dx && !d.small && !d.mma_large && (want_da || want_db)) {
+    if (want_dx && !d.small && (want_da || want_db)) {
         side = side_stream();
         if (side && (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
                      cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess ||
@@ -560,7 +510,7 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     if (want_dx) {
         if (d.small) {
             RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st));
-        } else if (!d.mma_large) {
+        } else {
             // the extension operand is A itself when no padding, pooling or scaling applies
             const bool direct = d.g == 1 && r == d.rp64 && aligned16(A);
             int rcx = direct ? QLORA_OK : launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st);
@@ -571,28 +521,13 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
                 if (ev_join) cudaEventDestroy(ev_join);
                 return rcx;
             }
-        } else {
-            RC(launch_pad_rows(A, d.Din, r, d.rp, d.g, 1.f / d.g, w.Aext, st));
-            RC(launch_nf4_dequantize(*q, cb, w.Wdeq, st));
-            MmaGemmArgs a{};
-            a.seg[0] = MmaSeg{MmaOperand{dY, d.Dout, 1}, MmaOperand{w.Wdeq, d.Din, 0}, d.Dout};
-            a.seg[1] = MmaSeg{MmaOperand{w.sG, d.rp64, 1}, MmaOperand{w.Aext, d.rp, 1}, (int64_t)r};
-            a.nseg = 2;
-            a.P = M;
-            a.Q = d.Din;
-            a.out_scale = 1.f;
-            a.out_bf16 = dX;
-            a.bf_sp = d.Din;
-            a.bf_sq = 1;
-            a.splits = 1;
-            RC(launch_mma_gemm(a, 128, st));
         }
     }
     int rc = QLORA_OK;
     if (side && cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess) rc = QLORA_ECUDA;
     if (rc == QLORA_OK && want_da) {
         ProdPlan pl;
-        rc = run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), d.mma_large, w.dApart, d_status, ast, &pl);
+        rc = run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), w.dApart, d_status, ast, &pl);
         if (rc == QLORA_OK)
             rc = launch_reduce(w.dApart, pl.splits, d.Da, pl.Qp, d.rp, r, s, dA, r, 1, 0.f, nullptr,
                                0, nullptr, 0, ast);
@@ -607,7 +542,7 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
         if (rc == QLORA_OK) rc = launch_split_f32(T32, M, r, d.rp, w.Tsplit, ast);
         ProdPlan pl;
         if (rc == QLORA_OK)
-            rc = run_prod(prod_dB(d, dY, w.Tsplit), d.mma_large, w.dBpart, d_status, ast, &pl);
+            rc = run_prod(prod_dB(d, dY, w.Tsplit), w.dBpart, d_status, ast, &pl);
         if (rc == QLORA_OK)
             rc = launch_reduce(w.dBpart, pl.splits, d.Dout, pl.Qp, d.rp, r, s, dB, 1, d.Dout, 0.f,
                                nullptr, 0, nullptr, 0, ast);

@@ -169,13 +169,3 @@ def test_config5_large_sampled(orc, qlib, lin):
     run_case(orc, qlib, spec, 8192, 5, lin=lin, rows=rows, arrays=a, check_dadb=False)
     small = dict(W=a["W"], A=a["A"], B=a["B"], x=a["x"][:512].copy(), dY=a["dY"][:512].copy())
     run_case(orc, qlib, spec, 512, 5, lin=lin, arrays=small)
-
-
-@pytest.mark.parametrize("M", [17, 300])
-def test_warp_mma_large_path(orc, qlib, M, monkeypatch):
-    """The alternative large-M path (dequantize + warp-MMA GEMM) agrees too."""
-    monkeypatch.setenv("QLORA_LARGE_M_PATH", "mma")
-    spec = LinearSpec("t", 192, 200, 8, 16.0, True)
-    run_case(orc, qlib, spec, M, 16)
-    spec = LinearSpec("p", 512, 136, 8, 8.0, True, pool_group=64)
-    run_case(orc, qlib, spec, M, 17)
