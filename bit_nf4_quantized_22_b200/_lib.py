@@ -21,6 +21,7 @@ EXPORTS = (
     "nf4_dequantize", "qlora_workspace_size", "qlora_forward", "qlora_backward",
     "qlora_launch_count", "qlora_profile_enable", "qlora_profile_reset", "qlora_profile_read",
     "qlora_forward_noalloc", "qlora_merge", "qlora_selftest_wait_timeout", "nf4_dequantize_dtype",
+    "nf4_codebook",
 )
 
 
@@ -95,6 +96,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_selftest_wait_timeout.argtypes = [P, P]
     lib.qlora_merge.restype = ctypes.c_int
     lib.qlora_merge.argtypes = [W, P, P, P, i32, ctypes.c_float, i32, P, P]
+    lib.nf4_codebook.restype = ctypes.c_int
+    lib.nf4_codebook.argtypes = [ctypes.c_double, P]
     _lib = lib
     return lib
 

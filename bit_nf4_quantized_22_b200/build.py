@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqlora.so")
-SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "adapter.cu", "umma_gemm.cu", "profile.cu", "noalloc.cu", "umma_skinny.cu", "merge.cu", "selftest.cu"]
+SOURCES = ["api.cu", "codebook.cpp", "quantize.cu", "gemv.cu", "adapter.cu", "umma_gemm.cu", "profile.cu", "noalloc.cu", "umma_skinny.cu", "merge.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [

@@ -92,6 +92,23 @@ const char *qlora_strerror(int code);
 /* Library ABI version (major*100 + minor). */
 int qlora_version(void);
 
+/* nf4_codebook -- the 16 NF4 levels, built on the host (no device work).
+ * "QLoRA：用4比特行李箱装下整个大模型" chapter 3: the levels are standard-normal
+ * quantiles of equal-probability pieces of the CDF; bitsandbytes article (CSDN)
+ * section 6.2: one fixed table, normalised to [-1, 1], built asymmetrically
+ * around an exact 0.  With Phi^-1 the standard normal quantile:
+ *   out[0..6]  = -Phi^-1(delta + (1/2 - delta) i / 7) / Phi^-1(delta), i = 0..6
+ *   out[7]     = 0
+ *   out[15-i]  =  Phi^-1(delta + (1/2 - delta) i / 8) / Phi^-1(delta), i = 0..7
+ * each rounded once to fp32, so out[0] = -1, out[15] = +1 and the table is
+ * strictly increasing.  QLORA_NF4_DELTA, 1 - (1/32 + 1/30)/2, is the mean of
+ * the outermost interval-midpoint probabilities for 16 and for 15 pieces.
+ *   delta   in (1/2, 1)
+ *   out     host fp32[16] (output, caller-owned)
+ * Errors: EINVAL for a NULL out or delta outside (1/2, 1). */
+#define QLORA_NF4_DELTA 0.96770833333333333333
+int nf4_codebook(double delta, float out[16]);
+
 /* Host-side check of a codebook (no device work): 16 finite fp32 values,
  * strictly increasing, inside [-1, 1], one of them exactly 0.
  * Returns QLORA_OK or QLORA_EINVAL. */

@@ -137,10 +137,23 @@ def test_workspace_size_deterministic(lib):
     assert lib.qlora_workspace_size(4, ctypes.byref(_wc()), 0, 1, 0) == 0
 
 
-def test_product_codebook_matches_oracle(orc):
-    a = q.nf4_codebook().numpy()
-    b = orc.nf4_codebook()
+@pytest.mark.parametrize("delta", [None, 1 - 1 / 32, 0.9, 0.99, 0.75, 0.999])
+def test_product_codebook_matches_oracle(orc, delta):
+    """The library's nf4_codebook (its own inverse normal: AS 241 plus a
+    Halley step) gives the oracle's table (bisection on erfc) bit for bit."""
+    a = (q.nf4_codebook() if delta is None else q.nf4_codebook(delta)).numpy()
+    b = orc.nf4_codebook() if delta is None else orc.nf4_codebook(delta)
     assert np.array_equal(a.view(np.int32), b.view(np.int32))
+    assert a[0] == -1 and a[7] == 0 and a[15] == 1
+
+
+def test_codebook_call_rejects_bad_delta(lib):
+    out = (ctypes.c_float * 16)()
+    for bad in (0.5, 0.3, 1.0, 1.5, float("nan")):
+        assert lib.nf4_codebook(bad, out) == _lib.QLORA_EINVAL
+    assert lib.nf4_codebook(0.9, None) == _lib.QLORA_EINVAL
+    assert lib.nf4_codebook(0.9677083333333333, out) == 0
+    assert lib.qlora_check_codebook(out) == 0
 
 
 def test_binding_requires_cuda_tensors(lib):
