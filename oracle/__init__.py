@@ -57,6 +57,8 @@ def _L():
         lib.orc_normal_ppf.argtypes = [ctypes.c_double]
         lib.orc_nf4_codebook.restype = None
         lib.orc_nf4_codebook.argtypes = [ctypes.c_double, P]
+        lib.orc_fp4_codebook.restype = None
+        lib.orc_fp4_codebook.argtypes = [P]
         lib.orc_quantize.restype = ctypes.c_int
         lib.orc_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
                                      P]
@@ -115,6 +117,13 @@ def normal_ppf(p: float) -> float:
 def nf4_codebook(delta: float = NF4_DELTA) -> np.ndarray:
     out = np.zeros(16, dtype=np.float32)
     _L().orc_nf4_codebook(float(delta), _p(out))
+    return out
+
+
+def fp4_codebook() -> np.ndarray:
+    """The FP4 (E2M1 / 6) table: 16 non-decreasing fp32 levels, -0 before +0."""
+    out = np.zeros(16, dtype=np.float32)
+    _L().orc_fp4_codebook(_p(out))
     return out
 
 

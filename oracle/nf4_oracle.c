@@ -149,6 +149,26 @@ void orc_nf4_codebook(double delta, float out[16]) {
     for (int i = 0; i < 16; ++i) out[i] = (float)v[i];
 }
 
+/* The FP4 codebook ([CSDN] 6.4-6.5, 9.3: bitsandbytes' other 4-bit type, and
+ * its configuration default, is a "4-bit float-style" table, not uniform
+ * INT4; the pages print no values).  Reading: the FP4 E2M1 layout of the OCP
+ * Microscaling formats -- 1 sign bit, 2 exponent bits with bias 1, 1 mantissa
+ * bit, exponent field 0 holding the subnormals 0 and 0.5 -- divided by its
+ * largest magnitude 6 so that absmax scaling maps the ends to -1 and +1.
+ * Its 16 codes hold 15 distinct values: -0 and +0 are both kept, -0 first,
+ * so the table is non-decreasing with one repeated level.  Rounded to fp32. */
+void orc_fp4_codebook(float out[16]) {
+    double mag[8];
+    for (int code = 0; code < 8; ++code) {     /* exponent field e, mantissa bit m */
+        const int e = code >> 1, m = code & 1;
+        mag[code] = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    }
+    for (int i = 0; i < 8; ++i) {
+        out[7 - i] = (float)(-mag[i] / 6.0);   /* -0, -1/12, ..., -1 */
+        out[8 + i] = (float)(mag[i] / 6.0);    /* +0, +1/12, ..., +1 */
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Blockwise quantization ([CSDN] 5.2) and double quantization ([CSDN] 7.2) */
 /* ------------------------------------------------------------------------ */

@@ -13,6 +13,8 @@ import numpy as np
 import pytest
 from scipy.stats import norm
 
+from conftest import floats, read_golden
+
 
 def test_ppf_textbook_values(orc):
     assert orc.normal_ppf(0.5) == pytest.approx(0.0, abs=1e-15)
@@ -90,3 +92,61 @@ def test_codebook_delta_variant(orc):
     assert cb[0] == -1 and cb[15] == 1 and cb[7] == 0
     assert np.all(np.diff(cb) > 0)
     assert not np.array_equal(cb, orc.nf4_codebook())
+
+
+# ---------------------------------------------------------------- FP4 table
+# bitsandbytes' other 4-bit type is a "4-bit float-style" table (bitsandbytes
+# article (CSDN) 6.4-6.5, 9.3).  Reading: FP4 E2M1 of the OCP Microscaling
+# formats, scaled by 1/6 into [-1, 1]; the magnitudes are the golden list.
+
+def test_fp4_codebook_is_e2m1_over_6(orc):
+    g = read_golden("fp4_e2m1_values.txt")
+    mags = floats(g["magnitudes"])
+    top = float(g["max_magnitude"])
+    cb = orc.fp4_codebook()
+    assert cb.dtype == np.float32 and cb.shape == (16,)
+    want_pos = np.array([m / top for m in mags], dtype=np.float32)
+    assert np.array_equal(cb[8:], want_pos)
+    assert np.array_equal(cb[:8], -want_pos[::-1])
+    assert cb[0] == -1 and cb[15] == 1
+
+
+def test_fp4_codebook_structure(orc):
+    """Non-decreasing; the one repeated level is the zero, -0 (index 7) before
+    +0 (index 8); antisymmetric; each magnitude times 6 has one significant
+    bit after the leading one at most (a 1-bit mantissa)."""
+    cb = orc.fp4_codebook()
+    assert np.all(np.diff(cb.astype(np.float64)) >= 0)
+    eq = np.flatnonzero(np.diff(cb.astype(np.float64)) == 0)
+    assert list(eq) == [7]
+    assert cb[7] == 0 and np.signbit(cb[7]) and cb[8] == 0 and not np.signbit(cb[8])
+    assert np.array_equal(cb[::-1], -cb)
+    for m in np.abs(cb.astype(np.float64)) * 6:
+        m = float(np.float32(m))
+        if m:
+            mant, _ = math.frexp(m)
+            assert (mant * 4) == int(mant * 4)
+
+
+def test_fp4_quantize_first_minimum(orc):
+    """Quantizing with the FP4 table: every weight takes the first nearest
+    level in exact arithmetic; in zero's basin that is -0 (index 7) for
+    weights of either sign, and the +0 code is never produced."""
+    from fractions import Fraction as Fr
+    cb = orc.fp4_codebook()
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((6, 64)) * 0.02).astype(np.float32)
+    W[0, 1:9] = np.array([1e-9, -1e-9, 0.0, -0.0, 1e-3, -1e-3, 2e-4, -2e-4], np.float32)
+    q = orc.quantize(W, cb, False)
+    flat = W.reshape(-1)
+    idx = np.empty(flat.size, np.int64)
+    idx[0::2], idx[1::2] = q.packed >> 4, q.packed & 15
+    for b in range(flat.size // 64):
+        blk = flat[64 * b:64 * b + 64]
+        a = Fr(float(np.max(np.abs(blk))))
+        for i, w in enumerate(blk):
+            d = [abs(Fr(float(w)) - Fr(float(c)) * a) for c in cb]
+            assert idx[64 * b + i] == d.index(min(d))
+    assert not np.any(idx == 8)
+    deq = orc.dequantize(q, cb).reshape(-1)
+    assert deq[2] == 0x8000 and deq[3] == 0x8000          # +-1e-9 -> -0 in bf16
