@@ -60,13 +60,13 @@ def _L():
         lib.orc_fp4_codebook.restype = None
         lib.orc_fp4_codebook.argtypes = [P]
         lib.orc_quantize.restype = ctypes.c_int
-        lib.orc_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
+        lib.orc_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P, P,
                                      P]
         lib.orc_dequantize.restype = None
-        lib.orc_dequantize.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
+        lib.orc_dequantize.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P, P,
                                        P, P]
         lib.orc_dequantize_dt.restype = None
-        lib.orc_dequantize_dt.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P,
+        lib.orc_dequantize_dt.argtypes = [i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P,
                                           P, P, ctypes.c_int, P]
         lib.orc_fp16_bits.restype = None
         lib.orc_fp16_bits.argtypes = [P, i64, P]
@@ -127,6 +127,12 @@ def fp4_codebook() -> np.ndarray:
     return out
 
 
+# Double-quantization codes of the first-level scales: the unsigned 8-bit
+# code (step = max / 255), the signed INT8 absmax code (step = max / 127), and
+# the signed INT8 code of the scales minus their group mean.
+DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3}
+
+
 @dataclass
 class QuantizedWeight:
     rows: int
@@ -134,22 +140,28 @@ class QuantizedWeight:
     double_quant: bool
     packed: np.ndarray            # uint8 [rows*cols/2]
     absmax: np.ndarray | None     # float32 [nb]
-    codes: np.ndarray | None      # uint8 [nb]
+    codes: np.ndarray | None      # uint8 [nb] (int8 two's complement for "mean")
     steps: np.ndarray | None      # float32 [ceil(nb/256)]
     status: int
     block: int = BLOCK            # weights per first-level scale
+    dq_variant: str = "u8"
+    offsets: np.ndarray | None = None   # float32 [ceil(nb/256)] group means ("mean")
+
+    @property
+    def dq_code(self) -> int:
+        return DQ_VARIANTS[self.dq_variant] if self.double_quant else 0
 
     @property
     def nbytes(self) -> int:
         n = self.packed.nbytes
-        for a in (self.absmax, self.codes, self.steps):
+        for a in (self.absmax, self.codes, self.steps, self.offsets):
             if a is not None:
                 n += a.nbytes
         return n
 
 
 def quantize(W: np.ndarray, codebook: np.ndarray, double_quant: bool,
-             dq_group: int = DQ_GROUP, block: int = BLOCK) -> QuantizedWeight:
+             dq_group: int = DQ_GROUP, block: int = BLOCK, dq_variant: str = "u8") -> QuantizedWeight:
     W = _c(W, np.float32)
     rows, cols = W.shape
     assert block % 2 == 0 and cols % block == 0
@@ -160,17 +172,20 @@ def quantize(W: np.ndarray, codebook: np.ndarray, double_quant: bool,
     codes = np.zeros(nb, dtype=np.uint8) if double_quant else None
     ng = (nb + dq_group - 1) // dq_group
     steps = np.zeros(ng, dtype=np.float32) if double_quant else None
-    st = _L().orc_quantize(_p(W), rows, cols, block, _p(cb), int(double_quant), dq_group,
-                           _p(packed), _p(absmax), _p(codes), _p(steps))
-    return QuantizedWeight(rows, cols, double_quant, packed, absmax, codes, steps, int(st), block)
+    offsets = np.zeros(ng, dtype=np.float32) if double_quant and dq_variant == "mean" else None
+    dq = DQ_VARIANTS[dq_variant] if double_quant else 0
+    st = _L().orc_quantize(_p(W), rows, cols, block, _p(cb), dq, dq_group,
+                           _p(packed), _p(absmax), _p(codes), _p(steps), _p(offsets))
+    return QuantizedWeight(rows, cols, double_quant, packed, absmax, codes, steps, int(st), block,
+                           dq_variant, offsets)
 
 
 def dequantize(q: QuantizedWeight, codebook: np.ndarray, dq_group: int = DQ_GROUP) -> np.ndarray:
     """bf16 bit patterns [rows, cols]."""
     cb = _c(codebook, np.float32)
     out = np.zeros((q.rows, q.cols), dtype=np.uint16)
-    _L().orc_dequantize(q.rows, q.cols, q.block, _p(cb), int(q.double_quant), dq_group, _p(q.packed),
-                        _p(q.absmax), _p(q.codes), _p(q.steps), _p(out))
+    _L().orc_dequantize(q.rows, q.cols, q.block, _p(cb), q.dq_code, dq_group, _p(q.packed),
+                        _p(q.absmax), _p(q.codes), _p(q.steps), _p(q.offsets), _p(out))
     return out
 
 
@@ -183,9 +198,9 @@ def dequantize_dt(q: QuantizedWeight, codebook: np.ndarray, dtype: str,
     fp16, float32 values for fp32."""
     cb = _c(codebook, np.float32)
     out = np.zeros((q.rows, q.cols), dtype=np.float32 if dtype == "fp32" else np.uint16)
-    _L().orc_dequantize_dt(q.rows, q.cols, q.block, _p(cb), int(q.double_quant), dq_group,
-                           _p(q.packed), _p(q.absmax), _p(q.codes), _p(q.steps), DTYPES[dtype],
-                           _p(out))
+    _L().orc_dequantize_dt(q.rows, q.cols, q.block, _p(cb), q.dq_code, dq_group,
+                           _p(q.packed), _p(q.absmax), _p(q.codes), _p(q.steps), _p(q.offsets),
+                           DTYPES[dtype], _p(out))
     return out
 
 

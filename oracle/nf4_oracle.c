@@ -33,6 +33,11 @@
 #include <string.h>
 
 #define ORC_STATUS_NONFINITE 1
+/* Double-quantization codes of the first-level scales (the `dq` argument). */
+#define ORC_DQ_NONE 0
+#define ORC_DQ_U8 1     /* unsigned, step = max / 255, codes 0..255 */
+#define ORC_DQ_S8 2     /* signed INT8 absmax code of [CSDN] 4.1: step = max / 127, codes 0..127 */
+#define ORC_DQ_MEAN 3   /* signed INT8 code of a_b minus the group mean; one mean per group */
 
 /* ------------------------------------------------------------------------ */
 /* bf16 <-> fp32 helpers (storage format of the inputs and of dequant out)  */
@@ -217,6 +222,45 @@ static int nearest_level(float w, float a, const float cb[16], int zero_idx) {
     return best;
 }
 
+/* Double quantization with the group mean taken out first (a variant of
+ * [CSDN] 7.2's structure, whose 8-bit code the pages do not give; reading:
+ * centre the scales on their mean, then a symmetric INT8 code as in [CSDN]
+ * 4.1).  Every step is one stated rounding:
+ *   mu   = RN32(S / n), S the fp64 sum of the group's a_b in block order
+ *   d_b  = RN32(a_b - mu)
+ *   f    = RN32(max_b |d_b| / 127)
+ *   code = clamp(round-half-even(d_b / f), -127, 127), stored as int8
+ * decoded as a_hat = RN32(mu + RN32(code * f)); f = 0 gives codes of 0.
+ * d_b / f is a ratio of two fp32 values of magnitude <= 127.5 (before the
+ * clamp): unless it is a half-integer it lies at least 2^-32 (relative) away
+ * from one, far above fp64 rounding, so rint of the fp64 quotient is the
+ * exact rule.  In the decode, fp32 + fp32 done in fp64 and rounded to fp32 is
+ * the correctly rounded fp32 sum (53 >= 2*24 + 2). */
+static void dq_group_mean(const float *a, int64_t n, uint8_t *codes, float *step, float *offset) {
+    double sum = 0.0;
+    for (int64_t i = 0; i < n; ++i) sum += (double)a[i];
+    const float mu = (float)(sum / (double)n);
+    float mx = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        const float d = a[i] - mu;
+        if (fabsf(d) > mx) mx = fabsf(d);
+    }
+    const float f = (float)((double)mx / 127.0);
+    *step = f;
+    *offset = mu;
+    for (int64_t i = 0; i < n; ++i) {
+        int code = 0;
+        if (f > 0.0f) {
+            const float d = a[i] - mu;
+            double qd = rint((double)d / (double)f);
+            if (qd < -127.0) qd = -127.0;
+            if (qd > 127.0) qd = 127.0;
+            code = (int)qd;
+        }
+        codes[i] = (uint8_t)(int8_t)code;
+    }
+}
+
 /* Quantize Wt:[rows, cols] (fp32, row-major) in blocks of `block` weights
  * (64 by default; 32, 128 or 256 trade scale resolution against metadata,
  * [CSDN] 5.1).  The row-major flattening is cut into consecutive blocks; cols
@@ -239,7 +283,7 @@ static int nearest_level(float w, float a, const float cb[16], int zero_idx) {
  * the weights). */
 int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const float cb[16],
                  int dq, int dq_group, uint8_t *packed, float *absmax,
-                 uint8_t *codes, float *steps) {
+                 uint8_t *codes, float *steps, float *offsets) {
     const int64_t n = rows * cols;
     const int64_t nb = n / block;
     const int zero_idx = zero_level_index(cb);
@@ -268,12 +312,20 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const fl
         for (int64_t g = 0; g < ng; ++g) {
             int64_t b0 = g * dq_group;
             int64_t b1 = b0 + dq_group < nb ? b0 + dq_group : nb;
+            if (dq == ORC_DQ_MEAN) {
+                dq_group_mean(a_all + b0, b1 - b0, codes + b0, steps + g, offsets + g);
+                continue;
+            }
+            /* the top code: 255 for the unsigned code, 127 for the signed
+             * INT8 code of [CSDN] 4.1 (absmax values are >= 0, so only its
+             * codes 0..127 occur) */
+            const double top = dq == ORC_DQ_S8 ? 127.0 : 255.0;
             float mx = 0.0f;
             for (int64_t b = b0; b < b1; ++b)
                 if (a_all[b] > mx) mx = a_all[b];
-            /* RN32(mx/255): fp64 division then one rounding to fp32 is the
+            /* RN32(mx/top): fp64 division then one rounding to fp32 is the
              * correctly rounded fp32 quotient (53 >= 2*24+2). */
-            float f = (float)((double)mx / 255.0);
+            float f = (float)((double)mx / top);
             steps[g] = f;
             for (int64_t b = b0; b < b1; ++b) {
                 int code = 0;
@@ -284,7 +336,7 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const fl
                      * fp64 quotient is round-half-even of the exact ratio. */
                     double qd = rint((double)a_all[b] / (double)f);
                     if (qd < 0.0) qd = 0.0;
-                    if (qd > 255.0) qd = 255.0;
+                    if (qd > top) qd = top;
                     code = (int)qd;
                 }
                 codes[b] = (uint8_t)code;
@@ -297,11 +349,17 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const fl
 
 /* Decoded first-level scale of block b: a_b itself, or with double
  * quantization RN32(code_b * f_g) -- the product is exact in fp64 and is
- * rounded once to fp32. */
+ * rounded once to fp32 -- or, for the mean-offset variant with a signed
+ * code, RN32(mu_g + RN32(code_b * f_g)). */
 static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
-                         const uint8_t *codes, const float *steps) {
+                         const uint8_t *codes, const float *steps, const float *offsets) {
     if (!dq) return absmax[b];
-    return (float)((double)codes[b] * (double)steps[b / dq_group]);
+    const int64_t g = b / dq_group;
+    if (dq == ORC_DQ_MEAN) {
+        const float d = (float)((double)(int8_t)codes[b] * (double)steps[g]);
+        return (float)((double)offsets[g] + (double)d);
+    }
+    return (float)((double)codes[b] * (double)steps[g]);
 }
 
 /* Dequantize ([CSDN] 5.2 w_hat = a * c_q; 8.6 the result is in the compute
@@ -309,14 +367,14 @@ static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
  * the scale of block e / block.  Output is bf16 bit patterns, [rows, cols]. */
 void orc_dequantize(int64_t rows, int64_t cols, int block, const float cb[16], int dq,
                     int dq_group, const uint8_t *packed, const float *absmax,
-                    const uint8_t *codes, const float *steps, uint16_t *out) {
+                    const uint8_t *codes, const float *steps, const float *offsets, uint16_t *out) {
     const int64_t n = rows * cols;
 #pragma omp parallel for schedule(static)
     for (int64_t e = 0; e < n; ++e) {
         int64_t b = e / block;
         uint8_t byte = packed[e / 2];
         int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
-        float ah = block_scale(b, dq, dq_group, absmax, codes, steps);
+        float ah = block_scale(b, dq, dq_group, absmax, codes, steps, offsets);
         float w = (float)((double)ah * (double)cb[q]);
         out[e] = float_to_bf16_rne(w);
     }
@@ -355,13 +413,14 @@ static uint16_t float_to_fp16_rne(float f) {
  * in out), 2 = fp32 (out holds fp32 values). */
 void orc_dequantize_dt(int64_t rows, int64_t cols, int block, const float cb[16], int dq,
                        int dq_group, const uint8_t *packed, const float *absmax,
-                       const uint8_t *codes, const float *steps, int dtype, void *out) {
+                       const uint8_t *codes, const float *steps, const float *offsets, int dtype,
+                       void *out) {
     const int64_t n = rows * cols;
 #pragma omp parallel for schedule(static)
     for (int64_t e = 0; e < n; ++e) {
         uint8_t byte = packed[e / 2];
         int q = (e % 2 == 0) ? (byte >> 4) : (byte & 0x0f);
-        float ah = block_scale(e / block, dq, dq_group, absmax, codes, steps);
+        float ah = block_scale(e / block, dq, dq_group, absmax, codes, steps, offsets);
         float w = (float)((double)ah * (double)cb[q]);
         if (dtype == 2)
             ((float *)out)[e] = w;

@@ -451,3 +451,95 @@ def test_dequantize_compute_dtypes(orc, block):
         assert np.array_equal(orc.dequantize_dt(q, cb, "fp16").reshape(-1), f16)
         assert np.array_equal(orc.dequantize_dt(q, cb, "bf16"), orc.dequantize(q, cb))
         assert np.array_equal(orc.dequantize(q, cb).reshape(-1), bf16_of_f32(f32.reshape(-1)))
+
+
+# ---------------------------------------------------------------- double-quant variants
+# The pages give double quantization's structure (8-bit first-level scales,
+# one fp32 constant per 256; CSDN 7.2) but no 8-bit code.  Besides the
+# unsigned code above, two variants: the signed INT8 absmax code of CSDN 4.1
+# (s = 127 / max|x|) applied to the scales, and a code of the scales minus
+# their group mean.
+
+def _rn32(fr):
+    return rn32(fr)
+
+
+def test_dq_signed_int8_bruteforce(orc):
+    """Step RN32(max / 127); code = round-half-even(a / step) over 0..127,
+    brute force in exact arithmetic; decode RN32(code * step)."""
+    rng = np.random.default_rng(21)
+    cb = orc.nf4_codebook()
+    am = np.abs(rng.standard_normal(256 + 61) * 0.05).astype(np.float32)
+    am[3] = 0.0
+    q = orc.quantize(_dq_blocks(am), cb, double_quant=True, dq_variant="s8")
+    for g0 in (0, 256):
+        grp = am[g0:g0 + 256]
+        f = _rn32(Fr(float(np.max(grp))) / 127)
+        assert q.steps[g0 // 256] == f
+        ff = Fr(float(f))
+        for i, a in enumerate(grp):
+            want = min(range(128), key=lambda c: (abs(c * ff - Fr(float(a))), c & 1))
+            assert q.codes[g0 + i] == want
+        assert q.codes[g0 + int(np.argmax(grp))] == 127
+    # the weights are encoded with the true absmax, whatever the scale code
+    assert np.array_equal(q.packed, orc.quantize(_dq_blocks(am), cb, double_quant=False).packed)
+    # decode: RN32(code * step), as the unsigned code
+    deq = orc.dequantize(q, cb).reshape(-1)
+    idx = unpack(q.packed, deq.size)
+    for e in range(0, deq.size, 13):
+        b = e // BLOCK
+        ah = _rn32(Fr(int(q.codes[b])) * Fr(float(q.steps[b // 256])))
+        assert deq[e] == bf16_of_f32(_rn32(Fr(float(ah)) * Fr(float(cb[idx[e]]))))
+
+
+def test_dq_mean_offset_bruteforce(orc):
+    """mu = RN32(fp64 sum / n); d = RN32(a - mu) (numpy's fp32 subtraction);
+    step RN32(max|d| / 127); code = round-half-even(d / step) over -127..127 by
+    brute force in exact arithmetic; decode RN32(mu + RN32(code * step))."""
+    rng = np.random.default_rng(22)
+    cb = orc.nf4_codebook()
+    am = np.abs(rng.standard_normal(256 + 40) * 0.05).astype(np.float32)
+    am[7] = 0.0
+    am[200] = np.float32(0.4)                      # one large scale pulls the mean
+    q = orc.quantize(_dq_blocks(am), cb, double_quant=True, dq_variant="mean")
+    assert q.offsets is not None and q.offsets.size == 2
+    for g0 in (0, 256):
+        grp = am[g0:g0 + 256]
+        # the values are fp32 in [2^-30, 1): their fp64 sum is exact, so mu is
+        # the exact mean rounded once
+        mu = _rn32(sum(Fr(float(a)) for a in grp) / len(grp))
+        assert q.offsets[g0 // 256] == mu
+        d = (grp - np.float32(mu)).astype(np.float32)          # IEEE fp32 subtraction
+        f = _rn32(Fr(float(np.max(np.abs(d)))) / 127)
+        assert q.steps[g0 // 256] == f
+        ff = Fr(float(f))
+        codes = q.codes[g0:g0 + len(grp)].view(np.int8)
+        for i, di in enumerate(d):
+            want = min(range(-127, 128), key=lambda c: (abs(c * ff - Fr(float(di))), c & 1))
+            assert codes[i] == want, (g0, i)
+        # every decoded scale is within half a step of its d (plus one rounding)
+        dec = [_rn32(Fr(float(mu)) + Fr(float(_rn32(int(c) * ff)))) for c in codes]
+        for a, ah in zip(grp, dec):
+            assert abs(Fr(float(ah)) - Fr(float(a))) <= ff / 2 + Fr(float(np.spacing(np.float32(a)))) * 2
+    deq = orc.dequantize(q, cb).reshape(-1)
+    idx = unpack(q.packed, deq.size)
+    for e in range(0, deq.size, 11):
+        b = e // BLOCK
+        g = b // 256
+        d = _rn32(int(q.codes.view(np.int8)[b]) * Fr(float(q.steps[g])))
+        ah = _rn32(Fr(float(q.offsets[g])) + Fr(float(d)))
+        assert deq[e] == bf16_of_f32(_rn32(Fr(float(ah)) * Fr(float(cb[idx[e]]))))
+
+
+def test_dq_variants_bits_per_parameter(orc):
+    """The signed code costs what the unsigned one does (8/64 + 32/(64*256)
+    bits per parameter); the mean-offset code stores one more fp32 per group:
+    8/64 + 64/(64*256)."""
+    rng = np.random.default_rng(23)
+    cb = orc.nf4_codebook()
+    W = (rng.standard_normal((256, 4096)) * 0.02).astype(np.float32)
+    n = W.size
+    q_s8 = orc.quantize(W, cb, double_quant=True, dq_variant="s8")
+    q_mean = orc.quantize(W, cb, double_quant=True, dq_variant="mean")
+    assert 8 * q_s8.nbytes / n - 4 == 8 / 64 + 32 / (64 * 256)
+    assert 8 * q_mean.nbytes / n - 4 == 8 / 64 + 64 / (64 * 256)
