@@ -171,64 +171,91 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- reference arm
+def oracle_step_estimate(a, spec, M, rows, quant_rows):
+    """The oracle on a bounded sample of one step: nf4_quantize (+ dequantize)
+    of the first `quant_rows` weight rows, and forward + backward (dX, dA, dB)
+    of `rows` token rows.  The full step's time is extrapolated from the two
+    parts (quantize scales with the weight rows, the layer with the tokens)."""
+    import oracle
+    cb = oracle.nf4_codebook()
+    t0 = time.perf_counter()
+    oracle.dequantize(oracle.quantize(a["W"][:quant_rows], cb, True), cb)
+    tq = time.perf_counter() - t0
+    Wt = oracle.dequantize(oracle.quantize(a["W"], cb, True), cb)
+    sel = (np.arange(rows) * 131) % M
+    t0 = time.perf_counter()
+    oracle.forward(a["x"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
+    oracle.backward(a["x"][sel], a["dY"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
+    tl = time.perf_counter() - t0
+    step_s = tq * (spec.Dout / quant_rows) + tl * (M / rows)
+    return {"value": layer_flops(M, spec.Din, spec.Dout, spec.r) / step_s / 1e12, "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"quantize of {quant_rows} of {spec.Dout} weight rows ({tq:.2f} s) and "
+                       f"fwd+bwd of {rows} of {M} token rows ({tl:.2f} s), extrapolated to the "
+                       f"full step ({step_s:.1f} s)"),
+            "step_s_extrapolated": step_s}
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
-    import oracle
     spec = synth.CONFIGS[CFG]["linears"][0]
     M = synth.CONFIGS[CFG]["M"][0]
     a = synth.draw(spec, M, CFG)
-    cb = oracle.nf4_codebook()
     S = args.ref_rows
-    flops = layer_flops(S, spec.Din, spec.Dout, spec.r)
-
-    def step(i):
-        rows = (np.arange(S) * 131 + i * 17) % M
-        qw = oracle.quantize(a["W"], cb, True)
-        Wt = oracle.dequantize(qw, cb)
-        oracle.forward(a["x"][rows], Wt, a["A"], a["B"], spec.r, spec.alpha)
-        oracle.backward(a["x"][rows], a["dY"][rows], Wt, a["A"], a["B"], spec.r, spec.alpha)
-
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(args.warmup + i)
-    dt = (time.perf_counter() - t0) / args.steps
-    v = flops / dt / 1e12
-    sample = (f"{S} of {M} token rows per step (forward, dX, dA, dB on those rows) "
-              f"+ full-weight quantize/dequantize")
+    for _ in range(args.warmup):
+        oracle_step_estimate(a, spec, M, S, spec.Dout)
+    est = []
+    for _ in range(args.steps):
+        est.append(oracle_step_estimate(a, spec, M, S, spec.Dout))
+    dt = statistics.mean(e["step_s_extrapolated"] for e in est)
+    v = layer_flops(M, spec.Din, spec.Dout, spec.r) / dt / 1e12
+    cpu = dict(est[-1])
+    cpu["value"] = v
+    cpu.pop("step_s_extrapolated", None)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded numpy PCG64)",
-        "config": {"workload": WORKLOAD, "sample": sample},
-        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": sample},
+        "config": {"workload": WORKLOAD, "sample": cpu["sample"]},
+        "cpu_baseline": cpu,
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
 # --------------------------------------------------------------------------- our arm
-def cpu_baseline(rows=1024):
-    """The oracle as it stands on a bounded sample of the workload."""
-    import oracle
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_baseline(rows=1024, rows_1core=64):
+    """The oracle as it stands, on the host's cores (all of them) and on one
+    core (a child process with OMP_NUM_THREADS=1), each on a bounded sample of
+    the step extrapolated to the full step."""
     spec = synth.CONFIGS[CFG]["linears"][0]
     M = synth.CONFIGS[CFG]["M"][0]
     a = synth.draw(spec, M, CFG)
-    cb = oracle.nf4_codebook()
-    sel = np.arange(rows)
-    t0 = time.perf_counter()
-    qw = oracle.quantize(a["W"], cb, True)
-    Wt = oracle.dequantize(qw, cb)
-    oracle.forward(a["x"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
-    oracle.backward(a["x"][sel], a["dY"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha)
-    dt = time.perf_counter() - t0
-    return {"value": layer_flops(rows, spec.Din, spec.Dout, spec.r) / dt / 1e12, "unit": "TFLOP/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows} of {M} token rows (forward, dX, dA, dB) + full-weight quantize; "
-                      f"{dt:.1f} s"}
+    out = oracle_step_estimate(a, spec, M, rows, spec.Dout)
+    out.pop("step_s_extrapolated", None)
+    out["cpu_model"] = cpu_model()
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-sample",
+                            str(rows_1core), str(spec.Dout // 4)], env=env, capture_output=True,
+                           text=True, timeout=600)
+        one = json.loads(r.stdout.strip().splitlines()[-1])
+        one.pop("step_s_extrapolated", None)
+        out["single_core"] = one
+    except Exception as e:   # reported, not fatal: the GPU numbers stand alone
+        out["single_core"] = {"error": str(e)[:200]}
+    return out
 
 
 def run_ours(args, rank, world, dist):
@@ -371,10 +398,14 @@ def run_ours(args, rank, world, dist):
     e2e = {"value": world * e2e_steps * flops_step / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
-    # ---------------- decode-shaped GEMV lines (M = 1, 16; forward only)
-    extras = {}
+    # ---------------- the same step captured once in a CUDA graph, replayed
+    graph = graph_median(torch, step, flush, args.graph_replays, flops_step) if world == 1 else None
+
+    # ---------------- decode-shaped GEMV lines (M = 1, 16) and the other workloads
+    extras, workloads = {}, {}
     if not args.no_extras:
         extras = decode_lines(args, q, lib, torch, dev, hbm, flush)
+        workloads = workload_lines(q, lib, torch, dev, flush, tf_burst)
 
     if rank != 0:
         return
@@ -392,11 +423,132 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": int(launches),
         "clocks": csum,
         "step_ms": {"median": statistics.median(step_ms), "min": min(step_ms), "max": max(step_ms)},
+        "graph": graph,
         "decode": extras,
+        "workloads": workloads,
     }
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.cpu_rows)
     print(json.dumps(out), flush=True)
+
+
+def graph_median(torch, step, flush, replays, flops_step):
+    """One step (quantize + forward + backward) captured in a CUDA graph and
+    replayed: 10 warm-up replays, then `replays` timed ones with L2 flushed
+    before each (outside the events); the median replay time."""
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(10):
+        g.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    del g
+    return {"replays": replays, "median_ms": ms, "tflops": flops_step / (ms / 1e3) / 1e12,
+            "l2": "flushed before each replay, outside the events"}
+
+
+def layer_timing(q, lib, torch, dev, flush, tf_peak, spec, cfg, lin, M, reps=3):
+    """nf4_quantize, qlora_forward and qlora_backward of one linear at M
+    tokens: median time of each (L2 flushed before each call, outside the
+    events), and the tcgen05 GEMM's time (library events) with its fraction of
+    the bf16 peak when the tensor-core path runs."""
+    import ctypes
+    a = synth.draw(spec, M, cfg, lin)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    W = torch.from_numpy(a["W"]).to(dev)
+    x, A, B, dy = bf(a["x"]), bf(a["A"]), bf(a["B"]), bf(a["dY"])
+    del a
+    g = spec.pool_group
+    w = q.NF4Weight.empty(spec.Dout, spec.Din, spec.double_quant, dev)
+    ws_f = torch.empty(max(1, q.workspace_size(M, w, spec.r, g, 0)), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(1, q.workspace_size(M, w, spec.r, g, 1)), dtype=torch.uint8, device=dev)
+    y = torch.empty(M, spec.Dout, dtype=torch.bfloat16, device=dev)
+    saved = {}
+
+    def fwd():
+        saved["T"] = q.forward(x, w, A, B, spec.alpha, g, out=y, workspace=ws_f)[1]
+
+    calls = (("quantize", lambda: q.quantize(W, double_quant=spec.double_quant, out=w)),
+             ("forward", fwd),
+             ("backward", lambda: q.backward(x, dy, w, A, B, spec.alpha, g, T=saved["T"], workspace=ws_b)))
+    for _ in range(2):
+        for _, fn in calls:
+            fn()
+    torch.cuda.synchronize()
+    ev = {n: [] for n, _ in calls}
+    lib.qlora_profile_reset()
+    lib.qlora_profile_enable(1)
+    for _ in range(reps):
+        for n, fn in calls:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+            ev[n].append((e0, e1))
+    torch.cuda.synchronize()
+    lib.qlora_profile_enable(0)
+    un, ums = ctypes.c_int64(), ctypes.c_double()
+    lib.qlora_profile_read(0, ctypes.byref(un), ctypes.byref(ums))
+    ms = {n: statistics.median(e0.elapsed_time(e1) for e0, e1 in ev[n]) for n in ev}
+    fwd_f = 2 * M * spec.Din * spec.Dout + 2 * M * spec.r * (spec.Din + spec.Dout)
+    bwd_f = 2 * M * spec.Din * spec.Dout + 4 * M * spec.r * (spec.Din + spec.Dout)
+    out = {"shape": f"{spec.Din}->{spec.Dout}", "M": M, "r": spec.r, "pool_group": g,
+           "quantize_ms": ms["quantize"], "forward_ms": ms["forward"], "backward_ms": ms["backward"],
+           "step_ms": sum(ms.values()),
+           "fwd_bwd_tflops": (fwd_f + bwd_f) / ((ms["forward"] + ms["backward"]) / 1e3) / 1e12}
+    if un.value:
+        per = ums.value / un.value
+        gemm_f = 2 * M * spec.Din * spec.Dout
+        # forward and dX launches alternate; each carries its adapter extension
+        ext = M * spec.r * (spec.Din // g + spec.Dout)
+        tf = (2 * gemm_f + 2 * ext) / 2 / (per / 1e3) / 1e12
+        out["gemm"] = {"kernel": "k_umma_qgemm", "launches": un.value, "ms_per_launch": per,
+                       "tflops": tf, "frac_of_burst_peak": tf / tf_peak}
+    del W, x, A, B, dy, w, ws_f, ws_b, y, saved
+    torch.cuda.empty_cache()
+    return out
+
+
+def workload_lines(q, lib, torch, dev, flush, tf_peak):
+    """The workloads beside the headline: config 1 (one 256 x 256 linear,
+    M = 16), config 4 (a 7B decoder layer's seven linears at M = 2048) and
+    config 5 at M = 8192 (the 70B MLP up and down projections, and the up
+    projection with the pooled adapter)."""
+    res = {}
+    c1 = synth.CONFIGS[1]
+    res["config1"] = layer_timing(q, lib, torch, dev, flush, tf_peak, c1["linears"][0], 1, 0, c1["M"][0])
+    c4 = synth.CONFIGS[4]
+    lins = {}
+    for i, spec in enumerate(c4["linears"]):
+        lins[spec.name] = layer_timing(q, lib, torch, dev, flush, tf_peak, spec, 4, i, c4["M"][0])
+    tot = sum(v["step_ms"] for v in lins.values())
+    fl = sum(layer_flops(c4["M"][0], s.Din, s.Dout, s.r) for s in c4["linears"])
+    res["config4"] = {"linears": lins, "layer_step_ms": tot, "layer_tflops": fl / (tot / 1e3) / 1e12,
+                      "note": "quantize of all seven weights + forward + backward of each, M = 2048"}
+    c5 = synth.CONFIGS[5]
+    for i, spec in enumerate(c5["linears"]):
+        res[f"config5_{spec.name}_M8192"] = layer_timing(q, lib, torch, dev, flush, tf_peak, spec, 5, i, 8192,
+                                                         reps=2)
+    return res
 
 
 def decode_lines(args, q, lib, torch, dev, hbm, flush):
@@ -564,7 +716,7 @@ def backward_line(q, lib, torch, dev, hbm, flush, spec, cfg, lin, w, A, B, x, M)
     kern_ms = ms.value / max(1, n.value)
     alg = (weight_bytes(spec.Din, spec.Dout) + 2 * M * spec.Dout + 2 * M * spec.Din
            + 2 * spec.r * spec.Din + 4 * M * spec.r)
-    return {"backward_ms": step, "kernel": "k_gemv_bwd", "kernel_ms": kern_ms,
+    return {"backward_ms": step, "kernel": "k_gemv_bwd_stream", "kernel_ms": kern_ms,
             "kernel_GBps": alg / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else None,
             "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None}
 
@@ -606,6 +758,29 @@ def merge_line(q, lib, torch, dev, hbm, flush):
             "kernel_frac_hbm": (alg / (kern_ms / 1e3) / 1e9) / hbm if kern_ms > 0 else None}
 
 
+def profile_case(cfg, lin, M):
+    """One nf4_quantize, one qlora_forward and one qlora_backward of a
+    workload linear, in that order, then exit: kernel launches in a fixed
+    order for profiler captures (the first forward and backward launches of
+    each kernel are the ones of this case)."""
+    import torch
+    import bit_nf4_quantized_22_b200 as q
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    spec = synth.CONFIGS[cfg]["linears"][lin]
+    a = synth.draw(spec, M, cfg, lin)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    w = q.quantize(torch.from_numpy(a["W"]).to(dev), double_quant=spec.double_quant)
+    x, A, B, dy = bf(a["x"]), bf(a["A"]), bf(a["B"]), bf(a["dY"])
+    _, T = q.forward(x, w, A, B, spec.alpha, spec.pool_group)
+    q.backward(x, dy, w, A, B, spec.alpha, spec.pool_group, T=T)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": f"{cfg}:{lin}:{M}", "shape": f"{spec.Din}->{spec.Dout}"}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -616,10 +791,24 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--graph-replays", type=int, default=50)
+    ap.add_argument("--profile-case", metavar="CFG:LIN:M",
+                    help="run one quantize + forward + backward of config CFG, linear LIN at M "
+                         "tokens and exit (a small, fixed launch sequence for ncu captures)")
+    ap.add_argument("--oracle-sample", nargs=2, type=int, metavar=("ROWS", "QUANT_ROWS"),
+                    help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.oracle_sample:
+        spec = synth.CONFIGS[CFG]["linears"][0]
+        M = synth.CONFIGS[CFG]["M"][0]
+        print(json.dumps(oracle_step_estimate(synth.draw(spec, M, CFG), spec, M, *args.oracle_sample)))
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.profile_case:
+        profile_case(*[int(v) for v in args.profile_case.split(":")])
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

@@ -21,7 +21,7 @@ EXPORTS = (
     "nf4_dequantize", "qlora_workspace_size", "qlora_forward", "qlora_backward",
     "qlora_launch_count", "qlora_profile_enable", "qlora_profile_reset", "qlora_profile_read",
     "qlora_forward_noalloc", "qlora_merge", "qlora_selftest_wait_timeout", "nf4_dequantize_dtype",
-    "nf4_codebook",
+    "nf4_codebook", "fp4_codebook",
 )
 
 
@@ -33,11 +33,12 @@ class NF4WeightC(ctypes.Structure):
         ("block", ctypes.c_int32),
         ("double_quant", ctypes.c_int32),
         ("dq_group", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("compute_dtype", ctypes.c_int32),
         ("packed", ctypes.c_void_p),
         ("absmax", ctypes.c_void_p),
         ("absmax_code", ctypes.c_void_p),
         ("dq_step", ctypes.c_void_p),
+        ("dq_mean", ctypes.c_void_p),
     ]
 
 
@@ -98,6 +99,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_merge.argtypes = [W, P, P, P, i32, ctypes.c_float, i32, P, P]
     lib.nf4_codebook.restype = ctypes.c_int
     lib.nf4_codebook.argtypes = [ctypes.c_double, P]
+    lib.fp4_codebook.restype = ctypes.c_int
+    lib.fp4_codebook.argtypes = [P]
     _lib = lib
     return lib
 

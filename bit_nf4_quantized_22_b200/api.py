@@ -17,6 +17,8 @@ from .codebook import nf4_codebook
 
 BLOCK = 64
 DQ_GROUP = 256
+# double-quantization codes of the block scales (QLORA_DQ_* in qlora.h)
+DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3}
 
 
 def _ptr(t: torch.Tensor | None):
@@ -50,34 +52,46 @@ class NF4Weight:
     double_quant: bool
     packed: torch.Tensor                   # uint8 [rows*cols/2]
     absmax: torch.Tensor | None = None     # fp32 [nb]
-    codes: torch.Tensor | None = None      # uint8 [nb]
+    codes: torch.Tensor | None = None      # uint8 [nb] (int8 two's complement for "mean")
     steps: torch.Tensor | None = None      # fp32 [ceil(nb/256)]
     block: int = BLOCK                     # weights per first-level scale (32, 64, 128, 256)
+    dq_variant: str = "u8"                 # code of the scales: "u8", "s8" or "mean"
+    means: torch.Tensor | None = None      # fp32 [ceil(nb/256)] group means ("mean")
+    # the layer calls' 16-bit dtype (x, A, B, dY, y, dX, merged weight)
+    compute_dtype: torch.dtype = torch.bfloat16
 
     @staticmethod
-    def empty(rows: int, cols: int, double_quant: bool, device="cuda", block: int = BLOCK) -> "NF4Weight":
+    def empty(rows: int, cols: int, double_quant: bool, device="cuda", block: int = BLOCK,
+              dq_variant: str = "u8") -> "NF4Weight":
         nb = rows * cols // block
         packed = torch.empty(rows * cols // 2, dtype=torch.uint8, device=device)
         if double_quant:
+            if dq_variant not in DQ_VARIANTS:
+                raise ValueError(f"dq_variant: one of {sorted(DQ_VARIANTS)}")
             ng = (nb + DQ_GROUP - 1) // DQ_GROUP
+            means = torch.empty(ng, dtype=torch.float32, device=device) if dq_variant == "mean" else None
             return NF4Weight(rows, cols, True, packed,
                              codes=torch.empty(nb, dtype=torch.uint8, device=device),
-                             steps=torch.empty(ng, dtype=torch.float32, device=device), block=block)
+                             steps=torch.empty(ng, dtype=torch.float32, device=device), block=block,
+                             dq_variant=dq_variant, means=means)
         return NF4Weight(rows, cols, False, packed,
                          absmax=torch.empty(nb, dtype=torch.float32, device=device), block=block)
 
     def c_struct(self) -> _lib.NF4WeightC:
         return _lib.NF4WeightC(
-            self.rows, self.cols, self.block, int(self.double_quant), DQ_GROUP, 0,
+            self.rows, self.cols, self.block,
+            DQ_VARIANTS[self.dq_variant] if self.double_quant else 0, DQ_GROUP,
+            _DTYPE_CODES[self.compute_dtype],
             self.packed.data_ptr(),
             self.absmax.data_ptr() if self.absmax is not None else None,
             self.codes.data_ptr() if self.codes is not None else None,
-            self.steps.data_ptr() if self.steps is not None else None)
+            self.steps.data_ptr() if self.steps is not None else None,
+            self.means.data_ptr() if self.means is not None else None)
 
     @property
     def nbytes(self) -> int:
         n = self.packed.numel()
-        for t in (self.absmax, self.codes, self.steps):
+        for t in (self.absmax, self.codes, self.steps, self.means):
             if t is not None:
                 n += t.numel() * t.element_size()
         return n
@@ -94,12 +108,20 @@ def check_codebook(codebook: torch.Tensor) -> int:
 
 def quantize(W: torch.Tensor, double_quant: bool = True, codebook: torch.Tensor | None = None,
              status: torch.Tensor | None = None, out: NF4Weight | None = None,
-             block: int = BLOCK) -> NF4Weight:
+             block: int = BLOCK, dq_variant: str = "u8",
+             compute_dtype: torch.dtype = torch.bfloat16) -> NF4Weight:
     """nf4_quantize on W (fp32 [Dout, Din], CUDA) in blocks of `block` weights
-    (32, 64, 128 or 256; the layer calls need 64)."""
+    (32, 64, 128 or 256; the layer calls need 64); with double quantization
+    the block scales take the `dq_variant` code ("u8", "s8" or "mean").
+    `compute_dtype` (bf16 or fp16) is the dtype the layer calls then use."""
     _need(W, torch.float32, "W", 2)
+    if compute_dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("compute_dtype: torch.bfloat16 or torch.float16")
     rows, cols = W.shape
-    q = out if out is not None else NF4Weight.empty(rows, cols, double_quant, W.device, block)
+    q = out if out is not None else NF4Weight.empty(rows, cols, double_quant, W.device, block,
+                                                    dq_variant)
+    if out is None:
+        q.compute_dtype = compute_dtype
     qc = q.c_struct()
     rc = load().nf4_quantize(_ptr(W), ctypes.byref(qc), _cb_host(codebook), _ptr(status), _stream())
     _lib.check(rc, "nf4_quantize")
@@ -132,7 +154,7 @@ def merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, pool_gro
           codebook: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
     """bf16 [Dout, Din] weight with the adapter folded in (qlora_merge)."""
     r = B.shape[0]
-    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=torch.bfloat16,
+    out = out if out is not None else torch.empty(q.rows, q.cols, dtype=q.compute_dtype,
                                                   device=q.packed.device)
     qc = q.c_struct()
     rc = load().qlora_merge(ctypes.byref(qc), _cb_host(codebook), _ptr(A), _ptr(B), r,
@@ -159,12 +181,12 @@ def forward(x: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alp
             workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
             out: torch.Tensor | None = None):
     """y = x dequant(W4) + (alpha/r) (u A) B.  Returns (y bf16 [M, Dout], T fp32 [M, r] or None)."""
-    _need(x, torch.bfloat16, "x", 2)
-    _need(A, torch.bfloat16, "A", 2)
-    _need(B, torch.bfloat16, "B", 2)
+    _need(x, q.compute_dtype, "x", 2)
+    _need(A, q.compute_dtype, "A", 2)
+    _need(B, q.compute_dtype, "B", 2)
     M = x.shape[0]
     r = A.shape[1]
-    y = out if out is not None else torch.empty(M, q.rows, dtype=torch.bfloat16, device=x.device)
+    y = out if out is not None else torch.empty(M, q.rows, dtype=q.compute_dtype, device=x.device)
     T = torch.empty(M, r, dtype=torch.float32, device=x.device) if save_T else None
     ws, nbytes = _workspace(workspace_size(M, q, r, pool_group, 0), x.device, workspace)
     qc = q.c_struct()
@@ -181,13 +203,13 @@ def backward(x: torch.Tensor | None, dy: torch.Tensor, q: NF4Weight, A: torch.Te
              codebook: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
              status: torch.Tensor | None = None):
     """Returns (dX bf16 [M, Din] | None, dA fp32 | None, dB fp32 | None); W4 gets none."""
-    _need(dy, torch.bfloat16, "dy", 2)
-    _need(A, torch.bfloat16, "A", 2)
-    _need(B, torch.bfloat16, "B", 2)
+    _need(dy, q.compute_dtype, "dy", 2)
+    _need(A, q.compute_dtype, "A", 2)
+    _need(B, q.compute_dtype, "B", 2)
     M = dy.shape[0]
     r = A.shape[1]
     dev = dy.device
-    dX = torch.empty(M, q.cols, dtype=torch.bfloat16, device=dev) if need_dx else None
+    dX = torch.empty(M, q.cols, dtype=q.compute_dtype, device=dev) if need_dx else None
     dA = torch.empty(A.shape[0], r, dtype=torch.float32, device=dev) if need_dA else None
     dB = torch.empty(r, q.rows, dtype=torch.float32, device=dev) if need_dB else None
     ws, nbytes = _workspace(workspace_size(M, q, r, pool_group, 1), dev, workspace)
@@ -206,11 +228,11 @@ def forward_noalloc(x: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Ten
     """qlora_forward_noalloc: the forward with the library's built-in scratch
     array instead of a workspace.  The caller passes the outputs (`out`,
     `T_out`); when omitted they are created here, which allocates."""
-    _need(x, torch.bfloat16, "x", 2)
-    _need(A, torch.bfloat16, "A", 2)
-    _need(B, torch.bfloat16, "B", 2)
+    _need(x, q.compute_dtype, "x", 2)
+    _need(A, q.compute_dtype, "A", 2)
+    _need(B, q.compute_dtype, "B", 2)
     M, r = x.shape[0], A.shape[1]
-    y = out if out is not None else torch.empty(M, q.rows, dtype=torch.bfloat16, device=x.device)
+    y = out if out is not None else torch.empty(M, q.rows, dtype=q.compute_dtype, device=x.device)
     qc = q.c_struct()
     rc = load().qlora_forward_noalloc(_ptr(x), M, ctypes.byref(qc), _cb_host(codebook), _ptr(A),
                                       _ptr(B), r, float(alpha), pool_group, _ptr(y), _ptr(T_out),

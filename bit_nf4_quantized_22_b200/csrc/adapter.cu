@@ -16,27 +16,21 @@
 namespace qlora {
 namespace {
 
-__device__ __forceinline__ uint16_t to_bf16(float v) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-__device__ __forceinline__ float from_bf16(uint16_t v) {
-    return __bfloat162float(__ushort_as_bfloat16(v));
-}
-
-// dst[i][j] = j < r ? src[(i / rep)][j] * mul : 0     (dst: [rows][rp])
+// dst[i][j] = j < r ? src[(i / rep)][j] * mul : 0     (dst: [rows][rp]; 16-bit
+// values in the compute dtype, bf16 or fp16 when f16)
 __global__ void k_pad_rows(const uint16_t *__restrict__ src, int64_t rows, int r, int rp, int rep,
-                           float mul, uint16_t *__restrict__ dst) {
+                           float mul, uint16_t *__restrict__ dst, bool f16) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= rows * rp) return;
     const int64_t row = i / rp;
     const int j = (int)(i % rp);
-    dst[i] = j < r ? to_bf16(from_bf16(src[(row / rep) * r + j]) * mul) : (uint16_t)0;
+    dst[i] = j < r ? enc16(dec16(src[(row / rep) * r + j], f16) * mul, f16) : (uint16_t)0;
 }
 
-// pool(x)[m][k'] = (1/g) sum_i x[m][k' g + i], emitted as hi/lo bf16 terms
-// into [M][ld] buffers (columns k' >= Din/g are zero).
+// pool(x)[m][k'] = (1/g) sum_i x[m][k' g + i], emitted as hi/lo terms of the
+// compute dtype into [M][ld] buffers (columns k' >= Din/g are zero).
 __global__ void k_pool_split(const uint16_t *__restrict__ X, int64_t M, int64_t Din, int g,
-                             int64_t ld, uint16_t *__restrict__ hi, uint16_t *__restrict__ lo) {
+                             int64_t ld, uint16_t *__restrict__ hi, uint16_t *__restrict__ lo, bool f16) {
     const int64_t Da = Din / g;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= M * ld) return;
@@ -48,16 +42,16 @@ __global__ void k_pool_split(const uint16_t *__restrict__ X, int64_t M, int64_t 
     }
     const uint16_t *p = X + m * Din + k * g;
     float sum = 0.f;
-    for (int e = 0; e < g; ++e) sum += from_bf16(p[e]);
+    for (int e = 0; e < g; ++e) sum += dec16(p[e], f16);
     const float v = sum / (float)g;
-    const uint16_t h = to_bf16(v);
+    const uint16_t h = enc16(v, f16);
     hi[i] = h;
-    lo[i] = to_bf16(v - from_bf16(h));
+    lo[i] = enc16(v - dec16(h, f16), f16);
 }
 
-// fp32 [rows][r] -> bf16 [rows][2 rp] = [hi | lo] with zero padding
+// fp32 [rows][r] -> compute dtype [rows][2 rp] = [hi | lo] with zero padding
 __global__ void k_split_f32(const float *__restrict__ src, int64_t rows, int r, int rp,
-                            uint16_t *__restrict__ dst) {
+                            uint16_t *__restrict__ dst, bool f16) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= rows * rp) return;
     const int64_t row = i / rp;
@@ -65,8 +59,8 @@ __global__ void k_split_f32(const float *__restrict__ src, int64_t rows, int r, 
     uint16_t h = 0, l = 0;
     if (j < r) {
         const float v = src[row * r + j];
-        h = to_bf16(v);
-        l = to_bf16(v - from_bf16(h));
+        h = enc16(v, f16);
+        l = enc16(v - dec16(h, f16), f16);
     }
     dst[row * 2 * rp + j] = h;
     dst[row * 2 * rp + rp + j] = l;
@@ -87,6 +81,7 @@ struct ReduceArgs {
     float f32_scale; float *out_f32; int64_t fsp, fsq;
     float bf_scale; uint16_t *out_bf16; int64_t bsp;
     uint16_t *out_split; int64_t sp;
+    bool f16;             // 16-bit outputs in fp16 (else bf16)
 };
 
 // General layout (any Qp): one thread per output element.
@@ -102,11 +97,11 @@ __global__ void k_reduce_scalar(ReduceArgs a) {
         if (a.H) v += base[q + a.H];
     }
     if (a.out_f32) a.out_f32[p * a.fsp + q * a.fsq] = a.f32_scale * v;
-    if (a.out_bf16) a.out_bf16[p * a.bsp + q] = to_bf16(a.bf_scale * v);
+    if (a.out_bf16) a.out_bf16[p * a.bsp + q] = enc16(a.bf_scale * v, a.f16);
     if (a.out_split) {
-        const uint16_t h = to_bf16(v);
+        const uint16_t h = enc16(v, a.f16);
         a.out_split[p * 2 * a.sp + q] = h;
-        a.out_split[p * 2 * a.sp + a.sp + q] = to_bf16(v - from_bf16(h));
+        a.out_split[p * 2 * a.sp + a.sp + q] = enc16(v - dec16(h, a.f16), a.f16);
     }
 }
 
@@ -135,11 +130,11 @@ __global__ void __launch_bounds__(256) k_reduce(ReduceArgs a) {
         const int q = q0 + e;
         if (q >= a.Qv) break;
         if (a.out_f32) a.out_f32[p * a.fsp + q * a.fsq] = a.f32_scale * vv[e];
-        if (a.out_bf16) a.out_bf16[p * a.bsp + q] = to_bf16(a.bf_scale * vv[e]);
+        if (a.out_bf16) a.out_bf16[p * a.bsp + q] = enc16(a.bf_scale * vv[e], a.f16);
         if (a.out_split) {
-            const uint16_t h = to_bf16(vv[e]);
+            const uint16_t h = enc16(vv[e], a.f16);
             a.out_split[p * 2 * a.sp + q] = h;
-            a.out_split[p * 2 * a.sp + a.sp + q] = to_bf16(vv[e] - from_bf16(h));
+            a.out_split[p * 2 * a.sp + a.sp + q] = enc16(vv[e] - dec16(h, a.f16), a.f16);
         }
     }
 }
@@ -149,27 +144,28 @@ inline unsigned blocks_for(int64_t n, int t = 256) { return (unsigned)((n + t - 
 }  // namespace
 
 int launch_pad_rows(const uint16_t *src, int64_t rows, int r, int rp, int rep, float mul,
-                    uint16_t *dst, cudaStream_t st) {
+                    uint16_t *dst, cudaStream_t st, bool f16) {
     const int64_t n = rows * rp;
     if (n == 0) return QLORA_OK;
-    k_pad_rows<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, rep, mul, dst);
+    k_pad_rows<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, rep, mul, dst, f16);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }
 
 int launch_pool_split(const uint16_t *X, int64_t M, int64_t Din, int g, int64_t ld, uint16_t *hi,
-                      uint16_t *lo, cudaStream_t st) {
+                      uint16_t *lo, cudaStream_t st, bool f16) {
     const int64_t n = M * ld;
     if (n == 0) return QLORA_OK;
-    k_pool_split<<<blocks_for(n), 256, 0, st>>>(X, M, Din, g, ld, hi, lo);
+    k_pool_split<<<blocks_for(n), 256, 0, st>>>(X, M, Din, g, ld, hi, lo, f16);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }
 
-int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st) {
+int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st,
+                     bool f16) {
     const int64_t n = rows * rp;
     if (n == 0) return QLORA_OK;
-    k_split_f32<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, dst);
+    k_split_f32<<<blocks_for(n), 256, 0, st>>>(src, rows, r, rp, dst, f16);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }
@@ -177,9 +173,9 @@ int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *ds
 int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H, int Qv,
                   float f32_scale, float *out_f32, int64_t fsp, int64_t fsq, float bf_scale,
                   uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp,
-                  cudaStream_t st) {
+                  cudaStream_t st, bool f16) {
     ReduceArgs a{partial, splits, P, Qp, H, Qv, f32_scale, out_f32, fsp, fsq,
-                 bf_scale, out_bf16, bsp, out_split, sp};
+                 bf_scale, out_bf16, bsp, out_split, sp, f16};
     if (P * Qv == 0) return QLORA_OK;
     if (Qp % 4 != 0 || H % 4 != 0 || (reinterpret_cast<uintptr_t>(partial) & 15u) != 0) {
         k_reduce_scalar<<<blocks_for(P * Qv), 256, 0, st>>>(a);

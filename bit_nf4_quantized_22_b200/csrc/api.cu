@@ -15,27 +15,29 @@ int launch_nf4_dequantize_dtype(const nf4_weight_t &q, const Codebook &cb, int d
                                 cudaStream_t st);
 // merge.cu
 int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, const uint16_t *B,
-                 int r, int gp, float s, uint16_t *W_out, cudaStream_t st);
+                 int r, int gp, float s, uint16_t *W_out, cudaStream_t st, bool f16);
 // gemv.cu
 size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout);
 size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout);
 size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r);
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, uint32_t *d_status, cudaStream_t st,
+                    float *partial, uint32_t *d_status, cudaStream_t st, bool f16,
                     const uint16_t *Aad = nullptr, float *Tpart = nullptr, float *T_out = nullptr);
 int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *G, const uint16_t *Al, int r, int pool, float s, uint16_t *dX,
-                    float *partial, cudaStream_t st);
+                    float *partial, cudaStream_t st, bool f16);
 // adapter.cu
 int launch_pad_rows(const uint16_t *src, int64_t rows, int r, int rp, int rep, float mul,
-                    uint16_t *dst, cudaStream_t st);
+                    uint16_t *dst, cudaStream_t st, bool f16);
 int launch_pool_split(const uint16_t *X, int64_t M, int64_t Din, int g, int64_t ld, uint16_t *hi,
-                      uint16_t *lo, cudaStream_t st);
-int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st);
+                      uint16_t *lo, cudaStream_t st, bool f16);
+int launch_split_f32(const float *src, int64_t rows, int r, int rp, uint16_t *dst, cudaStream_t st,
+                     bool f16);
 int launch_reduce(const float *partial, int splits, int64_t P, int64_t Qp, int H, int Qv,
                   float f32_scale, float *out_f32, int64_t fsp, int64_t fsq, float bf_scale,
-                  uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp, cudaStream_t st);
+                  uint16_t *out_bf16, int64_t bsp, uint16_t *out_split, int64_t sp, cudaStream_t st,
+                  bool f16);
 // umma_skinny.cu
 struct SkinnySeg {
     const uint16_t *a;
@@ -50,11 +52,11 @@ struct SkinnySeg {
 int skinny_k_tiles(const SkinnySeg *segs, int nseg);
 void skinny_splits(int64_t P, int64_t Q, int nk, int *splits, int *per);
 int launch_umma_skinny(const SkinnySeg *segs, int nseg, int64_t P, int64_t Q, int64_t Qp,
-                       float *partial, uint32_t *d_status, cudaStream_t st);
+                       float *partial, uint32_t *d_status, cudaStream_t st, bool f16);
 // umma_gemm.cu
 int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t &q,
                       const Codebook &cb, const uint16_t *sAct, int r, const uint16_t *adapter,
-                      uint16_t *Y, uint32_t *d_status, cudaStream_t st);
+                      uint16_t *Y, uint32_t *d_status, cudaStream_t st, bool f16);
 
 namespace {
 
@@ -64,13 +66,17 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// 16 finite levels in [-1, 1], strictly increasing except that the zero
+// level may appear twice in a row (the FP4 table's -0 and +0); zero_idx is
+// the first zero, the level an all-zero block maps to.
 int check_codebook(const float *cb, int *zero_idx) {
     if (!cb) return QLORA_EINVAL;
     int zi = -1;
     for (int j = 0; j < 16; ++j) {
         if (!std::isfinite(cb[j]) || cb[j] < -1.f || cb[j] > 1.f) return QLORA_EINVAL;
-        if (j > 0 && !(cb[j] > cb[j - 1])) return QLORA_EINVAL;
-        if (cb[j] == 0.f) zi = j;
+        if (j > 0 && !(cb[j] > cb[j - 1]) && !(cb[j] == 0.f && cb[j - 1] == 0.f)) return QLORA_EINVAL;
+        if (j > 1 && cb[j] == 0.f && cb[j - 2] == 0.f) return QLORA_EINVAL;   // at most two zeros
+        if (cb[j] == 0.f && zi < 0) zi = j;
     }
     if (zi < 0) return QLORA_EINVAL;
     if (zero_idx) *zero_idx = zi;
@@ -91,12 +97,14 @@ int check_weight(const nf4_weight_t *q, bool need_rows, bool codec = false) {
         if (q->cols % 64 != 0) return QLORA_EINVAL;
         if (q->block != 64) return QLORA_EUNSUPPORTED;
     }
-    if (q->double_quant != 0 && q->double_quant != 1) return QLORA_EINVAL;
+    if (q->double_quant < QLORA_DQ_NONE || q->double_quant > QLORA_DQ_MEAN) return QLORA_EINVAL;
+    if (q->compute_dtype != QLORA_DTYPE_BF16 && q->compute_dtype != QLORA_DTYPE_FP16) return QLORA_EINVAL;
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!q->packed || !aligned16(q->packed)) return QLORA_EINVAL;
     if (q->double_quant) {
         if (q->dq_group != 256) return QLORA_EUNSUPPORTED;
         if (!q->absmax_code || !q->dq_step) return QLORA_EINVAL;
+        if (q->double_quant == QLORA_DQ_MEAN && !q->dq_mean) return QLORA_EINVAL;
     } else {
         if (!q->absmax) return QLORA_EINVAL;
     }
@@ -122,6 +130,7 @@ struct Dims {
     int r, rp, rp64, g;
     int64_t Da, Dap;
     bool small;
+    bool f16;   // the compute dtype is fp16 (else bf16)
 };
 
 Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
@@ -136,6 +145,7 @@ Dims make_dims(int64_t M, const nf4_weight_t *q, int r, int g) {
     d.Da = d.Din / g;
     d.Dap = round_up(d.Da, 8);
     d.small = M <= kGemvMaxM;
+    d.f16 = q->compute_dtype == QLORA_DTYPE_FP16;
     return d;
 }
 
@@ -165,9 +175,10 @@ size_t prod_partial_floats(const Prod &pr) {
     return (size_t)pl.splits * pr.P * pl.Qp;
 }
 
-int run_prod(const Prod &pr, float *partial, uint32_t *status, cudaStream_t st, ProdPlan *plan) {
+int run_prod(const Prod &pr, float *partial, uint32_t *status, cudaStream_t st, ProdPlan *plan,
+             bool f16) {
     *plan = plan_prod(pr);
-    return launch_umma_skinny(pr.seg, pr.nseg, pr.P, pr.Q, plan->Qp, partial, status, st);
+    return launch_umma_skinny(pr.seg, pr.nseg, pr.P, pr.Q, plan->Qp, partial, status, st, f16);
 }
 
 // T = u . A    (u = x [M, Din], or pooled hi/lo [M, Dap]; A padded [Da, rp])
@@ -317,19 +328,19 @@ int run_adapter_down(const Dims &d, const uint16_t *X, const uint16_t *A, uint16
     // A already has the padded row length (r a multiple of 16): use it in place
     const uint16_t *Ause = A;
     if (d.r != d.rp || !aligned16(A)) {
-        RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st));
+        RC(launch_pad_rows(A, d.Da, d.r, d.rp, 1, 1.f, Apad, st, d.f16));
         Ause = Apad;
     }
     ProdPlan plan;
-    RC(run_prod(prod_T(d, X, Ause, ph, pl), Tpart, status, st, &plan));
+    RC(run_prod(prod_T(d, X, Ause, ph, pl), Tpart, status, st, &plan, d.f16));
     if (sT && cudaMemsetAsync(sT, 0, d.M * d.rp64 * sizeof(uint16_t), st) != cudaSuccess)
         return QLORA_ECUDA;
     return launch_reduce(Tpart, plan.splits, d.M, plan.Qp, 0, d.r, 1.f, T32, d.r, 1, s, sT, d.rp64,
-                         nullptr, 0, st);
+                         nullptr, 0, st, d.f16);
 }
 
 int run_pool(const Dims &d, const uint16_t *X, uint16_t *ph, uint16_t *pl, cudaStream_t st) {
-    return launch_pool_split(X, d.M, d.Din, d.g, d.Dap, ph, pl, st);
+    return launch_pool_split(X, d.M, d.Din, d.g, d.Dap, ph, pl, st, d.f16);
 }
 
 }  // namespace
@@ -350,7 +361,7 @@ const char *qlora_strerror(int code) {
     }
 }
 
-int qlora_version(void) { return 100; }
+int qlora_version(void) { return 200; }
 
 int qlora_check_codebook(const float codebook[16]) { return check_codebook(codebook, nullptr); }
 
@@ -396,7 +407,7 @@ int qlora_merge(const nf4_weight_t *q, const float codebook[16], const uint16_t 
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!A || !B || !W_out || !aligned16(W_out)) return QLORA_EINVAL;
     return launch_merge(*q, to_cb(codebook), A, B, r, pool_group, alpha / (float)r, W_out,
-                        (cudaStream_t)stream);
+                        (cudaStream_t)stream, q->compute_dtype == QLORA_DTYPE_FP16);
 }
 
 size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t pool_group,
@@ -432,14 +443,15 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
         // one streamed kernel computes the base product and the adapter-down
         // partials, one finalize reduces both; else the general sequence
         const int rc = launch_gemv_fwd(X, (int)M, *q, cb, nullptr, B, r, s, Y, w.gemv_part, d_status,
-                                       st, A, w.gemv_tpart, T32);
+                                       st, d.f16, A, w.gemv_tpart, T32);
         if (rc != QLORA_EUNSUPPORTED) return rc;
     }
     if (d.g > 1) RC(run_pool(d, X, w.ph, w.pl, st));
     RC(run_adapter_down(d, X, A, w.Apad, w.ph, w.pl, w.Tpart, T32, s, d.small ? nullptr : w.sT,
                         d_status, st));
-    if (d.small) return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, d_status, st);
-    return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st);
+    if (d.small)
+        return launch_gemv_fwd(X, (int)M, *q, cb, T32, B, r, s, Y, w.gemv_part, d_status, st, d.f16);
+    return launch_umma_qgemm(0, X, M, *q, cb, w.sT, r, B, Y, d_status, st, d.f16);
 }
 
 // A second stream per device for the backward's adapter-gradient products,
@@ -480,16 +492,16 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     const Codebook cb = to_cb(codebook);
     const float s = alpha / (float)r;
 
-    // G = dY . B^T  (fp32), s*G (bf16, large M), hi/lo split (for dA)
+    // G = dY . B^T  (fp32), s*G (compute dtype, large M), hi/lo split (for dA)
     {
         ProdPlan pl;
-        RC(run_prod(prod_G(d, dY, B), w.Gpart, d_status, st, &pl));
+        RC(run_prod(prod_G(d, dY, B), w.Gpart, d_status, st, &pl, d.f16));
         uint16_t *sG = (want_dx && !d.small) ? w.sG : nullptr;
         if (sG && cudaMemsetAsync(sG, 0, M * d.rp64 * 2, st) != cudaSuccess) return QLORA_ECUDA;
         if (w.Gsplit && cudaMemsetAsync(w.Gsplit, 0, M * 2 * d.rp * 2, st) != cudaSuccess)
             return QLORA_ECUDA;
         RC(launch_reduce(w.Gpart, pl.splits, M, pl.Qp, 0, r, 1.f, w.G32, r, 1, s, sG, d.rp64,
-                         w.Gsplit, d.rp, st));
+                         w.Gsplit, d.rp, st, d.f16));
     }
     if (d.g > 1 && w.ph) RC(run_pool(d, X, w.ph, w.pl, st));
 
@@ -509,13 +521,15 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
 
     if (want_dx) {
         if (d.small) {
-            RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st));
+            RC(launch_gemv_bwd(dY, (int)M, *q, cb, w.G32, A, r, d.g, s, dX, w.gemv_part, st, d.f16));
         } else {
             // the extension operand is A itself when no padding, pooling or scaling applies
             const bool direct = d.g == 1 && r == d.rp64 && aligned16(A);
-            int rcx = direct ? QLORA_OK : launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st);
+            int rcx = direct ? QLORA_OK
+                             : launch_pad_rows(A, d.Din, r, d.rp64, d.g, 1.f / d.g, w.Aext, st, d.f16);
             if (rcx == QLORA_OK)
-                rcx = launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, direct ? A : w.Aext, dX, d_status, st);
+                rcx = launch_umma_qgemm(1, dY, M, *q, cb, w.sG, r, direct ? A : w.Aext, dX, d_status, st,
+                                        d.f16);
             if (rcx != QLORA_OK) {
                 if (ev_fork) cudaEventDestroy(ev_fork);
                 if (ev_join) cudaEventDestroy(ev_join);
@@ -527,10 +541,10 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
     if (side && cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess) rc = QLORA_ECUDA;
     if (rc == QLORA_OK && want_da) {
         ProdPlan pl;
-        rc = run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), w.dApart, d_status, ast, &pl);
+        rc = run_prod(prod_dA(d, X, w.ph, w.pl, w.Gsplit), w.dApart, d_status, ast, &pl, d.f16);
         if (rc == QLORA_OK)
             rc = launch_reduce(w.dApart, pl.splits, d.Da, pl.Qp, d.rp, r, s, dA, r, 1, 0.f, nullptr,
-                               0, nullptr, 0, ast);
+                               0, nullptr, 0, ast, d.f16);
     }
     if (rc == QLORA_OK && want_db) {
         const float *T32 = T_saved;
@@ -539,13 +553,13 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
                                   ast);
             T32 = w.T32;
         }
-        if (rc == QLORA_OK) rc = launch_split_f32(T32, M, r, d.rp, w.Tsplit, ast);
+        if (rc == QLORA_OK) rc = launch_split_f32(T32, M, r, d.rp, w.Tsplit, ast, d.f16);
         ProdPlan pl;
         if (rc == QLORA_OK)
-            rc = run_prod(prod_dB(d, dY, w.Tsplit), w.dBpart, d_status, ast, &pl);
+            rc = run_prod(prod_dB(d, dY, w.Tsplit), w.dBpart, d_status, ast, &pl, d.f16);
         if (rc == QLORA_OK)
             rc = launch_reduce(w.dBpart, pl.splits, d.Dout, pl.Qp, d.rp, r, s, dB, 1, d.Dout, 0.f,
-                               nullptr, 0, nullptr, 0, ast);
+                               nullptr, 0, nullptr, 0, ast, d.f16);
     }
     if (side) {
         // join: the caller's stream sees all of the backward (also on errors,

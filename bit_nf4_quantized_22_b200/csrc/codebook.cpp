@@ -1,4 +1,5 @@
-// codebook.cpp -- step 1 of the method on the host: the 16 NF4 levels.
+// codebook.cpp -- step 1 of the method on the host: the 16 levels of the
+// NF4 table, and of the FP4 table.
 //
 // "QLoRA：用4比特行李箱装下整个大模型" chapter 3 takes the levels from the
 // standard normal distribution: the CDF is cut into equal-probability pieces
@@ -105,5 +106,27 @@ extern "C" int nf4_codebook(double delta, float out[16]) {
     v[7] = 0.0;
     for (int i = 0; i < 8; ++i) v[15 - i] = inv_normal(delta + (0.5 - delta) * i / 8.0) / z;
     for (int i = 0; i < 16; ++i) out[i] = (float)v[i];
+    return QLORA_OK;
+}
+
+// FP4 ("大模型量化从0到1（十）：bitsandbytes" 6.4-6.5 and 9.3: bitsandbytes' other
+// 4-bit type is a float-style table, values not given).  The layout read for
+// it is E2M1 of the OCP Microscaling formats: sign, two exponent bits with
+// bias 1, one mantissa bit; exponent field 0 is subnormal (0 and 1/2).  Each
+// value is divided by the largest, 6, and the 16 codes are listed in
+// ascending order with -0 before +0.
+extern "C" int fp4_codebook(float out[16]) {
+    if (!out) return QLORA_EINVAL;
+    float v[16];
+    for (int code = 0; code < 16; ++code) {
+        const int sign = code >> 3, e = (code >> 1) & 3, m = code & 1;
+        const float mag = e ? std::ldexp(2.f + m, e - 2) : 0.5f * m;   // 2^(e-1) (1 + m/2)
+        v[code] = (sign ? -mag : mag) / 6.f;
+    }
+    // negative codes 15..8 (largest magnitude first), then positive codes 0..7
+    for (int i = 0; i < 8; ++i) {
+        out[i] = v[15 - i];
+        out[8 + i] = v[i];
+    }
     return QLORA_OK;
 }

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,19 +15,33 @@ struct Codebook {
     float c[16];
 };
 
-// Decoded first-level scale of block b: the fp32 absmax, or with double
-// quantization RN32(code * step) (one rounding of an exact product).
+// Decoded first-level scale of block b: the fp32 absmax (dq == 0), or with
+// double quantization RN32(code * step) (dq == 1: unsigned code, step max/255;
+// dq == 2: signed INT8 code, step max/127; one rounding of an exact product),
+// or RN32(mean + RN32(code * step)) with a signed code (dq == 3: the code of
+// the scale minus its group's mean).  One step and one mean per 256 blocks.
 struct ScaleSrc {
     const float *absmax;      // when !dq
     const uint8_t *code;      // when dq
     const float *step;        // when dq
     int dq;
+    const float *mean;        // when dq == 3
 };
+
+__device__ __forceinline__ float dq_decode(uint32_t code, float step, float mean, int dq) {
+    if (dq == 3) return __fadd_rn(mean, __fmul_rn((float)(int8_t)(uint8_t)code, step));
+    return __fmul_rn((float)code, step);
+}
 
 __device__ __forceinline__ float load_scale(const ScaleSrc &s, int64_t b) {
     if (!s.dq) return __ldg(s.absmax + b);
-    float f = __ldg(s.step + (b >> 8));
-    return __fmul_rn((float)__ldg(s.code + b), f);
+    const float f = __ldg(s.step + (b >> 8));
+    const float mu = s.dq == 3 ? __ldg(s.mean + (b >> 8)) : 0.f;
+    return dq_decode(__ldg(s.code + b), f, mu, s.dq);
+}
+
+__host__ __forceinline__ ScaleSrc scale_src(const nf4_weight_t &q) {
+    return ScaleSrc{q.absmax, q.absmax_code, q.dq_step, q.double_quant, q.dq_mean};
 }
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
@@ -36,6 +51,27 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// The layer's 16-bit compute dtype (bitsandbytes article (CSDN) 8.3):
+// bf16 (f16 == false) or IEEE binary16 (f16 == true).  Conversions round to
+// nearest even; fp16 keeps subnormals and overflows to infinity.
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool f16) {
+    if (!f16) return bf16x2_bits(lo, hi);
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float lo16(uint32_t v, bool f16) {
+    return f16 ? __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))) : bf16_lo(v);
+}
+__device__ __forceinline__ float hi16(uint32_t v, bool f16) {
+    return f16 ? __half2float(__ushort_as_half((unsigned short)(v >> 16))) : bf16_hi(v);
+}
+__device__ __forceinline__ float dec16(uint16_t v, bool f16) {
+    return f16 ? __half2float(__ushort_as_half(v)) : __bfloat162float(__ushort_as_bfloat16(v));
+}
+__device__ __forceinline__ uint16_t enc16(float v, bool f16) {
+    return f16 ? __half_as_ushort(__float2half_rn(v)) : __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
 
 // ---------------------------------------------------------------------------
 // NF4 decode through a per-block product table.
@@ -51,11 +87,11 @@ struct ProdTable {
     uint32_t hi[4];   // hi[i] byte k = high byte of entry 4i+k
 };
 
-__device__ __forceinline__ void build_table(float ah, const Codebook &cb, ProdTable &t) {
+__device__ __forceinline__ void build_table(float ah, const Codebook &cb, ProdTable &t, bool f16 = false) {
     uint32_t p[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-        p[i] = bf16x2_bits(__fmul_rn(ah, cb.c[2 * i]), __fmul_rn(ah, cb.c[2 * i + 1]));
+        p[i] = pack2(__fmul_rn(ah, cb.c[2 * i]), __fmul_rn(ah, cb.c[2 * i + 1]), f16);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         t.lo[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x6420);
@@ -96,6 +132,21 @@ __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// m16n8k16 in the compute dtype (both operands of one type, fp32 accumulate)
+template <bool F16>
+__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], const uint32_t b[2]) {
+    if (F16)
+        mma_f16_16816(d, a, b);
+    else
+        mma_bf16_16816(d, a, b);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -135,6 +186,9 @@ void prof_end(int kind, cudaStream_t st);
 // Streaming multiprocessors of the current device (cached per device; 148
 // if the query fails), for grids sized to whole waves.
 int device_sms();
+// cudaFuncSetAttribute(fn, MaxDynamicSharedMemorySize, bytes), made once per
+// (device, kernel) and remembered.
+cudaError_t set_max_smem(const void *fn, int bytes);
 }  // namespace qlora
 
 // Host-side launch check used after every kernel launch.

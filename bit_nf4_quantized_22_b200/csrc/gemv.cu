@@ -14,17 +14,19 @@
 namespace qlora {
 namespace {
 
-// Scale words fetched ahead of use (code + step, or the fp32 absmax).
+// Scale words fetched ahead of use (code + step (+ group mean), or the fp32 absmax).
 struct ScaleRawG {
     float f;
+    float mu;
     uint32_t code;
 };
 __device__ __forceinline__ ScaleRawG fetch_scale_g(const ScaleSrc &s, int64_t b, bool valid) {
-    ScaleRawG r{0.f, 0u};
+    ScaleRawG r{0.f, 0.f, 0u};
     if (valid) {
         if (s.dq) {
             r.code = __ldg(s.code + b);
             r.f = __ldg(s.step + (b >> 8));
+            if (s.dq == QLORA_DQ_MEAN) r.mu = __ldg(s.mean + (b >> 8));
         } else {
             r.f = __ldg(s.absmax + b);
         }
@@ -32,7 +34,7 @@ __device__ __forceinline__ ScaleRawG fetch_scale_g(const ScaleSrc &s, int64_t b,
     return r;
 }
 __device__ __forceinline__ float decode_scale_g(const ScaleRawG &r, int dq) {
-    return dq ? __fmul_rn((float)r.code, r.f) : r.f;
+    return dq ? dq_decode(r.code, r.f, r.mu, dq) : r.f;
 }
 
 constexpr int kGemvWarps = 8;
@@ -63,7 +65,7 @@ struct FwdBlockData {
     ScaleRawG s[2];
 };
 
-template <int NT>
+template <int NT, bool F16>
 __global__ void __launch_bounds__(kGemvWarps * 32, 2)
 k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
            const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
@@ -100,7 +102,7 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
     // 16-byte stores, rotated by lane so a warp's stores spread over banks.
     {
         const int e = threadIdx.x;
-        const uint32_t v = bf16x2_bits(cb.c[e >> 4], cb.c[e & 15]);
+        const uint32_t v = pack2(cb.c[e >> 4], cb.c[e & 15], F16);
         uint4 *row = reinterpret_cast<uint4 *>(lut + e * 32);
         const uint4 vv = make_uint4(v, v, v, v);
 #pragma unroll
@@ -152,7 +154,7 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
             for (int n = 0; n < NT; ++n) {
                 const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][64 * b + 16 * t + 4 * st]);
                 const uint32_t bb[2] = {xv.x, xv.y};
-                mma_bf16_16816(tmp[n], a, bb);
+                mma16816<F16>(tmp[n], a, bb);
             }
         }
         const float a0 = decode_scale_g(cur.s[0], sc.dq), a1 = decode_scale_g(cur.s[1], sc.dq);
@@ -178,16 +180,21 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
 }
 
 // ------------------------------------------------------------------ forward, streamed
-// Persistent variant: one CTA per SM walks a contiguous range of
-// (input-slice, 128-row) tiles, slices of 1024 inputs.  A producer warp
-// streams each tile as two half-tiles (128 rows x 256 packed bytes, two
-// 128-byte-swizzled TMA boxes, plus the rows' scale codes) through a
-// three-stage shared-memory ring, so loads run ahead independently of
-// registers.
+// Persistent: one CTA per SM walks a contiguous range of units (slice z of
+// 1024 inputs, tile of 128 rows), numbered slice-major so that a CTA
+// restages its x slice rarely.  A producer warp streams each unit as two
+// half-tiles (128 rows x 256 packed bytes, two 128-byte-swizzled TMA boxes)
+// through a three-stage shared-memory ring.  Its 32 lanes also decode the
+// half-tile's block scales a_hat (lane l: rows l, l + 32, l + 64, l + 96, eight
+// blocks each, from scale words loaded one half-tile ahead) into the stage,
+// stored [block parity][row][4] so that a compute lane reads the four scales
+// it needs of one row with a single 16-byte load.
 //
-// Sixteen compute warps: warps w and w + 8 own the same 16 rows and take
-// the even and the odd 64-blocks of each half-tile, four blocks each; the
-// two warps' sums meet in shared memory once per tile (even + odd).
+// Sixteen compute warps: warps w and w + 8 own the same 16 rows and take the
+// even and the odd 64-blocks of each half-tile, four blocks each.  The four
+// blocks' MMA chains are independent (one accumulator set per block, scaled
+// by its a_hat and summed afterwards).  The two warps' sums meet in shared
+// memory once per unit, ordered by a barrier of those two warps alone.
 //
 // Decode: the byte -> bf16-pair table has one 256-byte row per byte value,
 // lane l's copy at +4l, so the shared address of a lookup is exactly
@@ -199,11 +206,10 @@ k_gemv_fwd(const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout,
 // tiles, also compute the adapter-down partials of one rank tile each,
 // Tpart[z][b][m][j] = sum over the 64 inputs k of block b of x[m][k] A[k][j],
 // warp w taking block w, as MMAs with the 16 ranks on the M side (A^T
-// gathered from the row-major A) and the tokens on the N side.  Needs the scale rows to be TMA-tileable: Din/64 a
-// multiple of 16 (codes) or of 4 (fp32 absmax).
+// gathered from the row-major A) and the tokens on the N side.
 constexpr int kStRows = 128, kStBlocks = 16;              // tile: 128 rows x 1024 inputs
 constexpr int kStHalf = kStRows * 8 * 32;                 // half-tile packed bytes: 32 KB
-constexpr int kStStage = kStHalf + 4096;                  // + scales (codes 2 KB / fp32 4 KB)
+constexpr int kStStage = kStHalf + 4096;                  // + a_hat [2][128][4] fp32
 constexpr int kStStages = 3;
 constexpr int kStCompute = 16;                            // compute warps
 static_assert(kStCompute == kStBlocks, "the adapter-down work gives each warp one block");
@@ -214,13 +220,12 @@ constexpr int kStX = (16 * kStXPitch * 2 + 1023) / 1024 * 1024;
 constexpr int kStRed = 2 * 8 * 32 * 8 * 4;                // two buffers of the odd warps' sums
 constexpr int kStSmem = kStLut + kStX + kStStages * kStStage + kStRed + 1024 + 256;
 
-template <int NT>
+template <bool DQ, int NT, bool F16>
 __global__ void __launch_bounds__(kStThreads, 1)
-k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmC,
-                  const uint16_t *__restrict__ X, int M, int64_t Din, int64_t Dout, ScaleSrc sc,
-                  Codebook cb, int ntr, int ntiles, float *__restrict__ partial,
-                  const uint16_t *__restrict__ Aad, int r, float *__restrict__ Tpart,
-                  uint32_t *__restrict__ status) {
+k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const uint16_t *__restrict__ X, int M,
+                  int64_t Din, int64_t Dout, ScaleSrc sc, Codebook cb, int ntr, int ntiles,
+                  float *__restrict__ partial, const uint16_t *__restrict__ Aad, int r,
+                  float *__restrict__ Tpart, uint32_t *__restrict__ status) {
     extern __shared__ __align__(1024) uint8_t ssm[];
     const uint32_t raw = smem_u32(ssm);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -249,7 +254,7 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
 #pragma unroll
         for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
         for (int s = 0; s < kStStages; ++s) {
-            tc::mbar_init(full(s), 1);
+            tc::mbar_init(full(s), 32);
             tc::mbar_init(empty(s), kStCompute);
         }
         *abort_flag = 0;
@@ -259,7 +264,7 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
     __syncthreads();
     if (threadIdx.x < 256) {   // table row e: 32 copies of (c[e >> 4], c[e & 15]) in bf16
         const int e = threadIdx.x;
-        const uint32_t v = bf16x2_bits(cbs[e >> 4], cbs[e & 15]);
+        const uint32_t v = pack2(cbs[e >> 4], cbs[e & 15], F16);
         uint4 *row = reinterpret_cast<uint4 *>(gbase + e * 256);
         const uint4 vv = make_uint4(v, v, v, v);
 #pragma unroll
@@ -278,30 +283,75 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
 
     if (warp == kStCompute) {
         // ---------------------------------------------------------- producer
-        if (lane == 0) {
-            const uint32_t cbytes = sc.dq ? kStRows * 16 : kStRows * 8 * 4;
-            int hi = 0;
-            for (int tt = t0; tt < t1 && ok; ++tt) {
-                const int z = tt / ntr, rt = tt % ntr;
-                const int nh = halves(z);
-                for (int h = 0; h < nh && ok; ++h, ++hi) {
-                    const int s = hi % kStStages;
-                    if (hi >= kStStages) ok = tc::mbar_wait(empty(s), ((hi / kStStages) & 1) ^ 1, abort_flag);
-                    if (!ok) break;
-                    const uint32_t st = ring + s * kStStage;
-                    tc::mbar_expect_tx(full(s), kStHalf + cbytes);
+        uint2 cw[4];        // DQ: the half's 8 codes of rows lane + 32 j
+        float sf[4], smu[4];   // DQ: their second-level step (and group mean)
+        float4 am[4][2];    // fp32 absmax of the same rows
+        auto fetch = [&](int tt, int h) {
+            const int z = tt / ntr, rt = tt % ntr;
+            const int64_t kb0 = (int64_t)z * kStBlocks + 8 * h;      // first block of the half
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t n = (int64_t)rt * kStRows + lane + 32 * j;
+                const bool okr = n < Dout;
+                const int64_t b0 = n * nbr + kb0;
+                if (DQ) {
+                    // 8 | nbr: the half's 8 blocks start 8-aligned, inside one group of 256
+                    cw[j] = okr ? __ldg(reinterpret_cast<const uint2 *>(sc.code + b0)) : make_uint2(0u, 0u);
+                    sf[j] = okr ? __ldg(sc.step + (b0 >> 8)) : 0.f;
+                    smu[j] = okr && sc.dq == QLORA_DQ_MEAN ? __ldg(sc.mean + (b0 >> 8)) : 0.f;
+                } else {
+                    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 *p = reinterpret_cast<const float4 *>(sc.absmax + b0);
+                    am[j][0] = okr ? __ldg(p) : z4;
+                    am[j][1] = (okr && kb0 + 4 < nbr) ? __ldg(p + 1) : z4;
+                }
+            }
+        };
+        int hi = 0;
+        if (t0 < t1) fetch(t0, 0);
+        for (int tt = t0; tt < t1 && ok; ++tt) {
+            const int z = tt / ntr, rt = tt % ntr;
+            const int nh = halves(z);
+            for (int h = 0; h < nh; ++h, ++hi) {
+                const int s = hi % kStStages;
+                if (hi >= kStStages)
+                    ok = __all_sync(0xffffffffu, tc::mbar_wait(empty(s), ((hi / kStStages) & 1) ^ 1, abort_flag));
+                if (!ok) break;
+                const uint32_t st = ring + s * kStStage;
+                if (lane == 0) {
+                    tc::mbar_expect_tx_only(full(s), kStHalf);
 #pragma unroll
                     for (int q = 0; q < 2; ++q)
                         tc::tma_load_2d(st + q * (kStRows * 128), &tmP,
                                         z * (kFwdKS / 2) + h * 256 + 128 * q, rt * kStRows, full(s));
-                    if (sc.dq)   // the whole slice's 16 codes per row, read by both halves
-                        tc::tma_load_2d(st + kStHalf, &tmC, z * kStBlocks, rt * kStRows, full(s));
-                    else
-                        tc::tma_load_2d(st + kStHalf, &tmC, z * kStBlocks + 8 * h, rt * kStRows, full(s));
                 }
+                float4 *ah = reinterpret_cast<float4 *>(gring + s * kStStage + kStHalf);   // [2][128]
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float4 ev, od;   // blocks 0, 2, 4, 6 and 1, 3, 5, 7 of the half
+                    if (DQ) {
+                        const uint32_t x = cw[j].x, y = cw[j].y;
+                        const float f = sf[j], mu = smu[j];
+                        const int k = sc.dq;
+                        // rows of scale-less padding (past Dout) decode to 0 or mu * 0: harmless
+                        ev = make_float4(dq_decode(x & 0xffu, f, mu, k), dq_decode((x >> 16) & 0xffu, f, mu, k),
+                                         dq_decode(y & 0xffu, f, mu, k), dq_decode((y >> 16) & 0xffu, f, mu, k));
+                        od = make_float4(dq_decode((x >> 8) & 0xffu, f, mu, k), dq_decode(x >> 24, f, mu, k),
+                                         dq_decode((y >> 8) & 0xffu, f, mu, k), dq_decode(y >> 24, f, mu, k));
+                    } else {
+                        const float4 a0 = am[j][0], a1 = am[j][1];
+                        ev = make_float4(a0.x, a0.z, a1.x, a1.z);
+                        od = make_float4(a0.y, a0.w, a1.y, a1.w);
+                    }
+                    ah[lane + 32 * j] = ev;
+                    ah[kStRows + lane + 32 * j] = od;
+                }
+                tc::mbar_arrive(full(s));
+                if (h + 1 < nh) fetch(tt, h + 1);
+                else if (tt + 1 < t1) fetch(tt + 1, 0);
             }
-            if (!ok) *abort_flag = 1;
         }
+        if (!ok && lane == 0) *abort_flag = 1;
     } else {
         // ---------------------------------------------------------- compute warps
         // lookup address = (byte << 8) | 4 * lane, from one permute
@@ -312,6 +362,17 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
         };
         const int rl = (warp & 7) * 16 + g;            // rows rl and rl + 8 of the tile
         const int bpar = warp >> 3;                    // this warp's blocks: b = bpar mod 2
+        const uint32_t pair_bar = 8u + (uint32_t)(warp & 7);   // named barrier of warps w, w + 8
+        // packed bytes of block bh = 2i + bpar of row rl: box bh / 4 holds rows x 128 B;
+        // this lane's 8 bytes are 16-byte chunk 2 (bh % 4) + t / 2 (swizzled by row), half t % 2
+        int pko[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int bh = 2 * i + bpar;
+            const int chunk = 2 * (bh & 3) + (t >> 1);
+            pko[i] = (bh >> 2) * (kStRows * 128) + rl * 128 + ((chunk ^ (rl & 7)) << 4) + 8 * (t & 1);
+        }
+        const int aho = kStHalf + (bpar * kStRows + rl) * 16;
         // Every compute warp walks the same tiles and meets the same named
         // barriers; after a failed wait a warp keeps walking (skipping the
         // work) so that no other warp is left at a barrier.
@@ -320,14 +381,6 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
             const int z = tt / ntr, rt = tt % ntr;
             const int64_t k0 = (int64_t)z * kFwdKS;
             const int64_t row0 = (int64_t)rt * kStRows + rl;
-            const bool ok0 = row0 < Dout, ok1 = row0 + 8 < Dout;
-            // with double quantization a row's 16 blocks of this slice start at a
-            // multiple of 16 and so lie inside one group of 256 blocks
-            float step0 = 0.f, step1 = 0.f;
-            if (sc.dq) {
-                if (ok0) step0 = __ldg(sc.step + ((row0 * nbr + z * kStBlocks) >> 8));
-                if (ok1) step1 = __ldg(sc.step + (((row0 + 8) * nbr + z * kStBlocks) >> 8));
-            }
             if (z != prev_z) {                         // stage x[:M, k0 : k0 + 1024]
                 asm volatile("bar.sync 1, %0;\n" ::"n"(kStCompute * 32));
                 for (int j = threadIdx.x; j < M * (kFwdKS / 4); j += kStCompute * 32) {
@@ -350,66 +403,58 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
                 const int s = hi % kStStages;
                 if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (hi / kStStages) & 1, abort_flag));
                 if (!ok) {
-                    *abort_flag = 1;
+                    if (lane == 0) *abort_flag = 1;
                     continue;
                 }
                 const uint8_t *stg = gring + s * kStStage;
-                const int hb = nblk - 8 * h < 8 ? nblk - 8 * h : 8;   // blocks in this half
-                auto block = [&](int bh) {
-                    // packed: box bh/4 holds rows x 128 B; this lane's 8 bytes of
-                    // block bh are 16-byte chunk 2(bh%4) + t/2 (swizzled by row), half t%2
-                    const int chunk = 2 * (bh & 3) + (t >> 1);
-                    const uint8_t *pb = stg + (bh >> 2) * (kStRows * 128) + ((chunk ^ (rl & 7)) << 4) + 8 * (t & 1);
-                    const uint2 w0 = *reinterpret_cast<const uint2 *>(pb + rl * 128);
-                    const uint2 w1 = *reinterpret_cast<const uint2 *>(pb + (rl + 8) * 128);
-                    float a0, a1;
-                    if (sc.dq) {
-                        const uint8_t *cs = stg + kStHalf;
-                        a0 = __fmul_rn((float)cs[rl * 16 + 8 * h + bh], step0);
-                        a1 = __fmul_rn((float)cs[(rl + 8) * 16 + 8 * h + bh], step1);
-                    } else {
-                        const float *as = reinterpret_cast<const float *>(stg + kStHalf);
-                        a0 = as[rl * 8 + bh];
-                        a1 = as[(rl + 8) * 8 + bh];
-                    }
-                    float tmp[NT][4];
+                // blocks past a ragged end hold zero-filled packed bytes, a zero
+                // scale and zero x: they add nothing
+                const float4 s0 = *reinterpret_cast<const float4 *>(stg + aho);
+                const float4 s1 = *reinterpret_cast<const float4 *>(stg + aho + 8 * 16);
+                uint2 w0[4], w1[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    w0[i] = *reinterpret_cast<const uint2 *>(stg + pko[i]);
+                    w1[i] = *reinterpret_cast<const uint2 *>(stg + pko[i] + 8 * 128);
+                }
+                float tmp[4][NT][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int n = 0; n < NT; ++n)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) tmp[n][e] = 0.f;
-                    const int kx = 64 * (8 * h + bh) + 16 * t;
+                        for (int e = 0; e < 4; ++e) tmp[i][n][e] = 0.f;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t x0 = q < 2 ? w0.x : w0.y;
-                        const uint32_t x1 = q < 2 ? w1.x : w1.y;
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t x0 = q < 2 ? w0[i].x : w0[i].y;
+                        const uint32_t x1 = q < 2 ? w1[i].x : w1[i].y;
                         const int i0 = (2 * q) & 3;
                         const uint32_t a[4] = {lookup(x0, i0), lookup(x1, i0), lookup(x0, i0 + 1),
                                                lookup(x1, i0 + 1)};
+                        const int kx = 64 * (8 * h + 2 * i + bpar) + 16 * t + 4 * q;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
                             // token rows past M are zero: skip their shared loads
                             const uint2 xv = g + 8 * n < M
-                                                 ? *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kx + 4 * q])
+                                                 ? *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kx])
                                                  : make_uint2(0u, 0u);
                             const uint32_t bb[2] = {xv.x, xv.y};
-                            mma_bf16_16816(tmp[n], a, bb);
+                            mma16816<F16>(tmp[i][n], a, bb);
                         }
                     }
+                }
+                const float c0[4] = {s0.x, s0.y, s0.z, s0.w}, c1[4] = {s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        acc[n][0] = fmaf(a0, tmp[n][0], acc[n][0]);
-                        acc[n][1] = fmaf(a0, tmp[n][1], acc[n][1]);
-                        acc[n][2] = fmaf(a1, tmp[n][2], acc[n][2]);
-                        acc[n][3] = fmaf(a1, tmp[n][3], acc[n][3]);
+                        acc[n][0] = fmaf(c0[i], tmp[i][n][0], acc[n][0]);
+                        acc[n][1] = fmaf(c0[i], tmp[i][n][1], acc[n][1]);
+                        acc[n][2] = fmaf(c1[i], tmp[i][n][2], acc[n][2]);
+                        acc[n][3] = fmaf(c1[i], tmp[i][n][3], acc[n][3]);
                     }
-                };
-                // this warp's blocks of the half: bh = bpar, bpar + 2, ...
-                if (hb == 8) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) block(2 * i + bpar);
-                } else {
-                    for (int bh = bpar; bh < hb; bh += 2) block(bh);
-                }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(empty(s));
             }
@@ -446,7 +491,7 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
                         for (int n = 0; n < NT; ++n) {
                             const uint2 xv = *reinterpret_cast<const uint2 *>(&sx[g + 8 * n][kk]);
                             const uint32_t bb[2] = {xv.x, xv.y};
-                            mma_bf16_16816(ta[n], a, bb);
+                            mma16816<F16>(ta[n], a, bb);
                         }
                     }
                     // ta[n]: (rank ja, tokens 8n + 2t, +1) and (rank jb, same tokens)
@@ -462,14 +507,14 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
                 }
             }
             // odd-block warps hand their sums to the even-block warps (buffer
-            // rpar; the barrier of the next tile orders its reuse)
+            // rpar; the pair's barrier of the next unit orders its reuse)
             float *rb = red + ((rpar * 8 + (warp & 7)) * 32 + lane) * 8;
             if (bpar) {
 #pragma unroll
                 for (int n = 0; n < NT; ++n)
                     *reinterpret_cast<float4 *>(rb + 4 * n) = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
             }
-            asm volatile("bar.sync 2, %0;\n" ::"n"(kStCompute * 32));
+            asm volatile("bar.sync %0, 64;\n" ::"r"(pair_bar) : "memory");
             if (!ok || bpar) continue;
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
@@ -498,7 +543,7 @@ k_gemv_fwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
 __global__ void __launch_bounds__(256)
 k_gemv_fwd_finalize_fused(const float *__restrict__ partial, int nsplit, int M, int64_t Dout,
                           const float *__restrict__ Tpart, int r, const uint16_t *__restrict__ Bl,
-                          float s, uint16_t *__restrict__ Y, float *__restrict__ T_out) {
+                          float s, uint16_t *__restrict__ Y, float *__restrict__ T_out, bool f16) {
     __shared__ float Ts[QLORA_MAX_RANK];
     __shared__ float Tg[256];
     const int m = blockIdx.y;
@@ -528,15 +573,15 @@ k_gemv_fwd_finalize_fused(const float *__restrict__ partial, int nsplit, int M, 
     for (int z = 0; z < nsplit; ++z) v += partial[((int64_t)z * M + m) * Dout + n];
     float ad = 0.f;
     for (int j = 0; j < r; ++j)
-        ad = fmaf(Ts[j], __bfloat162float(__ushort_as_bfloat16(Bl[(int64_t)j * Dout + n])), ad);
-    Y[(int64_t)m * Dout + n] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(s, ad, v)));
+        ad = fmaf(Ts[j], dec16(Bl[(int64_t)j * Dout + n], f16), ad);
+    Y[(int64_t)m * Dout + n] = enc16(fmaf(s, ad, v), f16);
 }
 
 // y[m, n] = sum_split partial + s * sum_j T[m, j] B[j, n]
 __global__ void k_gemv_fwd_finalize(const float *__restrict__ partial, int nsplit, int M,
                                     int64_t Dout, const float *__restrict__ T,
                                     const uint16_t *__restrict__ Bl, int r, float s,
-                                    uint16_t *__restrict__ Y) {
+                                    uint16_t *__restrict__ Y, bool f16) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)M * Dout) return;
     const int m = (int)(i / Dout);
@@ -545,8 +590,8 @@ __global__ void k_gemv_fwd_finalize(const float *__restrict__ partial, int nspli
     for (int z = 0; z < nsplit; ++z) v += partial[(int64_t)z * M * Dout + i];
     float ad = 0.f;
     for (int j = 0; j < r; ++j)
-        ad = fmaf(T[m * r + j], __bfloat162float(__ushort_as_bfloat16(Bl[(int64_t)j * Dout + nn])), ad);
-    Y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(s, ad, v)));
+        ad = fmaf(T[m * r + j], dec16(Bl[(int64_t)j * Dout + nn], f16), ad);
+    Y[i] = enc16(fmaf(s, ad, v), f16);
 }
 
 // ------------------------------------------------------------------ backward dX
@@ -557,6 +602,7 @@ __global__ void k_gemv_fwd_finalize(const float *__restrict__ partial, int nspli
 // (0..7) covers columns k0 + 8g' + i for g' = 0..7: the A operand is dY with
 // the 16 tokens as M and the 16 rows as the reduction, the B operand the 16
 // rows x 8 columns of weights.
+template <bool F16>
 __global__ void __launch_bounds__(kGemvWarps * 32)
 k_gemv_bwd(const uint16_t *__restrict__ dY, int M, int64_t Din, int64_t Dout,
            const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
@@ -609,7 +655,7 @@ k_gemv_bwd(const uint16_t *__restrict__ dY, int M, int64_t Din, int64_t Dout,
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             ProdTable tab;
-            build_table(ah[q][j], cb, tab);
+            build_table(ah[q][j], cb, tab, F16);
             decode8(wv[q][j], tab, R[j]);
         }
         const int nl = warp * kBwdRowsPerWarp + 16 * q + 4 * t;
@@ -623,7 +669,7 @@ k_gemv_bwd(const uint16_t *__restrict__ dY, int M, int64_t Din, int64_t Dout,
             const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
             const uint32_t b[2] = {__byte_perm(R[0][i >> 1], R[1][i >> 1], sel),
                                    __byte_perm(R[2][i >> 1], R[3][i >> 1], sel)};
-            mma_bf16_16816(acc[i], a, b);
+            mma16816<F16>(acc[i], a, b);
         }
     }
 
@@ -649,49 +695,73 @@ k_gemv_bwd(const uint16_t *__restrict__ dY, int M, int64_t Din, int64_t Dout,
             float ad = 0.f;
             const int64_t ka = k / pool;
             for (int j = 0; j < r; ++j)
-                ad = fmaf(G[m * r + j], __bfloat162float(__ushort_as_bfloat16(Al[ka * r + j])), ad);
-            dX[(int64_t)m * Din + k] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(s / pool, ad, v)));
+                ad = fmaf(G[m * r + j], dec16(Al[ka * r + j], F16), ad);
+            dX[(int64_t)m * Din + k] = enc16(fmaf(s / pool, ad, v), F16);
         }
     }
 }
 
 // ------------------------------------------------------------------ backward dX, streamed
-// grid (Din / 512 slices kz, nsplit): CTA (kz, sp) reduces over its range of
-// 128-row tiles of the weight, dX[m][k] for the slice's 512 inputs k.  A
-// producer warp streams each tile -- the packed rows (two 128-byte-swizzled
-// boxes of 128 rows x 128 bytes), the rows' scale codes and dY[:, rows] (two
-// 64-column swizzled boxes of min(M, 16) token rows; the rows past M hold
-// whatever the buffer held, which only reaches output rows that are never
-// stored) -- through a three-stage ring.
+// Work units are (slice kz of 512 inputs, tile of 128 weight rows), numbered
+// slice-major: u = kz * ntn + tile.  CTA c of G takes the contiguous units
+// [c T / G, (c + 1) T / G) of the T = nkz * ntn, so every SM gets the same
+// share of the weight whatever its shape.  Inside one slice a CTA's warps
+// keep dX[:, slice] in registers over its tiles and flush it to a partial
+// slot when the slice changes or the range ends; the slot of CTA c for slice
+// kz is c - owner(kz * ntn), owner(u) being the CTA whose range holds unit u.
 //
-// Sixteen compute warps: warp w owns the 64-block kb = w % 8 of the slice
-// and the 16-row groups q = w / 8, w / 8 + 2, ... of every tile, and keeps
-// its 16 tokens x 64 inputs accumulator in registers across the whole range
-// (warps w and w + 8 are added once at the end).  MMA m16n8k16: the tokens
-// are M, 8 inputs {8g' + i} are N (MMA i = 0..7), and the group's 16 rows are
-// K, relabelled so that lane t's K slots 2t, 2t+1, 2t+8, 2t+9 are its rows
-// 4t..4t+3.  Lane (g, t) reads one packed word (inputs 8g..8g+7) of each of
-// its four rows, decodes it with four lookups of the byte -> bf16-pair table
-// (the same table as the forward), and pairs rows with byte permutes.  The
-// weights there are the bare codebook values, so the per-row block scale is
-// moved onto dY: dY[m][n] * a_hat[n][kb], exactly, as a hi + lo pair of bf16
-// (two MMAs), so that only the codebook's own bf16 rounding remains.
+// Producer warp, per unit: lane 0 starts the TMA copies of the packed rows
+// (two 128-byte-swizzled boxes of 128 rows x 128 bytes) and of dY[:, rows]
+// (two 64-column boxes of min(M, 16) token rows; the rows past M hold
+// whatever the buffer held and only reach output rows that are never
+// stored).  All 32 lanes decode the block scales a_hat of their four rows
+// 4l..4l+3 for the slice's eight blocks, from scale words loaded one unit
+// ahead, store them [block][row] into the stage and arrive.
+//
+// Sixteen compute warps: warp w owns the 64-input block kb = w % 8 of the
+// slice and the 16-row groups q = w / 8, w / 8 + 2, ... of every tile.  MMA
+// m16n8k16: the tokens are M, 8 inputs {8g' + i} are N (MMA i = 0..7), the
+// group's 16 rows are K, relabelled so that lane t's K slots 2t, 2t+1, 2t+8,
+// 2t+9 are its rows 4t..4t+3.  The A operand is d = dY[m][n] a_hat[n][kb]
+// as an unevaluated pair of bf16 terms hi + lo (about 16 significant bits):
+// the row's block scale rides on dY.  With M <= 8 the lo terms fill the
+// MMA's empty token rows 8..15 and are added to rows 0..7 at the flush; with
+// more tokens a second MMA takes them.  For B, lane (g, t) reads
+// one packed word (inputs 8g..8g+7) of each of its four rows; interleaving
+// the nibbles of rows 4t and 4t+1 (and of 4t+2 and 4t+3) gives bytes holding
+// one input of both rows, and one lookup of the byte -> bf16-pair table (the
+// forward's) turns each such byte into the B register (row 4t, row 4t+1) of
+// that input.
 constexpr int kBsRows = 128, kBsCols = 512;
 constexpr int kBsPacked = kBsRows * kBsCols / 2;           // 32 KB
-constexpr int kBsScale = kBsRows * 8 * 4;                   // 4 KB (codes use 2 KB)
 constexpr int kBsDy = 2 * 16 * 128;                         // two [16][64] bf16 boxes
-constexpr int kBsStage = kBsPacked + kBsScale + kBsDy;      // 40 KB
+constexpr int kBsScale = 8 * kBsRows * 4;                   // a_hat [8 blocks][128 rows] fp32
+constexpr int kBsStage = kBsPacked + kBsDy + kBsScale;      // 40 KB
 constexpr int kBsStages = 3;
 constexpr int kBsThreads = 17 * 32;
 constexpr int kBsRed = 8 * 32 * 32 * 4;                    // odd-parity warps' sums
 constexpr int kBsSmem = kStLut + kBsStages * kBsStage + kBsRed + 1024 + 256;
 static_assert(kBsStage % 1024 == 0, "stages keep 1 KB swizzle alignment");
 
+// dY pair v (two 16-bit values of the compute dtype) times two scales, as
+// hi + lo pairs of that dtype: hi = RN(d), lo = RN(d - hi), d = RN32(dY * a_hat).
+template <bool F16>
+__device__ __forceinline__ void split_scaled(uint32_t v, float s0, float s1, uint32_t &hi, uint32_t &lo) {
+    const float d0 = lo16(v, F16) * s0, d1 = hi16(v, F16) * s1;
+    hi = pack2(d0, d1, F16);
+    lo = pack2(d0 - lo16(hi, F16), d1 - hi16(hi, F16), F16);
+}
+
+// The CTA (of G, over T units) whose contiguous range holds unit u.
+__host__ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t G, int64_t T) {
+    return ((u + 1) * G - 1) / T;
+}
+
+template <bool DQ, int MT, bool F16>
 __global__ void __launch_bounds__(kBsThreads, 1)
-k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmC,
-                  const __grid_constant__ CUtensorMap tmD, int M, int Mb, int64_t Din, int64_t Dout,
-                  ScaleSrc sc, Codebook cb, int ntn, int nsplit, float *__restrict__ partial,
-                  uint32_t *__restrict__ status) {
+k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmD,
+                  int M, int Mb, int64_t Din, int64_t Dout, ScaleSrc sc, Codebook cb, int ntn,
+                  int nkz, int nslot, float *__restrict__ partial, uint32_t *__restrict__ status) {
     extern __shared__ __align__(1024) uint8_t ssm[];
     const uint32_t raw = smem_u32(ssm);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -708,15 +778,15 @@ k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int kz = blockIdx.x, sp = blockIdx.y;
-    const int t0 = (int)((int64_t)sp * ntn / nsplit), t1 = (int)((int64_t)(sp + 1) * ntn / nsplit);
+    const int64_t T = (int64_t)nkz * ntn, G = gridDim.x, c = blockIdx.x;
+    const int64_t u0 = c * T / G, u1 = (c + 1) * T / G;
     const int64_t nbr = Din / 64;
 
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) cbs[j] = cb.c[j];
         for (int s = 0; s < kBsStages; ++s) {
-            tc::mbar_init(full(s), 1);
+            tc::mbar_init(full(s), 32);
             tc::mbar_init(empty(s), 16);
         }
         *abort_flag = 0;
@@ -726,7 +796,7 @@ k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
     __syncthreads();
     if (threadIdx.x < 256) {   // table row e: 32 copies of (c[e >> 4], c[e & 15]) in bf16
         const int e = threadIdx.x;
-        const uint32_t v = bf16x2_bits(cbs[e >> 4], cbs[e & 15]);
+        const uint32_t v = pack2(cbs[e >> 4], cbs[e & 15], F16);
         uint4 *row = reinterpret_cast<uint4 *>(gbase + e * 256);
         const uint4 vv = make_uint4(v, v, v, v);
 #pragma unroll
@@ -737,28 +807,68 @@ k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
 
     if (warp == 16) {
         // ---------------------------------------------------------- producer
-        if (lane == 0) {
-            const uint32_t cbytes = sc.dq ? kBsRows * 16 : kBsRows * 8 * 4;
-            for (int i = 0, tt = t0; tt < t1 && ok; ++i, ++tt) {
-                const int s = i % kBsStages;
-                if (i >= kBsStages) ok = tc::mbar_wait(empty(s), ((i / kBsStages) & 1) ^ 1, abort_flag);
-                if (!ok) break;
-                const uint32_t st = ring + s * kBsStage;
-                const int n0 = tt * kBsRows;
-                tc::mbar_expect_tx(full(s), kBsPacked + cbytes + 2 * Mb * 128);
+        uint2 cw[4];        // DQ: the 8 codes of rows 4l + j in this slice
+        float sf[4], smu[4];   // DQ: their second-level step (and group mean)
+        float4 am[4][2];    // fp32 absmax of rows 4l + j
+        auto fetch = [&](int64_t u) {
+            const int64_t kz = u / ntn, n0 = (u % ntn) * kBsRows;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t n = n0 + 4 * lane + j;
+                const bool okr = n < Dout;
+                const int64_t b0 = n * nbr + 8 * kz;
+                if (DQ) {
+                    // 8 | nbr: the slice's 8 blocks start 8-aligned, inside one group of 256
+                    cw[j] = okr ? __ldg(reinterpret_cast<const uint2 *>(sc.code + b0)) : make_uint2(0u, 0u);
+                    sf[j] = okr ? __ldg(sc.step + (b0 >> 8)) : 0.f;
+                    smu[j] = okr && sc.dq == QLORA_DQ_MEAN ? __ldg(sc.mean + (b0 >> 8)) : 0.f;
+                } else {
+                    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 *p = reinterpret_cast<const float4 *>(sc.absmax + b0);
+                    am[j][0] = okr ? __ldg(p) : z4;
+                    am[j][1] = (okr && 8 * kz + 4 < nbr) ? __ldg(p + 1) : z4;
+                }
+            }
+        };
+        int64_t i = 0;
+        if (u0 < u1) fetch(u0);
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int s = (int)(i % kBsStages);
+            if (i >= kBsStages)
+                ok = __all_sync(0xffffffffu, tc::mbar_wait(empty(s), (int)((i / kBsStages) & 1) ^ 1, abort_flag));
+            if (!ok) break;
+            const int kz = (int)(u / ntn), n0 = (int)(u % ntn) * kBsRows;
+            const uint32_t st = ring + s * kBsStage;
+            if (lane == 0) {
+                tc::mbar_expect_tx_only(full(s), kBsPacked + 2 * Mb * 128);
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
                     tc::tma_load_2d(st + q * (kBsRows * 128), &tmP, kz * (kBsCols / 2) + 128 * q, n0, full(s));
-                if (sc.dq)   // 16 codes per row from the 16-aligned start; this slice's 8 at 8 * (kz % 2)
-                    tc::tma_load_2d(st + kBsPacked, &tmC, 16 * (kz >> 1), n0, full(s));
-                else
-                    tc::tma_load_2d(st + kBsPacked, &tmC, 8 * kz, n0, full(s));
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
-                    tc::tma_load_2d(st + kBsPacked + kBsScale + q * 2048, &tmD, n0 + 64 * q, 0, full(s));
+                    tc::tma_load_2d(st + kBsPacked + q * 2048, &tmD, n0 + 64 * q, 0, full(s));
             }
-            if (!ok) *abort_flag = 1;
+            uint8_t *ah = gring + s * kBsStage + kBsPacked + kBsDy;
+#pragma unroll
+            for (int kb = 0; kb < 8; ++kb) {
+                float v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (DQ) {
+                        const uint32_t word = kb < 4 ? cw[j].x : cw[j].y;
+                        v[j] = dq_decode((word >> (8 * (kb & 3))) & 0xffu, sf[j], smu[j], sc.dq);
+                    } else {
+                        const float4 a = am[j][kb >> 2];
+                        v[j] = (kb & 3) == 0 ? a.x : (kb & 3) == 1 ? a.y : (kb & 3) == 2 ? a.z : a.w;
+                    }
+                }
+                *reinterpret_cast<float4 *>(ah + kb * (kBsRows * 4) + 16 * lane) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+            }
+            tc::mbar_arrive(full(s));
+            if (u + 1 < u1) fetch(u + 1);
         }
+        if (!ok && lane == 0) *abort_flag = 1;
     } else {
         // ---------------------------------------------------------- compute warps
         const uint32_t lanebits = 4u * lane;
@@ -767,111 +877,157 @@ k_gemv_bwd_stream(const __grid_constant__ CUtensorMap tmP, const __grid_constant
             return *reinterpret_cast<const uint32_t *>(lutb + off);
         };
         const int kb = warp & 7, qpar = warp >> 3;
+        // stage offsets of this lane's data; group q = 2 qq + qpar adds qq * 4096
+        // (packed), qq * 128 (a_hat) and, for dY, box qq / 2 and chunk 4 (qq % 2)
+        int pko[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int chunk = 2 * (kb & 3) + (g >> 2);
+            pko[j] = (kb >> 2) * (kBsRows * 128) + (16 * qpar + 4 * t + j) * 128 +
+                     ((chunk ^ ((4 * t + j) & 7)) << 4) + 4 * (g & 3);
+        }
+        const int aho = kBsPacked + kBsDy + (kb * kBsRows + 16 * qpar + 4 * t) * 4;
+        int dyo[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            dyo[h] = kBsPacked + g * 128 + (((4 * h + 2 * qpar + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
+        const bool tok0 = g < M, tok1 = g + 8 < M;
+
         float acc[8][4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
-        for (int i = 0, tt = t0; tt < t1; ++i, ++tt) {
-            const int s = i % kBsStages;
-            if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (i / kBsStages) & 1, abort_flag));
-            if (!ok) {
-                *abort_flag = 1;
-                break;   // no CTA-wide barrier inside this loop
-            }
-            const uint8_t *stg = gring + s * kBsStage;
-            const int64_t n0 = (int64_t)tt * kBsRows;
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int q = 2 * qq + qpar;                 // 16-row group of the tile
-                float ah[4];
-                uint32_t R[4][4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int rl = 16 * q + 4 * t + j;       // tile row
-                    const int64_t n = n0 + rl;
-                    // packed word: bytes 32 kb + 4 g .. + 3 of the tile row (box kb / 4)
-                    const int chunk = 2 * (kb & 3) + (g >> 2);
-                    const uint32_t word = *reinterpret_cast<const uint32_t *>(
-                        stg + (kb >> 2) * (kBsRows * 128) + rl * 128 + ((chunk ^ (rl & 7)) << 4) + 4 * (g & 3));
-                    float a = 0.f;
-                    if (n < Dout) {
-                        if (sc.dq) {
-                            const uint8_t code = stg[kBsPacked + rl * 16 + 8 * (kz & 1) + kb];
-                            // the slice's blocks of row n lie in one double-quant group
-                            const float step = __ldg(sc.step + (((uint32_t)n * (uint32_t)nbr +
-                                                                 16u * (uint32_t)(kz >> 1)) >> 8));
-                            a = __fmul_rn((float)code, step);
-                        } else {
-                            a = reinterpret_cast<const float *>(stg + kBsPacked)[rl * 8 + kb];
-                        }
-                    }
-                    ah[j] = a;
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) R[j][p] = lookup(word, p);
-                }
-                // A fragments: dY[token][row] * a_hat[row] as hi + lo bf16; rows 4t..4t+3
-                // of the group are K slots 2t, 2t+1 (reg 0/1) and 2t+8, 2t+9 (reg 2/3)
-                uint32_t ahi[4], alo[4];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {            // token g (h = 0) or g + 8
-                    const int m = g + 8 * h;
-                    const int nn = 16 * q + 4 * t;          // tile row of j = 0 (column of dY)
-                    const uint8_t *dyb = stg + kBsPacked + kBsScale + (nn >> 6) * 2048 + m * 128;
-                    const int cch = (nn & 63) >> 3;         // 16-byte chunk, 4 rows = 8 bytes
-                    const uint2 dv = *reinterpret_cast<const uint2 *>(dyb + ((cch ^ (m & 7)) << 4) + 2 * (nn & 7));
-                    const float d0 = bf16_lo(dv.x) * ah[0], d1 = bf16_hi(dv.x) * ah[1];
-                    const float d2 = bf16_lo(dv.y) * ah[2], d3 = bf16_hi(dv.y) * ah[3];
-                    const uint32_t h01 = bf16x2_bits(d0, d1), h23 = bf16x2_bits(d2, d3);
-                    ahi[h] = h01;
-                    ahi[2 + h] = h23;
-                    alo[h] = bf16x2_bits(d0 - bf16_lo(h01), d1 - bf16_hi(h01));
-                    alo[2 + h] = bf16x2_bits(d2 - bf16_lo(h23), d3 - bf16_hi(h23));
-                }
+        auto flush = [&](int64_t kz) {
+            if (MT == 1) {   // rows g + 8 hold the lo terms of tokens g
 #pragma unroll
                 for (int ii = 0; ii < 8; ++ii) {
-                    const uint32_t sel = (ii & 1) ? 0x7632u : 0x5410u;
-                    const uint32_t b[2] = {__byte_perm(R[0][ii >> 1], R[1][ii >> 1], sel),
-                                           __byte_perm(R[2][ii >> 1], R[3][ii >> 1], sel)};
-                    mma_bf16_16816(acc[ii], ahi, b);
-                    mma_bf16_16816(acc[ii], alo, b);
+                    acc[ii][0] += acc[ii][2];
+                    acc[ii][1] += acc[ii][3];
+                    acc[ii][2] = acc[ii][3] = 0.f;
+                }
+            }
+            // warps w + 8 hand their sums to warps w, which write the slot; acc[ii]
+            // holds (token g, input 16t + ii), (g, 16t + 8 + ii), (g + 8, 16t + ii),
+            // (g + 8, 16t + 8 + ii) of block kb
+            float *rb = red + (kb * 32 + lane) * 32;
+            asm volatile("bar.sync 1, %0;\n" ::"n"(16 * 32));   // red free
+            if (qpar) {
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii)
+                    *reinterpret_cast<float4 *>(rb + 4 * ii) =
+                        make_float4(acc[ii][0], acc[ii][1], acc[ii][2], acc[ii][3]);
+            }
+            asm volatile("bar.sync 1, %0;\n" ::"n"(16 * 32));
+            if (!qpar && ok) {
+                const int64_t slot = c - unit_owner(kz * ntn, G, T);
+                float *pp = partial + (kz * nslot + slot) * (int64_t)M * kBsCols;
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii) {
+                    const float4 o = *reinterpret_cast<const float4 *>(rb + 4 * ii);
+                    const float v[4] = {acc[ii][0] + o.x, acc[ii][1] + o.y, acc[ii][2] + o.z,
+                                        acc[ii][3] + o.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = g + 8 * (e >> 1);
+                        const int kk = 64 * kb + 16 * t + 8 * (e & 1) + ii;
+                        if (m < M && kz * kBsCols + kk < Din) pp[(int64_t)m * kBsCols + kk] = v[e];
+                    }
+                }
+            }
+        };
+
+        int64_t cur = -1;
+        int64_t i = 0;
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int64_t kz = u / ntn;
+            if (kz != cur) {
+                if (cur >= 0) flush(cur);
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[ii][e] = 0.f;
+                cur = kz;
+            }
+            const int s = (int)(i % kBsStages);
+            if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(full(s), (int)((i / kBsStages) & 1), abort_flag));
+            if (!ok) {
+                // keep walking, without work, so that every warp meets the flush barriers
+                if (lane == 0) *abort_flag = 1;
+                continue;
+            }
+            const uint8_t *stg = gring + s * kBsStage;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const float4 ah = *reinterpret_cast<const float4 *>(stg + aho + qq * 128);
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const uint32_t *>(stg + pko[j] + qq * 4096);
+                // A: d = dY[token][rows 4t..4t+3] * a_hat as hi + lo bf16 pairs
+                // (hi = RN_bf16(d), lo = RN_bf16(d - hi)); rows 4t, 4t+1 in reg 0/1,
+                // 4t+2, 4t+3 in reg 2/3.  With M <= 8 the lo terms take the empty
+                // token rows g + 8 of the same MMA; else a second MMA carries them.
+                uint32_t a[4], alo[4];
+                {
+                    const uint8_t *d0 = stg + dyo[qq & 1] + (qq >> 1) * 2048;
+                    const uint2 v0 = tok0 ? *reinterpret_cast<const uint2 *>(d0) : make_uint2(0u, 0u);
+                    split_scaled<F16>(v0.x, ah.x, ah.y, a[0], alo[0]);
+                    split_scaled<F16>(v0.y, ah.z, ah.w, a[2], alo[2]);
+                    if (MT == 2) {
+                        const uint2 v1 = tok1 ? *reinterpret_cast<const uint2 *>(d0 + 1024) : make_uint2(0u, 0u);
+                        split_scaled<F16>(v1.x, ah.x, ah.y, a[1], alo[1]);
+                        split_scaled<F16>(v1.y, ah.z, ah.w, a[3], alo[3]);
+                    } else {
+                        a[1] = alo[0];
+                        a[3] = alo[2];
+                    }
+                }
+                // B: byte p of e01 holds input 8g + 2p of rows 4t (high nibble) and
+                // 4t + 1 (low nibble); o01 the same for input 8g + 2p + 1
+                const uint32_t e01 = (w[0] & 0xF0F0F0F0u) | ((w[1] >> 4) & 0x0F0F0F0Fu);
+                const uint32_t o01 = ((w[0] << 4) & 0xF0F0F0F0u) | (w[1] & 0x0F0F0F0Fu);
+                const uint32_t e23 = (w[2] & 0xF0F0F0F0u) | ((w[3] >> 4) & 0x0F0F0F0Fu);
+                const uint32_t o23 = ((w[2] << 4) & 0xF0F0F0F0u) | (w[3] & 0x0F0F0F0Fu);
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii) {
+                    const uint32_t b[2] = {lookup((ii & 1) ? o01 : e01, ii >> 1),
+                                           lookup((ii & 1) ? o23 : e23, ii >> 1)};
+                    mma16816<F16>(acc[ii], a, b);
+                    if (MT == 2) mma16816<F16>(acc[ii], alo, b);
                 }
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(empty(s));
         }
-        // warps w + 8 hand their sums to warps w; columns: acc[ii] holds (token g,
-        // input 16t + ii), (g, 16t + 8 + ii), (g + 8, 16t + ii), (g + 8, 16t + 8 + ii)
-        float *rb = red + (kb * 32 + lane) * 32;
-        if (qpar) {
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii)
-                *reinterpret_cast<float4 *>(rb + 4 * ii) = make_float4(acc[ii][0], acc[ii][1], acc[ii][2], acc[ii][3]);
-        }
-        asm volatile("bar.sync 1, %0;\n" ::"n"(16 * 32));
-        if (!qpar && ok) {
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii) {
-                const float4 o = *reinterpret_cast<const float4 *>(rb + 4 * ii);
-                const float v[4] = {acc[ii][0] + o.x, acc[ii][1] + o.y, acc[ii][2] + o.z, acc[ii][3] + o.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = g + 8 * (e >> 1);
-                    const int64_t k = (int64_t)kz * kBsCols + 64 * kb + 16 * t + 8 * (e & 1) + ii;
-                    if (m < M && k < Din) partial[((int64_t)sp * M + m) * Din + k] = v[e];
-                }
-            }
-        }
+        if (cur >= 0) flush(cur);
     }
     if (!ok && status) atomicOr(status, QLORA_STATUS_TIMEOUT);
     __syncwarp();
     __syncthreads();
 }
 
-__global__ void k_gemv_bwd_finalize(const float *__restrict__ partial, int nsplit, int M,
-                                    int64_t Din, const float *__restrict__ G,
+// dX[m, k] = sum over the slots of slice k / 512 of partial + (s / g) G[m, :] A[k / g, :]^T
+__global__ void k_gemv_bwd_finalize(const float *__restrict__ partial, int ntn, int nkz, int Gc,
+                                    int nslot, int M, int64_t Din, const float *__restrict__ G,
                                     const uint16_t *__restrict__ Al, int r, int pool, float s,
-                                    uint16_t *__restrict__ dX) {
+                                    uint16_t *__restrict__ dX, bool f16) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)M * Din) return;
+    const int m = (int)(i / Din);
+    const int64_t k = i % Din;
+    const int64_t kz = k / kBsCols, kk = k % kBsCols;
+    const int64_t T = (int64_t)nkz * ntn;
+    const int64_t c0 = unit_owner(kz * ntn, Gc, T), c1 = unit_owner(kz * ntn + ntn - 1, Gc, T);
+    float v = 0.f;
+    for (int64_t sl = 0; sl <= c1 - c0; ++sl) v += partial[((kz * nslot + sl) * M + m) * kBsCols + kk];
+    float ad = 0.f;
+    const int64_t ka = k / pool;
+    for (int j = 0; j < r; ++j)
+        ad = fmaf(G[m * r + j], dec16(Al[ka * r + j], f16), ad);
+    dX[i] = enc16(fmaf(s / pool, ad, v), f16);
+}
+
+// dX[m, k] = sum over nsplit partials [nsplit][M][Din] + the adapter term (register kernel)
+__global__ void k_gemv_bwd_finalize_split(const float *__restrict__ partial, int nsplit, int M,
+                                          int64_t Din, const float *__restrict__ G,
+                                          const uint16_t *__restrict__ Al, int r, int pool, float s,
+                                          uint16_t *__restrict__ dX, bool f16) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)M * Din) return;
     const int m = (int)(i / Din);
@@ -881,8 +1037,8 @@ __global__ void k_gemv_bwd_finalize(const float *__restrict__ partial, int nspli
     float ad = 0.f;
     const int64_t ka = k / pool;
     for (int j = 0; j < r; ++j)
-        ad = fmaf(G[m * r + j], __bfloat162float(__ushort_as_bfloat16(Al[ka * r + j])), ad);
-    dX[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(s / pool, ad, v)));
+        ad = fmaf(G[m * r + j], dec16(Al[ka * r + j], f16), ad);
+    dX[i] = enc16(fmaf(s / pool, ad, v), f16);
 }
 
 }  // namespace
@@ -892,21 +1048,32 @@ size_t gemv_fwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     return (size_t)nsplit * M * Dout * sizeof(float);
 }
 
-// splits of the streamed backward: at most one CTA per SM over the slices
-// (one CTA fits on an SM; a second wave would double the time)
-static int bwd_stream_splits(int64_t Din, int64_t Dout) {
-    const int64_t nkz = (Din + kBsCols - 1) / kBsCols, ntn = (Dout + kBsRows - 1) / kBsRows;
-    int64_t ns = device_sms() / nkz;
-    if (ns > ntn) ns = ntn;
-    return (int)(ns < 1 ? 1 : ns);
+// Grid of the streamed backward: one CTA per SM (one fits) over the
+// T = nkz * ntn units, and the most CTAs that share one slice (its slots).
+struct BwdPlan {
+    int nkz, ntn, G, nslot;
+};
+static BwdPlan bwd_plan(int64_t Din, int64_t Dout) {
+    BwdPlan p;
+    p.nkz = (int)((Din + kBsCols - 1) / kBsCols);
+    p.ntn = (int)((Dout + kBsRows - 1) / kBsRows);
+    const int64_t T = (int64_t)p.nkz * p.ntn;
+    p.G = (int)(T < device_sms() ? T : device_sms());
+    int64_t mx = 1;
+    for (int64_t kz = 0; kz < p.nkz; ++kz) {
+        const int64_t d = unit_owner(kz * p.ntn + p.ntn - 1, p.G, T) - unit_owner(kz * p.ntn, p.G, T) + 1;
+        if (d > mx) mx = d;
+    }
+    p.nslot = (int)mx;
+    return p;
 }
 
 size_t gemv_bwd_partial_bytes(int M, int64_t Din, int64_t Dout) {
     const int64_t NS = kGemvWarps * kBwdRowsPerWarp;
-    int64_t nsplit = (Dout + NS - 1) / NS;
-    const int64_t ns2 = bwd_stream_splits(Din, Dout);   // the streamed kernel always writes partials
-    if (ns2 > nsplit) nsplit = ns2;
-    return (size_t)nsplit * M * Din * sizeof(float);
+    const size_t split = (size_t)((Dout + NS - 1) / NS) * M * Din * sizeof(float);
+    const BwdPlan p = bwd_plan(Din, Dout);
+    const size_t slots = (size_t)p.nkz * p.nslot * M * kBsCols * sizeof(float);
+    return split > slots ? split : slots;
 }
 
 size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r) {
@@ -920,121 +1087,114 @@ size_t gemv_fwd_tpart_floats(int M, int64_t Din, int r) {
 // enqueued.  Without Aad, T is the finished adapter-down product.
 int launch_gemv_fwd(const uint16_t *X, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *T, const uint16_t *Bl, int r, float s, uint16_t *Y,
-                    float *partial, uint32_t *d_status, cudaStream_t st, const uint16_t *Aad,
+                    float *partial, uint32_t *d_status, cudaStream_t st, bool f16, const uint16_t *Aad,
                     float *Tpart, float *T_out) {
     const int64_t Din = q.cols, Dout = q.rows;
-    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    const ScaleSrc sc = scale_src(q);
     const int64_t nsplit = (Din + kFwdKS - 1) / kFwdKS;
     const int64_t nbr = Din / 64;
-    // streamed kernel: scale rows must be TMA-tileable (row pitch a multiple
-    // of 16 bytes) and the weight at least one slice wide; else the register kernel
-    bool stream = Din >= kFwdKS && (q.double_quant ? (nbr % 16 == 0) : (nbr % 4 == 0));
-    CUtensorMap tmP, tmC;
-    if (stream) {
+    // streamed kernel: the weight at least one slice wide; the producer reads a
+    // row's 8 scale codes of a half-tile as one aligned 8-byte word (8 | Din/64),
+    // or its fp32 absmax as 16-byte words (4 | Din/64); else the register kernel
+    bool stream = Din >= kFwdKS &&
+                  (q.double_quant ? (nbr % 8 == 0 && (reinterpret_cast<uintptr_t>(q.absmax_code) & 7) == 0)
+                                  : (nbr % 4 == 0 && (reinterpret_cast<uintptr_t>(q.absmax) & 15) == 0));
+    CUtensorMap tmP;
+    if (stream)
         stream = tc::make_map(&tmP, q.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Din / 2, Dout, Din / 2,
                               128, kStRows, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (q.double_quant)
-            stream = stream && tc::make_map(&tmC, q.absmax_code, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nbr,
-                                            Dout, nbr, 16, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-        else
-            stream = stream && tc::make_map(&tmC, q.absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, nbr,
-                                            Dout, nbr * 4, 8, kStRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-    }
     if (Aad && !stream) return QLORA_EUNSUPPORTED;
-    prof_begin(kProfGemv, st);
     if (stream) {
         const int ntr = (int)((Dout + kStRows - 1) / kStRows);
         const int ntiles = (int)(ntr * nsplit);
         const int grid = ntiles < device_sms() ? ntiles : device_sms();
-        if (M <= 8) {
-            cudaFuncSetAttribute(k_gemv_fwd_stream<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
-            k_gemv_fwd_stream<1><<<grid, kStThreads, kStSmem, st>>>(
-                tmP, tmC, X, M, Din, Dout, sc, cb, ntr, ntiles, partial, Aad, r, Tpart, d_status);
-        } else {
-            cudaFuncSetAttribute(k_gemv_fwd_stream<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStSmem);
-            k_gemv_fwd_stream<2><<<grid, kStThreads, kStSmem, st>>>(
-                tmP, tmC, X, M, Din, Dout, sc, cb, ntr, ntiles, partial, Aad, r, Tpart, d_status);
-        }
+        auto kern = f16 ? (q.double_quant ? (M > 8 ? k_gemv_fwd_stream<true, 2, true> : k_gemv_fwd_stream<true, 1, true>)
+                                          : (M > 8 ? k_gemv_fwd_stream<false, 2, true> : k_gemv_fwd_stream<false, 1, true>))
+                        : (q.double_quant ? (M > 8 ? k_gemv_fwd_stream<true, 2, false> : k_gemv_fwd_stream<true, 1, false>)
+                                          : (M > 8 ? k_gemv_fwd_stream<false, 2, false> : k_gemv_fwd_stream<false, 1, false>));
+        if (set_max_smem(reinterpret_cast<const void *>(kern), kStSmem) != cudaSuccess) return QLORA_ECUDA;
+        prof_begin(kProfGemv, st);
+        kern<<<grid, kStThreads, kStSmem, st>>>(tmP, X, M, Din, Dout, sc, cb, ntr, ntiles, partial, Aad, r,
+                                                Tpart, d_status);
     } else {
-        const size_t smem = 256 * 32 * 4 + 16 * (kFwdKS + 8) * 2;   // pair table + x slice
+        const int smem = 256 * 32 * 4 + 16 * (kFwdKS + 8) * 2;   // pair table + x slice
         dim3 grid((unsigned)((Dout + kFwdRows - 1) / kFwdRows), (unsigned)nsplit);
-        if (M <= 8) {
-            cudaFuncSetAttribute(k_gemv_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            k_gemv_fwd<1><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
-        } else {
-            cudaFuncSetAttribute(k_gemv_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            k_gemv_fwd<2><<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
-        }
+        auto kern = f16 ? (M <= 8 ? k_gemv_fwd<1, true> : k_gemv_fwd<2, true>)
+                        : (M <= 8 ? k_gemv_fwd<1, false> : k_gemv_fwd<2, false>);
+        if (set_max_smem(reinterpret_cast<const void *>(kern), smem) != cudaSuccess) return QLORA_ECUDA;
+        prof_begin(kProfGemv, st);
+        kern<<<grid, kGemvWarps * 32, smem, st>>>(X, M, Din, Dout, q.packed, sc, cb, partial);
     }
     prof_end(kProfGemv, st);
     QLORA_LAUNCH_CHECK();
     if (Aad) {
         dim3 fg((unsigned)((Dout + 255) / 256), (unsigned)M);
         k_gemv_fwd_finalize_fused<<<fg, 256, 0, st>>>(partial, (int)nsplit, M, Dout, Tpart, r, Bl, s, Y,
-                                                     T_out);
+                                                     T_out, f16);
         QLORA_LAUNCH_CHECK();
         return QLORA_OK;
     }
     const int64_t n = (int64_t)M * Dout;
     k_gemv_fwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, (int)nsplit, M, Dout,
-                                                                     T, Bl, r, s, Y);
+                                                                     T, Bl, r, s, Y, f16);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
 }
 
 int launch_gemv_bwd(const uint16_t *dY, int M, const nf4_weight_t &q, const Codebook &cb,
                     const float *G, const uint16_t *Al, int r, int pool, float s, uint16_t *dX,
-                    float *partial, cudaStream_t st) {
+                    float *partial, cudaStream_t st, bool f16) {
     const int64_t Din = q.cols, Dout = q.rows;
-    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
-    // streamed kernel: scale rows TMA-tileable, at least one 512-input slice and one 128-row tile
+    const ScaleSrc sc = scale_src(q);
+    // streamed kernel: at least one 512-input slice and one 128-row tile; the
+    // producer reads a row's 8 scale codes of a slice as one aligned 8-byte
+    // word (8 | Din/64), or its fp32 absmax as 16-byte words (4 | Din/64)
     const int64_t nbr = Din / 64;
-    bool stream = Din >= kBsCols && Dout >= kBsRows && Dout * nbr < (int64_t(1) << 32) &&
-                  (q.double_quant ? (nbr % 16 == 0) : (nbr % 4 == 0));
-    CUtensorMap tmP, tmC, tmD;
+    bool stream = Din >= kBsCols && Dout >= kBsRows &&
+                  (q.double_quant ? (nbr % 8 == 0 && (reinterpret_cast<uintptr_t>(q.absmax_code) & 7) == 0)
+                                  : (nbr % 4 == 0 && (reinterpret_cast<uintptr_t>(q.absmax) & 15) == 0));
+    CUtensorMap tmP, tmD;
     const int Mb = M < 16 ? M : 16;
     if (stream) {
         stream = tc::make_map(&tmP, q.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Din / 2, Dout, Din / 2,
                               128, kBsRows, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (q.double_quant)
-            stream = stream && tc::make_map(&tmC, q.absmax_code, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nbr,
-                                            Dout, nbr, 16, kBsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-        else
-            stream = stream && tc::make_map(&tmC, q.absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, nbr,
-                                            Dout, nbr * 4, 8, kBsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         stream = stream && tc::make_map(&tmD, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dout, M, Dout * 2,
                                         64, Mb, CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (stream) {
-        const int nkz = (int)((Din + kBsCols - 1) / kBsCols), ntn = (int)((Dout + kBsRows - 1) / kBsRows);
-        const int nsplit = bwd_stream_splits(Din, Dout);
-        cudaFuncSetAttribute(k_gemv_bwd_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmem);
+        const BwdPlan p = bwd_plan(Din, Dout);
+        auto kern = f16 ? (q.double_quant ? (M > 8 ? k_gemv_bwd_stream<true, 2, true> : k_gemv_bwd_stream<true, 1, true>)
+                                          : (M > 8 ? k_gemv_bwd_stream<false, 2, true> : k_gemv_bwd_stream<false, 1, true>))
+                        : (q.double_quant ? (M > 8 ? k_gemv_bwd_stream<true, 2, false> : k_gemv_bwd_stream<true, 1, false>)
+                                          : (M > 8 ? k_gemv_bwd_stream<false, 2, false> : k_gemv_bwd_stream<false, 1, false>));
+        if (set_max_smem(reinterpret_cast<const void *>(kern), kBsSmem) != cudaSuccess) return QLORA_ECUDA;
         prof_begin(kProfGemv, st);
-        k_gemv_bwd_stream<<<dim3((unsigned)nkz, (unsigned)nsplit), kBsThreads, kBsSmem, st>>>(
-            tmP, tmC, tmD, M, Mb, Din, Dout, sc, cb, ntn, nsplit, partial, nullptr);
+        kern<<<(unsigned)p.G, kBsThreads, kBsSmem, st>>>(tmP, tmD, M, Mb, Din, Dout, sc, cb, p.ntn, p.nkz,
+                                                         p.nslot, partial, nullptr);
         prof_end(kProfGemv, st);
         QLORA_LAUNCH_CHECK();
         const int64_t n = (int64_t)M * Din;
-        k_gemv_bwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, nsplit, M, Din, G,
-                                                                         Al, r, pool, s, dX);
+        k_gemv_bwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            partial, p.ntn, p.nkz, p.G, p.nslot, M, Din, G, Al, r, pool, s, dX, f16);
         QLORA_LAUNCH_CHECK();
         return QLORA_OK;
     }
     constexpr int NS = kGemvWarps * kBwdRowsPerWarp;
     const int64_t nsplit = (Dout + NS - 1) / NS;
-    const size_t smem = 16 * (NS + 8) * 2 + kGemvWarps * 16 * 64 * 4;
-    cudaFuncSetAttribute(k_gemv_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int smem = 16 * (NS + 8) * 2 + kGemvWarps * 16 * 64 * 4;
+    auto kbr = f16 ? k_gemv_bwd<true> : k_gemv_bwd<false>;
+    if (set_max_smem(reinterpret_cast<const void *>(kbr), smem) != cudaSuccess) return QLORA_ECUDA;
     dim3 grid((unsigned)(Din / 64), (unsigned)nsplit);
     prof_begin(kProfGemv, st);
-    k_gemv_bwd<<<grid, kGemvWarps * 32, smem, st>>>(dY, M, Din, Dout, q.packed, sc, cb,
+    kbr<<<grid, kGemvWarps * 32, smem, st>>>(dY, M, Din, Dout, q.packed, sc, cb,
                                                     nsplit > 1 ? partial : nullptr, G, Al, r,
                                                     pool, s, dX);
     prof_end(kProfGemv, st);
     QLORA_LAUNCH_CHECK();
     if (nsplit > 1) {
         const int64_t n = (int64_t)M * Din;
-        k_gemv_bwd_finalize<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, (int)nsplit, M,
-                                                                         Din, G, Al, r, pool, s, dX);
+        k_gemv_bwd_finalize_split<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, (int)nsplit, M,
+                                                                               Din, G, Al, r, pool, s, dX, f16);
         QLORA_LAUNCH_CHECK();
     }
     return QLORA_OK;

@@ -1,12 +1,14 @@
-// merge.cu -- adapter merge for deployment: the bf16 weight with the LoRA
-// update folded in, W_eff = dequant(W4) + (alpha/r) A B, stored [Dout, Din]
+// merge.cu -- adapter merge for deployment: the weight with the LoRA update
+// folded in, W_eff = dequant(W4) + (alpha/r) A B, stored [Dout, Din] in the
+// compute dtype (bf16, or fp16)
 // ("从 LoRA 到 QLoRA、QA-LoRA" section 2, W_eff; bitsandbytes article (CSDN)
 // 12.10, merging the adapter before deployment; pooled adapter: every input
 // of a group shares (A_p B)/g, same blog section 5).
 //
-//   W_out[n][k] = RN_bf16( w_hat[n][k] + (s/g) sum_j A[k/g][j] B[j][n] )
+//   W_out[n][k] = RN_dt( w_hat[n][k] + (s/g) sum_j A[k/g][j] B[j][n] )
 //
-// w_hat = RN_bf16(RN32(a_hat c_q)) is the dequantized weight; the rank-r sum
+// w_hat = RN_dt(RN32(a_hat c_q)) is the dequantized weight in the compute
+// dtype dt; the rank-r sum
 // is an fp32 MMA.  HBM-bound: 0.52 bytes in and 2 bytes out per weight.
 //
 // Persistent: one CTA of 16 warps per SM walks a contiguous range of units,
@@ -50,17 +52,19 @@ struct MgRow {
     uint2 p;
     uint32_t code;
     float f;
+    float mu;      // group mean (mean-offset double quantization)
 };
 
 __device__ __forceinline__ MgRow mg_load(const uint8_t *__restrict__ packed, const ScaleSrc &sc,
                                          int64_t row, int64_t Dout, int64_t Din, int64_t kc, int t) {
-    MgRow m{make_uint2(0u, 0u), 0u, 0.f};
+    MgRow m{make_uint2(0u, 0u), 0u, 0.f, 0.f};
     if (row < Dout) {
         m.p = __ldg(reinterpret_cast<const uint2 *>(packed + row * (Din / 2) + kc / 2) + t);
         const int64_t b = row * (Din / 64) + kc / 64;
         if (sc.dq) {
             m.code = __ldg(sc.code + b);
             m.f = __ldg(sc.step + (b >> 8));
+            if (sc.dq == QLORA_DQ_MEAN) m.mu = __ldg(sc.mean + (b >> 8));
         } else {
             m.code = 1u;
             m.f = __ldg(sc.absmax + b);
@@ -122,6 +126,7 @@ __device__ __forceinline__ void mg_stage_a(uint16_t *sA, const uint16_t *__restr
     cp_async_commit();
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(kMgThreads, 1)
 k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
         const uint16_t *__restrict__ A, const uint16_t *__restrict__ B, int r, int gp, float sg,
@@ -218,8 +223,8 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
                 uint32_t b4[4];
                 ldmatrix_x4(b4, sAc + ldb + np * ldb_np + ks);
                 const uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
-                mma_bf16_16816(acc[2 * np], a, b0);
-                mma_bf16_16816(acc[2 * np + 1], a, b1);
+                mma16816<F16>(acc[2 * np], a, b0);
+                mma16816<F16>(acc[2 * np + 1], a, b1);
             }
         }
         // epilogue: row ra (hr 0) / ra + 8 (hr 1), inputs kc + 16t + 2nt, +1 = byte 8t + nt
@@ -228,14 +233,15 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
             const int64_t row = ra + 8 * hr;
             if (row >= Dout) continue;
             const MgRow m = hr ? cur1 : cur0;
-            const float ah = __fmul_rn((float)m.code, m.f);
+            const float ah = sc.dq ? dq_decode(m.code, m.f, m.mu, sc.dq) : m.f;
             uint32_t o[8];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const uint32_t byte = ((nt < 4 ? m.p.x : m.p.y) >> (8 * (nt & 3))) & 0xffu;
-                // both weights rounded to bf16 by one paired conversion
-                const uint32_t w = bf16x2_bits(__fmul_rn(ah, cbs[byte >> 4]), __fmul_rn(ah, cbs[byte & 15]));
-                o[nt] = bf16x2_bits(fmaf(sg, acc[nt][2 * hr], bf16_lo(w)), fmaf(sg, acc[nt][2 * hr + 1], bf16_hi(w)));
+                // both weights rounded to the compute dtype by one paired conversion
+                const uint32_t w = pack2(__fmul_rn(ah, cbs[byte >> 4]), __fmul_rn(ah, cbs[byte & 15]), F16);
+                o[nt] = pack2(fmaf(sg, acc[nt][2 * hr], lo16(w, F16)), fmaf(sg, acc[nt][2 * hr + 1], hi16(w, F16)),
+                              F16);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(W_out + row * Din + kc + 16 * t);
             __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
@@ -255,17 +261,18 @@ size_t merge_smem_bytes(int r) {
 }
 
 int launch_merge(const nf4_weight_t &q, const Codebook &cb, const uint16_t *A, const uint16_t *B,
-                 int r, int gp, float s, uint16_t *W_out, cudaStream_t st) {
+                 int r, int gp, float s, uint16_t *W_out, cudaStream_t st, bool f16) {
     const int64_t Dout = q.rows, Din = q.cols;
     if (Dout * Din == 0) return QLORA_OK;
-    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    const ScaleSrc sc = scale_src(q);
     const size_t smem = merge_smem_bytes(r);
     const int nbuf = smem == mg_smem(r, 3) ? 3 : 2;
-    cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = f16 ? k_merge<true> : k_merge<false>;
+    if (set_max_smem(reinterpret_cast<const void *>(kern), (int)smem) != cudaSuccess) return QLORA_ECUDA;
     const int64_t units = (Dout + kMgRows - 1) / kMgRows * (Din / 64);
     const unsigned grid = (unsigned)(units < device_sms() ? units : device_sms());
     prof_begin(kProfMerge, st);
-    k_merge<<<grid, kMgThreads, smem, st>>>(q.packed, sc, cb, A, B, r, gp, s / (float)gp, Dout, Din,
+    kern<<<grid, kMgThreads, smem, st>>>(q.packed, sc, cb, A, B, r, gp, s / (float)gp, Dout, Din,
                                             nbuf, W_out);
     prof_end(kProfMerge, st);
     QLORA_LAUNCH_CHECK();

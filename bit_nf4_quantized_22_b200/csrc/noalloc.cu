@@ -17,7 +17,9 @@ std::mutex g_mu;
 void *g_addr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached for the life of the process.
+// A cudaDeviceReset after that would leave the cached address stale; the
+// header states that resets are not supported once this entry point ran.
 int scratch_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ECUDA;

@@ -36,6 +36,19 @@ int device_sms() {
     return n;
 }
 
+cudaError_t set_max_smem(const void *fn, int bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<int, const void *>, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    std::lock_guard<std::mutex> lk(mu);
+    for (const auto &d : done)
+        if (d.first.first == dev && d.first.second == fn && d.second >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.push_back({{dev, fn}, bytes});
+    return e;
+}
+
 void prof_begin(int kind, cudaStream_t st) {
     if (!g_on.load(std::memory_order_relaxed)) return;
     std::lock_guard<std::mutex> lk(g_mu);

@@ -16,6 +16,17 @@ namespace {
 
 constexpr int kQuantThreads = 256;   // one thread per block, one CTA per DQ group
 
+// The levels whose midpoint is decision threshold j: (c_j, c_{j+1}), or,
+// where a level repeats (c_j == c_{j+1}, the FP4 table's -0 and +0), the next
+// pair of distinct levels, so that threshold j equals threshold j + 1 and
+// the repeated level's second copy is never chosen: the count of thresholds
+// below w is then the first nearest level, as with distinct levels.  With no
+// distinct pair above, both are +inf (a threshold never passed).
+struct ThreshPairs {
+    float lo[16];
+    float hi[16];
+};
+
 // Tables of the fast kernel: T[bin] for 32 bins, four bits each, and the
 // halved codebook midpoints h_k = (c_k + c_{k+1}) / 2 when each is exact in
 // fp64 with at most 29 significant bits (then h_k * a is exact in fp64).
@@ -69,28 +80,73 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return r;
 }
 
-// Double-quant code RNE(a / f) clamped to [0, 255].  For f in [2^-100, 2^100]:
-// an approximate quotient c (within one of the answer, as a / f <= 256 and
-// the approximation errs by < 2^-14), then the signs of a - (c +- 1/2) f
-// from one fma each -- a correctly rounded fma has the sign of the exact
-// value and is zero only when it is -- decide c - 1, c or c + 1, ties to
-// even.  Other f: the quotient in fp64, whose rint is exact for these ratios.
-__device__ __forceinline__ int dq_code(float a, float f) {
+// Double-quant code RNE(d / f) clamped to [-top, top] (d >= 0 for the
+// unsigned and signed absmax codes, either sign for the mean-offset code).
+// For f in [2^-100, 2^100]: an approximate quotient c (within one of the
+// answer, as |d / f| <= 256 and the approximation errs by < 2^-14), then the
+// signs of d - (c +- 1/2) f from one fma each -- a correctly rounded fma has
+// the sign of the exact value and is zero only when it is -- decide c - 1, c
+// or c + 1, ties to even.  Other f: the quotient in fp64, whose rint is exact
+// for these ratios of fp32 values.
+__device__ __forceinline__ int dq_code(float d, float f, int top) {
     if (!(f > 0.f)) return 0;
     float c;
     if (f >= 0x1p-100f && f <= 0x1p100f) {
-        c = rintf(__fmul_rn(a, rcp_approx(f)));
-        const float hi = fmaf(-(c + 0.5f), f, a);
-        const float lo = fmaf(-(c - 0.5f), f, a);
+        c = rintf(__fmul_rn(d, rcp_approx(f)));
+        const float hi = fmaf(-(c + 0.5f), f, d);
+        const float lo = fmaf(-(c - 0.5f), f, d);
         const bool odd = ((int)c & 1) != 0;
         if (hi > 0.f || (hi == 0.f && odd))
             c += 1.f;
         else if (lo < 0.f || (lo == 0.f && odd))
             c -= 1.f;
     } else {
-        c = (float)rint(__ddiv_rn((double)a, (double)f));
+        c = (float)rint(__ddiv_rn((double)d, (double)f));
     }
-    return (int)fminf(fmaxf(c, 0.f), 255.f);
+    return (int)fminf(fmaxf(c, -(float)top), (float)top);
+}
+
+// Double quantization of one group of first-level scales, one per thread of
+// the CTA (a, valid for the first nvalid threads): writes the step, the
+// codes and, for the mean-offset code, the group mean (the rules of
+// QLORA_DQ_U8 / _S8 / _MEAN in qlora.h).  s_a: the CTA's shared buffer of
+// kThreads floats; warp_max: kThreads / 32 floats; s_mu: one float.
+template <int kThreads>
+__device__ __forceinline__ void dq_group_encode(float a, bool valid, int nvalid, int dq, float *s_a,
+                                                float *warp_max, float *s_mu, uint8_t *code_out,
+                                                float *step_out, float *mean_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float v = valid ? a : 0.f, mu = 0.f;
+    if (dq == QLORA_DQ_MEAN) {
+        s_a[threadIdx.x] = v;
+        __syncthreads();
+        if (threadIdx.x == 0) {   // the fp64 sum in block order, then one division and one rounding
+            double sum = 0.0;
+            for (int i = 0; i < nvalid; ++i) sum = __dadd_rn(sum, (double)s_a[i]);
+            *s_mu = __double2float_rn(__ddiv_rn(sum, (double)nvalid));
+        }
+        __syncthreads();
+        mu = *s_mu;
+        v = valid ? fabsf(__fsub_rn(a, mu)) : 0.f;
+    }
+    float m = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) warp_max[warp] = m;
+    __syncthreads();
+    float gm = warp_max[0];
+#pragma unroll
+    for (int i = 1; i < kThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
+    const int top = dq == QLORA_DQ_U8 ? 255 : 127;
+    const float f = __fdiv_rn(gm, (float)top);
+    if (threadIdx.x == 0) {
+        *step_out = f;
+        if (dq == QLORA_DQ_MEAN) *mean_out = mu;
+    }
+    if (valid) {
+        const float d = dq == QLORA_DQ_MEAN ? __fsub_rn(a, mu) : a;
+        *code_out = (uint8_t)(int8_t)dq_code(d, f, top);
+    }
 }
 
 // One CTA per double-quant group of 256 blocks (64 KB of fp32 weights).
@@ -101,9 +157,9 @@ __device__ __forceinline__ int dq_code(float a, float f) {
 constexpr int kQuantSmem = 2 * 256 * 128 + 1024;
 
 __global__ void __launch_bounds__(kQuantThreads, 2)
-k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, int zero_idx,
+k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, ThreshPairs tp, int zero_idx,
                int dq, uint8_t *__restrict__ packed, float *__restrict__ absmax,
-               uint8_t *__restrict__ codes, float *__restrict__ steps,
+               uint8_t *__restrict__ codes, float *__restrict__ steps, float *__restrict__ means,
                uint32_t *__restrict__ status) {
     extern __shared__ __align__(1024) uint8_t qsm_raw[];
     __shared__ __align__(8) uint64_t bar_storage;
@@ -160,7 +216,7 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
         } else {
             float t[15];
 #pragma unroll
-            for (int j = 0; j < 15; ++j) t[j] = exact_threshold(cb.c[j], cb.c[j + 1], a);
+            for (int j = 0; j < 15; ++j) t[j] = exact_threshold(tp.lo[j], tp.hi[j], a);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 uint32_t word = 0;
@@ -180,28 +236,14 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, Codebook cb, 
     }
 
     if (dq) {
-        // group max over this CTA's 256 blocks (one double-quant group)
-        float m = a;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
-        __syncthreads();
-        float gm = warp_max[0];
-#pragma unroll
-        for (int i = 1; i < kQuantThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
-        const float f = __fdiv_rn(gm, 255.f);
-        if (threadIdx.x == 0) steps[blockIdx.x] = f;
-        if (valid) {
-            int code = 0;
-            if (f > 0.f) {
-                // a/f < 256 is a ratio of fp32 values: rint of the fp64
-                // quotient is round-half-even of the exact ratio.
-                double qd = rint(__ddiv_rn((double)a, (double)f));
-                qd = fmin(fmax(qd, 0.0), 255.0);
-                code = (int)qd;
-            }
-            codes[b] = (uint8_t)code;
-        }
+        __shared__ float s_grp[kQuantThreads];
+        __shared__ float s_mu;
+        const int nvalid = (int)(nb - (int64_t)blockIdx.x * kQuantThreads < kQuantThreads
+                                     ? nb - (int64_t)blockIdx.x * kQuantThreads : kQuantThreads);
+        uint8_t code = 0;
+        dq_group_encode<kQuantThreads>(a, valid, nvalid, dq, s_grp, warp_max, &s_mu, &code,
+                                       steps + blockIdx.x, means + blockIdx.x);
+        if (valid) codes[b] = code;
     }
 }
 
@@ -231,12 +273,12 @@ constexpr int kQfSmem = 0;
 // V weights per lane: 4 for blocks of 64, 2 for blocks of 32 (16 lanes per block either way).
 template <bool kExactHalf, int V>
 __global__ void __launch_bounds__(kQfThreads, 4)
-k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins,
+k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, QuantBins bins,
                     int zero_idx, int dq, uint8_t *__restrict__ packed,
                     float *__restrict__ absmax, uint8_t *__restrict__ codes,
-                    float *__restrict__ steps, uint32_t *__restrict__ status) {
+                    float *__restrict__ steps, float *__restrict__ means, uint32_t *__restrict__ status) {
     __shared__ float s_a[kQfThreads];
-    __shared__ float s_cb[16];
+    __shared__ float s_lo[16], s_hi[16];
     __shared__ double s_half[16];
     __shared__ uint32_t s_lut[32];
     __shared__ float warp_max[kQfThreads / 32];
@@ -246,7 +288,7 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     s_a[threadIdx.x] = 0.f;
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) s_cb[j] = cb.c[j];
+        for (int j = 0; j < 16; ++j) s_lo[j] = tp.lo[j], s_hi[j] = tp.hi[j];
 #pragma unroll
         for (int j = 0; j < 15; ++j) s_half[j] = bins.half[j];
 #pragma unroll
@@ -254,7 +296,7 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     }
     __syncthreads();
     const int j = lane & 15, half = lane >> 4;
-    const float c_lo = s_cb[j < 15 ? j : 14], c_hi = s_cb[j < 15 ? j + 1 : 15];
+    const float c_lo = s_lo[j < 15 ? j : 14], c_hi = s_hi[j < 15 ? j : 14];
     const double hk = s_half[j < 15 ? j : 14];
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
@@ -333,22 +375,15 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, Codebook cb, QuantB
     }
     if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
     if (dq) {
+        __shared__ float s_mu;
         __syncthreads();
         const bool valid = threadIdx.x < nblk;
         const float a = s_a[threadIdx.x];
-        float mx = a;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) warp_max[warp] = mx;
-        __syncthreads();
-        float gm = warp_max[0];
-#pragma unroll
-        for (int i = 1; i < kQfThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
-        const float f = __fdiv_rn(gm, 255.f);
-        if (threadIdx.x == 0) steps[blockIdx.x] = f;
-        if (valid) {
-            codes[b0 + threadIdx.x] = (uint8_t)dq_code(a, f);
-        }
+        __syncthreads();   // s_a is reused as the encoder's buffer
+        uint8_t code = 0;
+        dq_group_encode<kQfThreads>(a, valid, nblk, dq, s_a, warp_max, &s_mu, &code,
+                                    steps + blockIdx.x, means + blockIdx.x);
+        if (valid) codes[b0 + threadIdx.x] = code;
     }
 }
 
@@ -368,13 +403,13 @@ constexpr int kQbThreads = 256, kQbUnroll = 4;
 
 template <int V, bool kExactHalf>
 __global__ void __launch_bounds__(kQbThreads)
-k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBins bins, bool use_bins,
+k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, ThreshPairs tp, QuantBins bins, bool use_bins,
                    int zero_idx, int dq, uint8_t *__restrict__ packed, float *__restrict__ absmax,
-                   uint8_t *__restrict__ codes, float *__restrict__ steps,
+                   uint8_t *__restrict__ codes, float *__restrict__ steps, float *__restrict__ means,
                    uint32_t *__restrict__ status) {
     constexpr int B = 32 * V;
     __shared__ float s_a[kQbThreads];
-    __shared__ float s_cb[16];
+    __shared__ float s_lo[16], s_hi[16];
     __shared__ double s_half[16];
     __shared__ uint32_t s_lut[32];
     __shared__ float warp_max[kQbThreads / 32];
@@ -384,7 +419,7 @@ k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBi
     s_a[threadIdx.x] = 0.f;
     if (threadIdx.x == 0) {   // constant indices keep the parameters out of local memory
 #pragma unroll
-        for (int j = 0; j < 16; ++j) s_cb[j] = cb.c[j];
+        for (int j = 0; j < 16; ++j) s_lo[j] = tp.lo[j], s_hi[j] = tp.hi[j];
 #pragma unroll
         for (int j = 0; j < 15; ++j) s_half[j] = bins.half[j];
 #pragma unroll
@@ -392,7 +427,7 @@ k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBi
     }
     __syncthreads();
     const int j = lane < 15 ? lane : 14;
-    const float c_lo = s_cb[j], c_hi = s_cb[j + 1];
+    const float c_lo = s_lo[j], c_hi = s_hi[j];
     const double hk = s_half[j];
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
@@ -474,19 +509,14 @@ k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, Codebook cb, QuantBi
     }
     if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
     if (dq) {
+        __shared__ float s_mu;
         __syncthreads();
         const float a = s_a[threadIdx.x];
-        float mx = a;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) warp_max[warp] = mx;
-        __syncthreads();
-        float gm = warp_max[0];
-#pragma unroll
-        for (int i = 1; i < kQbThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
-        const float f = __fdiv_rn(gm, 255.f);
-        if (threadIdx.x == 0) steps[blockIdx.x] = f;
-        if (threadIdx.x < nblk) codes[b0 + threadIdx.x] = (uint8_t)dq_code(a, f);
+        __syncthreads();   // s_a is reused as the encoder's buffer
+        uint8_t code = 0;
+        dq_group_encode<kQbThreads>(a, threadIdx.x < nblk, nblk, dq, s_a, warp_max, &s_mu, &code,
+                                    steps + blockIdx.x, means + blockIdx.x);
+        if (threadIdx.x < nblk) codes[b0 + threadIdx.x] = code;
     }
 }
 
@@ -597,15 +627,27 @@ k_nf4_dequantize(const uint8_t *__restrict__ packed, ScaleSrc sc, int64_t nb, Co
 
 }  // namespace
 
+ThreshPairs make_pairs(const Codebook &cb) {
+    ThreshPairs tp{};
+    for (int j = 0; j < 15; ++j) {
+        int k = j;
+        while (k < 15 && cb.c[k] == cb.c[k + 1]) ++k;
+        tp.lo[j] = k < 15 ? cb.c[k] : INFINITY;
+        tp.hi[j] = k < 15 ? cb.c[k + 1] : INFINITY;
+    }
+    tp.lo[15] = tp.hi[15] = INFINITY;
+    return tp;
+}
+
 // T[bin] of the fast kernel for this codebook, or false when some bin,
 // widened by the margin, holds two thresholds (levels closer than about
 // 1/K apart): bin i holds every u with RN(K u + 16) = i.  The margin 2^-18
 // bounds both the error of w * RN(1/a) against w/a (< 2^-22 for |w| <= a) and
 // the distance of an exact threshold tau_k / a from its midpoint m_k.
-bool make_quant_bins(const Codebook &cb, QuantBins *out) {
+bool make_quant_bins(const ThreshPairs &tp, QuantBins *out) {
     const double K = (double)kBinK, margin = std::ldexp(1.0, -18);
     double m[15];
-    for (int k = 0; k < 15; ++k) m[k] = ((double)cb.c[k] + (double)cb.c[k + 1]) * 0.5;
+    for (int k = 0; k < 15; ++k) m[k] = ((double)tp.lo[k] + (double)tp.hi[k]) * 0.5;
     QuantBins qb{};
     for (int i = 0; i < 32; ++i) {
         const double lo = (i - 16.5) / K - margin, hi = (i - 15.5) / K + margin;
@@ -626,16 +668,16 @@ bool make_quant_bins(const Codebook &cb, QuantBins *out) {
 // Fills bins->half; true when every (c_k + c_{k+1}) / 2 is exact in fp64 and
 // has at most 29 significant bits, so that its product with any fp32 scale
 // is exact in fp64.
-bool make_exact_halves(const Codebook &cb, QuantBins *bins) {
+bool make_exact_halves(const ThreshPairs &tp, QuantBins *bins) {
     bool ok = true;
     for (int k = 0; k < 15; ++k) {
-        const double x = cb.c[k], y = cb.c[k + 1];
+        const double x = tp.lo[k], y = tp.hi[k];
         const double s = x + y;
         const double bb = s - x;
         const double err = (x - (s - bb)) + (y - bb);   // TwoSum: s + err == x + y
         const double h = s * 0.5;
         bins->half[k] = h;
-        if (err != 0.0) ok = false;
+        if (!(err == 0.0) || !std::isfinite(h)) ok = false;
         if (h != 0.0) {
             int e;
             const double m = std::frexp(std::fabs(h), &e);          // m in [0.5, 1)
@@ -654,13 +696,14 @@ void launch_quantize_blk(const float *W, const nf4_weight_t &q, const Codebook &
                          uint32_t *d_status, cudaStream_t st) {
     const int64_t nb = q.rows * q.cols / (32 * V);
     QuantBins bins{};
-    const bool use_bins = make_quant_bins(cb, &bins);
-    const bool exact_half = make_exact_halves(cb, &bins);
+    const ThreshPairs tp = make_pairs(cb);
+    const bool use_bins = make_quant_bins(tp, &bins);
+    const bool exact_half = make_exact_halves(tp, &bins);
     auto kern = exact_half ? k_nf4_quantize_blk<V, true> : k_nf4_quantize_blk<V, false>;
     prof_begin(kProfQuant, st);
-    kern<<<(unsigned)((nb + 255) / 256), kQbThreads, 0, st>>>(W, nb, cb, bins, use_bins, zero_idx,
+    kern<<<(unsigned)((nb + 255) / 256), kQbThreads, 0, st>>>(W, nb, tp, bins, use_bins, zero_idx,
                                                               q.double_quant, q.packed, q.absmax,
-                                                              q.absmax_code, q.dq_step, d_status);
+                                                              q.absmax_code, q.dq_step, q.dq_mean, d_status);
     prof_end(kProfQuant, st);
 }
 
@@ -668,17 +711,18 @@ void launch_quantize_blk(const float *W, const nf4_weight_t &q, const Codebook &
 
 int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &cb, int zero_idx,
                         uint32_t *d_status, cudaStream_t st) {
+    const ThreshPairs tp = make_pairs(cb);
     if (q.block != 64) {
         if (q.rows * q.cols == 0) return QLORA_OK;
         QuantBins bins32;
-        if (q.block == 32 && make_quant_bins(cb, &bins32)) {   // two blocks per warp, as at 64
+        if (q.block == 32 && make_quant_bins(tp, &bins32)) {   // two blocks per warp, as at 64
             const int64_t nb = q.rows * q.cols / 32;
-            auto kern = make_exact_halves(cb, &bins32) ? k_nf4_quantize_fast<true, 2>
+            auto kern = make_exact_halves(tp, &bins32) ? k_nf4_quantize_fast<true, 2>
                                                        : k_nf4_quantize_fast<false, 2>;
             prof_begin(kProfQuant, st);
             kern<<<(unsigned)((nb + 255) / 256), kQfThreads, kQfSmem, st>>>(
-                W, nb, cb, bins32, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code,
-                q.dq_step, d_status);
+                W, nb, tp, bins32, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code,
+                q.dq_step, q.dq_mean, d_status);
             prof_end(kProfQuant, st);
         } else if (q.block == 32) launch_quantize_blk<1>(W, q, cb, zero_idx, d_status, st);
         else if (q.block == 128) launch_quantize_blk<4>(W, q, cb, zero_idx, d_status, st);
@@ -690,14 +734,14 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
     QuantBins bins;
-    if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && make_quant_bins(cb, &bins)) {
-        const bool exact_half = make_exact_halves(cb, &bins);
+    if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && make_quant_bins(tp, &bins)) {
+        const bool exact_half = make_exact_halves(tp, &bins);
         auto kern = exact_half ? k_nf4_quantize_fast<true, 4> : k_nf4_quantize_fast<false, 4>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQfSmem);
+        if (set_max_smem(reinterpret_cast<const void *>(kern), kQfSmem) != cudaSuccess) return QLORA_ECUDA;
         prof_begin(kProfQuant, st);
         kern<<<(unsigned)((nb + 255) / 256), kQfThreads, kQfSmem, st>>>(
-            W, nb, cb, bins, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
-            d_status);
+            W, nb, tp, bins, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
+            q.dq_mean, d_status);
         prof_end(kProfQuant, st);
         QLORA_LAUNCH_CHECK();
         return QLORA_OK;
@@ -708,11 +752,11 @@ int launch_nf4_quantize(const float *W, const nf4_weight_t &q, const Codebook &c
     if (!tc::make_map(&tW, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, (uint64_t)nb, 256, 32, 256,
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return QLORA_EUNSUPPORTED;
-    cudaFuncSetAttribute(k_nf4_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
+    if (set_max_smem(reinterpret_cast<const void *>(k_nf4_quantize), kQuantSmem) != cudaSuccess) return QLORA_ECUDA;
     prof_begin(kProfQuant, st);
     k_nf4_quantize<<<(unsigned)grid, kQuantThreads, kQuantSmem, st>>>(
-        tW, nb, cb, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
-        d_status);
+        tW, nb, tp, zero_idx, q.double_quant, q.packed, q.absmax, q.absmax_code, q.dq_step,
+        q.dq_mean, d_status);
     prof_end(kProfQuant, st);
     QLORA_LAUNCH_CHECK();
     return QLORA_OK;
@@ -726,7 +770,7 @@ int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *o
         int lg = 0;
         while ((16 << lg) < q.block) ++lg;
         if ((16 << lg) != q.block) return QLORA_EUNSUPPORTED;
-        ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+        const ScaleSrc sc = scale_src(q);
         const int64_t need = (n16 + 255) / 256, cap = (int64_t)device_sms() * 8;
         k_nf4_dequantize_blk<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(q.packed, sc, n16, lg,
                                                                                cb, out);
@@ -735,7 +779,7 @@ int launch_nf4_dequantize(const nf4_weight_t &q, const Codebook &cb, uint16_t *o
     }
     const int64_t nb = q.rows * q.cols / 64;
     if (nb == 0) return QLORA_OK;
-    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    const ScaleSrc sc = scale_src(q);
     const int64_t threads = nb * 4;
     const int64_t grid = (threads + 255) / 256;
     k_nf4_dequantize<<<(unsigned)grid, 256, 0, st>>>(q.packed, sc, nb, cb, out);
@@ -750,7 +794,7 @@ int launch_nf4_dequantize_dtype(const nf4_weight_t &q, const Codebook &cb, int d
     int lg = 0;                                   // block = 8 << lg
     while ((8 << lg) < q.block) ++lg;
     if ((8 << lg) != q.block) return QLORA_EUNSUPPORTED;
-    ScaleSrc sc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    const ScaleSrc sc = scale_src(q);
     const int64_t cap = (int64_t)device_sms() * 8;
     if (dtype == QLORA_DTYPE_FP16) {
         const int64_t n16 = n / 16, need = (n16 + 255) / 256;

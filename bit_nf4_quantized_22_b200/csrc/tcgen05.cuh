@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace qlora {
@@ -25,6 +27,11 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+// Raises the barrier's expected transaction bytes without arriving.
+__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -108,6 +115,12 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t m, uint32_t n, uint32_t b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((n >> 3) << 17) |
            ((m >> 4) << 24);
+}
+
+// The same descriptor with fp16 A and B operands (format fields 0) in place
+// of bf16 (format 1): kind::f16 takes either, both operands of one type.
+__host__ __device__ constexpr uint32_t idesc_as_fp16(uint32_t idesc) {
+    return idesc & ~((7u << 7) | (7u << 10));
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
@@ -244,20 +257,54 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D tiled TMA descriptor over a row-major [outer][inner] array.
+// 2-D tiled TMA descriptor over a row-major [outer][inner] array.  A
+// descriptor depends only on the address and the geometry, so encoded ones
+// are kept (64 most recent, all keys compared) and a repeat call copies one.
 inline bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize, uint64_t inner,
               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
               CUtensorMapSwizzle sw) {
+    struct Key {
+        const void *ptr;
+        uint64_t inner, outer, row_bytes;
+        uint32_t box_inner, box_outer;
+        int dt, sw;
+        bool operator==(const Key &o) const {
+            return ptr == o.ptr && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+                   box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
+        }
+    };
+    struct Entry {
+        Key key;
+        CUtensorMap map;
+        bool used;
+    };
+    constexpr int kEntries = 64;
+    static Entry cache[kEntries];
+    static int next = 0;
+    static std::mutex mu;
+    (void)esize;
+    const Key key{ptr, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < kEntries; ++i)
+            if (cache[i].used && cache[i].key == key) {
+                *m = cache[i].map;
+                return true;
+            }
+    }
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    (void)esize;
-    return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lk(mu);
+    cache[next] = Entry{key, *m, true};
+    next = (next + 1) % kEntries;
+    return true;
 }
 
 }  // namespace tc

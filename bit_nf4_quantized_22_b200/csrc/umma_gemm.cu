@@ -22,10 +22,10 @@
 //   warp 1      TMEM allocation; in CTA 0 lane 0 issues the pair MMAs and
 //               commits them to both CTAs' barriers;
 //   warps 2..9  dequantize half a 64-weight block per thread per k-tile into
-//               the bf16 UMMA B operand (K-major for the forward, MN-major
+//               the UMMA B operand in the compute dtype, bf16 or fp16 (K-major for the forward, MN-major
 //               for the backward) and arrive on a local barrier, which
 //               CTA 1's warp 1 forwards to CTA 0 once per stage; then the epilogue
-//               TMEM -> registers -> bf16 -> global.
+//               TMEM -> registers -> compute dtype -> global.
 // After the K loop, ceil(r/64) extension k-tiles multiply the scaled
 // adapter activations (s T or s G, bf16, zero-padded to 64 columns) by the
 // adapter matrix (B, or A^T), both brought in by TMA.
@@ -64,20 +64,23 @@ struct UmmaParams {
     Codebook cb;
     uint16_t *Y;
     uint32_t *status;
+    int f16;             // the compute dtype: fp16 operands and output (else bf16)
 };
 
 // Raw scale words, fetched ahead of use and decoded when the tile arrives.
 struct ScaleRaw {
     float absmax_or_step;
+    float mu;            // group mean (mean-offset double quantization)
     uint32_t code;
     bool valid;
 };
 __device__ __forceinline__ ScaleRaw fetch_scale(const ScaleSrc &s, int64_t b, bool valid) {
-    ScaleRaw r{0.f, 0u, valid};
+    ScaleRaw r{0.f, 0.f, 0u, valid};
     if (valid) {
         if (s.dq) {
             r.code = __ldg(s.code + b);
             r.absmax_or_step = __ldg(s.step + (b >> 8));
+            if (s.dq == QLORA_DQ_MEAN) r.mu = __ldg(s.mean + (b >> 8));
         } else {
             r.absmax_or_step = __ldg(s.absmax + b);
         }
@@ -86,16 +89,16 @@ __device__ __forceinline__ ScaleRaw fetch_scale(const ScaleSrc &s, int64_t b, bo
 }
 __device__ __forceinline__ float decode_scale(const ScaleRaw &r, int dq) {
     if (!r.valid) return 0.f;
-    return dq ? __fmul_rn((float)r.code, r.absmax_or_step) : r.absmax_or_step;
+    return dq ? dq_decode(r.code, r.absmax_or_step, r.mu, dq) : r.absmax_or_step;
 }
 
 // Decode 32 weights (one 16-byte packed chunk) with block scale `ah` and
 // store them as 16-byte chunks [4h, 4h+4) of a 128-byte swizzled row at
 // `row_addr` (1 KB-aligned atom base + 128 * (row & 7)); `sw` = row & 7.
 __device__ __forceinline__ void decode_half(uint4 c, float ah, const Codebook &cb,
-                                            uint32_t row_addr, uint32_t sw, uint32_t h) {
+                                            uint32_t row_addr, uint32_t sw, uint32_t h, bool f16) {
     ProdTable tab;
-    build_table(ah, cb, tab);
+    build_table(ah, cb, tab, f16);
     uint32_t o[16];
     decode8(c.x, tab, o + 0);
     decode8(c.y, tab, o + 4);
@@ -210,8 +213,8 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         }
         // ---------------------------------------------------------- MMA issuer (CTA 0)
         if (lane == 0 && rank == 0) {
-            const uint32_t id_k = idesc_bf16(256, 256, 0);
-            const uint32_t id_mn = idesc_bf16(256, 256, 1);
+            const uint32_t id_k = p.f16 ? idesc_as_fp16(idesc_bf16(256, 256, 0)) : idesc_bf16(256, 256, 0);
+            const uint32_t id_mn = p.f16 ? idesc_as_fp16(idesc_bf16(256, 256, 1)) : idesc_bf16(256, 256, 1);
             for (int it = 0; it < total && ok; ++it) {
                 const int s = it % kStages;
                 const uint32_t par = (it / kStages) & 1;
@@ -280,12 +283,12 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             if (fwd) {
                 // packed tile [128 rows][32 B], 32-byte swizzle
                 const uint4 c = lds128(sp + pr * 32 + ((h ^ ((pr >> 2) & 1)) << 4));
-                decode_half(c, ah, p.cb, sb + (pr >> 3) * 1024 + (pr & 7) * 128, pr & 7, h);
+                decode_half(c, ah, p.cb, sb + (pr >> 3) * 1024 + (pr & 7) * 128, pr & 7, h, p.f16);
             } else {
                 // packed tile [64 rows][64 B], 64-byte swizzle
                 const uint32_t nl = pr & 63, a = pr >> 6;
                 const uint4 c = lds128(sp + nl * 64 + (((2 * a + h) ^ ((nl >> 1) & 3)) << 4));
-                decode_half(c, ah, p.cb, sb + a * 8192 + nl * 128, nl & 7, h);
+                decode_half(c, ah, p.cb, sb + a * 8192 + nl * 128, nl & 7, h, p.f16);
             }
             fence_proxy_async();
             __syncwarp();
@@ -327,11 +330,12 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint32_t chunk = 4 * (c & 1) + i;
+                    const bool f16 = p.f16;
                     sts128(box + ((chunk ^ (L & 7)) << 4),
-                           bf16x2_bits(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
-                           bf16x2_bits(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                           bf16x2_bits(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                           bf16x2_bits(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+                           pack2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), f16),
+                           pack2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), f16),
+                           pack2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), f16),
+                           pack2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), f16));
                 }
             }
             fence_proxy_async();                          // the writes, visible to the TMA engine
@@ -381,7 +385,7 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 // mode 1: Y[M, Din]  = X[M, Dout] W  + sAct[M, rp64] . Apad[Din, rp64]^T
 int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t &q,
                        const Codebook &cb, const uint16_t *sAct, int r, const uint16_t *adapter,
-                       uint16_t *Y, uint32_t *d_status, cudaStream_t st) {
+                       uint16_t *Y, uint32_t *d_status, cudaStream_t st, bool f16) {
     const int64_t Din = q.cols, Dout = q.rows;
     const int rp64 = (r + 63) / 64 * 64;
     CUtensorMap tA, tP, tAe, tBe;
@@ -420,11 +424,12 @@ int launch_umma_qgemm(int mode, const uint16_t *X, int64_t M, const nf4_weight_t
     p.nk = (int)((Kmain + kBK - 1) / kBK);
     p.ne = rp64 / 64;
     p.r = r;
-    p.sc = ScaleSrc{q.absmax, q.absmax_code, q.dq_step, q.double_quant};
+    p.sc = scale_src(q);
     p.cb = cb;
     p.Y = Y;
     p.status = d_status;
-    cudaFuncSetAttribute(k_umma_qgemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    p.f16 = f16 ? 1 : 0;
+    if (set_max_smem(reinterpret_cast<const void *>(k_umma_qgemm), kSmemBytes) != cudaSuccess) return QLORA_ECUDA;
     // clusters of two CTAs along x: pair index = N tile of 256, rank = half
     dim3 grid((unsigned)(2 * ((N + 255) / 256)), (unsigned)((M + 511) / 512));
     prof_begin(kProfUmma, st);

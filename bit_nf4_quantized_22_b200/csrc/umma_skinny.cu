@@ -52,6 +52,7 @@ struct SkinnyParams {
     float *partial;        // [splits][P][Qp]
     int64_t Qp;
     uint32_t *status;
+    int f16;               // operands in fp16 (else bf16)
 };
 
 __global__ void __launch_bounds__(kSThreads, 2)
@@ -143,8 +144,8 @@ k_umma_skinny(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ C
                 // 16-deep step advances 32 B.  MN-major: 64-wide atoms 8 KB
                 // apart, 8 k-rows per 1 KB group, a step advances 2 KB.
                 const bool akm = (p.a_kmajor >> sg) & 1, bkm = (p.b_kmajor >> sg) & 1;
-                const uint32_t idesc = idesc_bf16(128, (uint32_t)p.N, bkm ? 0u : 1u) |
-                                       (akm ? 0u : (1u << 15));
+                uint32_t idesc = idesc_bf16(128, (uint32_t)p.N, bkm ? 0u : 1u) | (akm ? 0u : (1u << 15));
+                if (p.f16) idesc = idesc_as_fp16(idesc);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = akm ? sdesc(sa + kk * 32, 16, 1024)
@@ -244,7 +245,7 @@ int skinny_k_tiles(const SkinnySeg *segs, int nseg) {
 
 // C[P, Q] partial sums into partial[splits][P][Qp] (Qp >= Q, multiple of 4).
 int launch_umma_skinny(const SkinnySeg *segs, int nseg, int64_t P, int64_t Q, int64_t Qp,
-                       float *partial, uint32_t *d_status, cudaStream_t st) {
+                       float *partial, uint32_t *d_status, cudaStream_t st, bool f16) {
     if (P <= 0 || Q <= 0) return QLORA_OK;
     const int N = skinny_n(Q < 256 ? Q : 256);
     CUtensorMap tA[2], tB[2];
@@ -270,7 +271,8 @@ int launch_umma_skinny(const SkinnySeg *segs, int nseg, int64_t P, int64_t Q, in
     prm.partial = partial;
     prm.Qp = Qp;
     prm.status = d_status;
-    cudaFuncSetAttribute(k_umma_skinny, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    prm.f16 = f16 ? 1 : 0;
+    if (set_max_smem(reinterpret_cast<const void *>(k_umma_skinny), (int)smem) != cudaSuccess) return QLORA_ECUDA;
     dim3 grid((unsigned)((P + kSBM - 1) / kSBM), (unsigned)((Q + N - 1) / N), (unsigned)splits);
     k_umma_skinny<<<grid, kSThreads, smem, st>>>(tA[0], tA[1], tB[0], tB[1], prm);
     QLORA_LAUNCH_CHECK();

@@ -45,9 +45,17 @@ class LinearSpec:
     pool_group: int = 1
 
 
-def draw(spec: LinearSpec, M: int, config: int, linear: int = 0, which=("W", "x", "A", "B", "dY")):
+def fp16_bits(a: np.ndarray) -> np.ndarray:
+    """fp32 -> IEEE binary16 bit patterns, round to nearest even."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def draw(spec: LinearSpec, M: int, config: int, linear: int = 0, which=("W", "x", "A", "B", "dY"),
+         fmt: str = "bf16"):
     """Arrays for one linear: W fp32 [Dout, Din]; x [M, Din], A [Din/g, r],
-    B [r, Dout], dY [M, Dout] as bf16 bits."""
+    B [r, Dout], dY [M, Dout] as 16-bit patterns of `fmt` ("bf16" or "fp16",
+    the layer's compute dtype), rounded from the same fp32 draws."""
+    bf16_bits = globals()["bf16_bits"] if fmt == "bf16" else fp16_bits
     out = {}
     if "W" in which:
         g = rng(config, linear, "W")

@@ -21,7 +21,9 @@
  *     16-entry codebook, which is a HOST array read during the call.  The
  *     library allocates nothing: scratch memory is the caller's `workspace`
  *     buffer, sized by qlora_workspace_size().
- *   - bf16 arrays are passed as uint16_t bit patterns; every 2-D array is
+ *   - 16-bit arrays are passed as uint16_t bit patterns: for the layer calls
+ *     and qlora_merge in the weight's compute dtype (q->compute_dtype: bf16,
+ *     or IEEE fp16), for nf4_dequantize in bf16.  Every 2-D array is
  *     row-major and densely packed.
  *   - The frozen weight is stored transposed, Wt:[Dout, Din] (the
  *     nn.Linear layout).  Flattened row-major it is cut into blocks of 64
@@ -64,26 +66,54 @@ extern "C" {
 #define QLORA_DQ_GROUP 256
 #define QLORA_MAX_RANK 256
 
+/* Double-quantization codes of the first-level scales (nf4_weight_t's
+ * double_quant).  bitsandbytes article (CSDN) 7.2 gives the structure -- an
+ * 8-bit code per block scale, one fp32 constant per 256 scales -- but not the
+ * code; three are provided, each step one stated rounding:
+ *   QLORA_DQ_U8    unsigned: step f = RN32(group max / 255),
+ *                  code = round-half-even(a / f) in 0..255
+ *   QLORA_DQ_S8    the signed INT8 absmax code of section 4.1 applied to the
+ *                  scales: f = RN32(group max / 127), code in 0..127 (scales
+ *                  are >= 0)
+ *   QLORA_DQ_MEAN  the group mean taken out first: mu = RN32(S / n), S the
+ *                  fp64 sum of the group's scales in block order; d = RN32(a - mu);
+ *                  f = RN32(max |d| / 127); code = round-half-even(d / f) in
+ *                  -127..127 stored as int8; one mu per group in dq_mean
+ * Decoded scale: RN32(code * f), or RN32(mu + RN32(code * f)) for QLORA_DQ_MEAN.
+ * The weights themselves are encoded with the exact block absmax. */
+/* Compute dtypes (bitsandbytes article (CSDN) 8.3: the dequantized weight
+ * and the arithmetic are FP32, BF16 or FP16; 8.5 on FP16's narrower range).
+ * The layer calls take BF16 or FP16 (nf4_weight_t's compute_dtype);
+ * nf4_dequantize_dtype also writes FP32. */
+#define QLORA_DTYPE_BF16 0
+#define QLORA_DTYPE_FP16 1
+#define QLORA_DTYPE_FP32 2
+
+#define QLORA_DQ_NONE 0
+#define QLORA_DQ_U8 1
+#define QLORA_DQ_S8 2
+#define QLORA_DQ_MEAN 3
+
 /* One quantized weight Wt:[rows = Dout, cols = Din]; nb = rows*cols/block.
  *   packed      [rows*cols/2] uint8   two 4-bit codebook indices per byte;
  *                                     element 2i in the HIGH nibble of byte i
  *   absmax      [nb] fp32             block absmax (double_quant == 0)
- *   absmax_code [nb] uint8            8-bit scale codes (double_quant == 1)
+ *   absmax_code [nb] uint8 / int8     8-bit scale codes (double_quant != 0)
  *   dq_step     [ceil(nb/256)] fp32   one second-level step per 256 blocks
- * With double quantization the decoded scale of block b is
- * RN32(absmax_code[b] * dq_step[b/256]); the codes are round-half-even of
- * absmax/step with step = RN32(group max / 255). */
+ *   dq_mean     [ceil(nb/256)] fp32   group means (double_quant == QLORA_DQ_MEAN)
+ * Unused arrays may be NULL. */
 typedef struct {
     int64_t rows;
     int64_t cols;
     int32_t block;          /* 64; the codec calls also take 32, 128, 256 */
-    int32_t double_quant;   /* 0 or 1 */
-    int32_t dq_group;       /* must be 256 when double_quant == 1 */
-    int32_t reserved;
+    int32_t double_quant;   /* QLORA_DQ_NONE, _U8, _S8 or _MEAN */
+    int32_t dq_group;       /* must be 256 when double_quant != 0 */
+    int32_t compute_dtype;  /* QLORA_DTYPE_BF16 or _FP16: the layer calls' 16-bit arrays */
     uint8_t *packed;
     float *absmax;
     uint8_t *absmax_code;
     float *dq_step;
+    float *dq_mean;
 } nf4_weight_t;
 
 /* Human-readable name of a return code (static storage). */
@@ -109,8 +139,23 @@ int qlora_version(void);
 #define QLORA_NF4_DELTA 0.96770833333333333333
 int nf4_codebook(double delta, float out[16]);
 
-/* Host-side check of a codebook (no device work): 16 finite fp32 values,
- * strictly increasing, inside [-1, 1], one of them exactly 0.
+/* fp4_codebook -- the FP4 table, built on the host (no device work).
+ * bitsandbytes article (CSDN) sections 6.4-6.5 and 9.3 name a "4-bit
+ * float-style" table (the library's default type) and print no values; the
+ * layout used is FP4 E2M1 (OCP Microscaling formats: sign bit, two exponent
+ * bits with bias 1, one mantissa bit, exponent field 0 subnormal), divided by
+ * its largest magnitude 6:
+ *   out = [-1, -2/3, -1/2, -1/3, -1/4, -1/6, -1/12, -0,
+ *          +0, 1/12, 1/6, 1/4, 1/3, 1/2, 2/3, 1]   (each rounded to fp32).
+ * Zero appears twice (-0, +0).  Quantization takes the first nearest level,
+ * so every weight in zero's basin gets -0 and the +0 code is never written.
+ *   out     host fp32[16] (output, caller-owned)
+ * Errors: EINVAL for a NULL out. */
+int fp4_codebook(float out[16]);
+
+/* Host-side check of a codebook (no device work): 16 finite fp32 values
+ * inside [-1, 1], strictly increasing except that the zero level may appear
+ * twice in a row (-0 then +0, as in the FP4 table), with at least one zero.
  * Returns QLORA_OK or QLORA_EINVAL. */
 int qlora_check_codebook(const float codebook[16]);
 
@@ -138,11 +183,6 @@ int nf4_quantize(const float *W, const nf4_weight_t *q, const float codebook[16]
 int nf4_dequantize(const nf4_weight_t *q, const float codebook[16], uint16_t *W_out,
                    void *stream);
 
-/* Compute dtypes of nf4_dequantize_dtype (section 8.3: FP32, BF16 or FP16). */
-#define QLORA_DTYPE_BF16 0
-#define QLORA_DTYPE_FP16 1
-#define QLORA_DTYPE_FP32 2
-
 /* nf4_dequantize_dtype -- as nf4_dequantize, into the compute dtype `dtype`
  * (bitsandbytes article (CSDN) section 8.3: the dequantized weights and the
  * arithmetic are FP32, BF16 or FP16; 8.5 on FP16's narrower range):
@@ -158,13 +198,14 @@ int nf4_dequantize_dtype(const nf4_weight_t *q, const float codebook[16], int32_
 /* qlora_merge -- the weight with the adapter folded in, for deployment
  * ("从 LoRA 到 QLoRA、QA-LoRA" section 2, W_eff = dequant(W4) + (alpha/r) A B;
  * bitsandbytes article (CSDN) 12.10, merging before deployment):
- *   W_out[n][k] = RN_bf16( w_hat[n][k] + (s/g) sum_j A[k/g][j] B[j][n] ),
- * s = alpha/r, g = pool_group, w_hat the bf16 dequantized weight as
+ *   W_out[n][k] = RN_dt( w_hat[n][k] + (s/g) sum_j A[k/g][j] B[j][n] ),
+ * s = alpha/r, g = pool_group, dt = q->compute_dtype, w_hat the dequantized
+ * weight RN_dt(RN32(a_hat c_q)), as
  * nf4_dequantize writes it; the rank-r sum is accumulated in fp32.  With
  * g = 64 every input of a group shares (A_p B)/g (the same blog, section 5),
  * so that x . W_out^T is the pooled layer's forward.
- *   A       device bf16 [Din/pool_group, r];  B  device bf16 [r, Dout]
- *   W_out   device bf16 [Dout, Din], 16-byte aligned (output)
+ *   A       device dt [Din/pool_group, r];  B  device dt [r, Dout]
+ *   W_out   device dt [Dout, Din], 16-byte aligned (output)
  * No workspace.  Errors as nf4_dequantize, plus EINVAL for r outside
  * [1, QLORA_MAX_RANK], a non-finite alpha or pool_group not 1 or 64. */
 int qlora_merge(const nf4_weight_t *q, const float codebook[16], const uint16_t *A,
@@ -179,13 +220,16 @@ size_t qlora_workspace_size(int64_t M, const nf4_weight_t *q, int32_t r, int32_t
 /* qlora_forward -- y = x . dequant(W4) + (alpha/r) T . B with
  * T = u . A, u = x (pool_group == 1) or the mean of each run of 64 input
  * features (pool_group == 64, the pooled adapter of QA-LoRA sections 3-4).
- *   X       device bf16 [M, Din]
- *   A       device bf16 [Din/pool_group, r];  B  device bf16 [r, Dout]
+ *   X       device [M, Din] in the compute dtype dt = q->compute_dtype
+ *           (bf16 or fp16; bitsandbytes article (CSDN) 8.3)
+ *   A       device dt [Din/pool_group, r];  B  device dt [r, Dout]
  *   r       1..256;  alpha finite;  pool_group 1 or 64
- *   Y       device bf16 [M, Dout] (output)
+ *   Y       device dt [M, Dout] (output)
  *   T_save  device fp32 [M, r] receiving T, or NULL
  *   workspace/ws_bytes  caller scratch of at least qlora_workspace_size(.., 0)
- * Accumulation is fp32; y is rounded once to bf16. */
+ * Accumulation is fp32; y is rounded once to dt.  With fp16, the fp32
+ * adapter intermediates (T, G, pooled inputs) are carried as fp16 hi + lo
+ * pairs, so they keep about 22 significant bits inside fp16's range (8.5). */
 int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const float codebook[16],
                   const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
                   int32_t pool_group, uint16_t *Y, float *T_save, void *workspace,
@@ -193,7 +237,7 @@ int qlora_forward(const uint16_t *X, int64_t M, const nf4_weight_t *q, const flo
 
 /* qlora_backward -- gradients of the layer for the upstream gradient dY:
  *   G  = dY . B^T                               (fp32 [M, r], internal)
- *   dX = dY . dequant(W4)^T + (s/g) G . A^T     (bf16 [M, Din]; with pooling
+ *   dX = dY . dequant(W4)^T + (s/g) G . A^T     (dt [M, Din]; with pooling
  *                                                each input feature of a
  *                                                group receives 1/g of it)
  *   dA = s u^T G                                (fp32 [Din/g, r])
@@ -217,12 +261,18 @@ int qlora_backward(const uint16_t *X, const uint16_t *dY, int64_t M, const nf4_w
  * library, which every GPU that loads the library holds until the process
  * exits.
  *   - Requests needing more scratch than that return QLORA_EWORKSPACE before
- *     anything is enqueued (qlora_workspace_size(M, q, r, pool_group, 0)
- *     tells the need; decode-sized calls fit, e.g. M <= 16 at 4096 x 4096).
+ *     anything is enqueued; qlora_workspace_size(M, q, r, pool_group, 0)
+ *     tells the need.  Decode shapes that fit: M <= 16 at 4096 x 4096
+ *     (r <= 64), and M = 1 on the 8192 <-> 28672 projections (r = 64); M = 16
+ *     there does not (its split partials alone take 14.7 MB).  On the
+ *     tensor-core path (M > 16) the need also depends on the GPU's SM count.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for the
+ *     life of the process; make that first call before any stream capture.
+ *     cudaDeviceReset after the first call on a device is not supported:
+ *     the module may come back at another address, and later calls would
+ *     still use the old one.
  *   - Every call shares the one array and leaves its contents behind; each
  *     call clears what it needs zeroed.  Calls that overlap on the GPU (two
  *     streams, or two host threads) race on the array: serialize them. */

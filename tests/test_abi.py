@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strerror(lib):
-    assert lib.qlora_version() == 100
+    assert lib.qlora_version() == 200
     assert lib.qlora_strerror(0) == b"ok"
     assert lib.qlora_strerror(4) == b"workspace too small"
 
@@ -60,7 +60,19 @@ def test_codebook_validation(lib):
 
 def _wc(rows=64, cols=128, dq=1, block=64, group=256, ptrs=True):
     fake = 1 << 20 if ptrs else 0   # never dereferenced: validation fails first or no launch
-    return _lib.NF4WeightC(rows, cols, block, dq, group, 0, fake, fake, fake, fake)
+    return _lib.NF4WeightC(rows, cols, block, dq, group, 0, fake, fake, fake, fake, fake)
+
+
+def test_dq_variant_validation(lib):
+    """double_quant is a code kind 0..3; the mean-offset kind needs dq_mean."""
+    cb = _cb(q.nf4_codebook().tolist())
+    W = ctypes.c_void_p(1 << 20)
+    for bad in (-1, 4):
+        assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=bad)), cb, None, None) == _lib.QLORA_EINVAL
+    wc = _wc(dq=3)
+    wc.dq_mean = None
+    assert lib.nf4_quantize(W, ctypes.byref(wc), cb, None, None) == _lib.QLORA_EINVAL
+    assert ctypes.sizeof(_lib.NF4WeightC) == 72 and _lib.NF4WeightC.dq_mean.offset == 64
 
 
 def test_quantize_rejects_bad_arguments(lib):
@@ -79,7 +91,6 @@ def test_quantize_rejects_bad_arguments(lib):
                                     None) == E.QLORA_EINVAL
     assert lib.nf4_dequantize_dtype(ctypes.byref(_wc(rows=0)), cb, 2, W, None) == E.QLORA_OK
     assert lib.nf4_quantize(W, ctypes.byref(_wc(group=128)), cb, None, None) == E.QLORA_EUNSUPPORTED
-    assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=2)), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_quantize(W, ctypes.byref(_wc(ptrs=False)), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_quantize(None, ctypes.byref(_wc()), cb, None, None) == E.QLORA_EINVAL
     assert lib.nf4_quantize(ctypes.c_void_p((1 << 20) + 4), ctypes.byref(_wc()), cb, None, None) == E.QLORA_EINVAL
@@ -145,6 +156,28 @@ def test_product_codebook_matches_oracle(orc, delta):
     b = orc.nf4_codebook() if delta is None else orc.nf4_codebook(delta)
     assert np.array_equal(a.view(np.int32), b.view(np.int32))
     assert a[0] == -1 and a[7] == 0 and a[15] == 1
+
+
+def test_product_fp4_codebook_matches_oracle(orc, lib):
+    """fp4_codebook (the library's E2M1 construction) gives the oracle's FP4
+    table bit for bit, -0 included, and passes the codebook check."""
+    a = q.fp4_codebook().numpy()
+    b = orc.fp4_codebook()
+    assert np.array_equal(a.view(np.int32), b.view(np.int32))
+    assert lib.qlora_check_codebook(_cb(a.tolist())) == 0
+    assert lib.fp4_codebook(None) == _lib.QLORA_EINVAL
+
+
+def test_codebook_check_repeated_levels(lib):
+    """Only the zero may repeat (twice, as -0 and +0); any other repeat, or a
+    third zero, is refused."""
+    base = q.nf4_codebook().tolist()
+    two_zeros = base[:7] + [-0.0, 0.0] + base[9:]
+    assert lib.qlora_check_codebook(_cb(two_zeros)) == 0
+    three_zeros = base[:6] + [0.0, -0.0, 0.0] + base[9:]
+    assert lib.qlora_check_codebook(_cb(three_zeros)) == _lib.QLORA_EINVAL
+    repeat = list(base); repeat[11] = repeat[10]
+    assert lib.qlora_check_codebook(_cb(repeat)) == _lib.QLORA_EINVAL
 
 
 def test_codebook_call_rejects_bad_delta(lib):

@@ -72,6 +72,8 @@ def test_ragged_small(orc, qlib, M, dq):
     (3, 1088, 264, True),     # Din/64 = 17: scale rows not tileable -> register GEMV
     (12, 4160, 136, False),   # Din/64 = 65 (odd): register GEMV, ragged slice
     (5, 1280, 392, False),    # streamed backward: last 512-input slice half full
+    (2, 1536, 392, True),     # double quantization, Din/64 = 24: half a forward slice at the end
+    (16, 2560, 520, True),    # double quantization, Din/64 = 40, ragged 128-row tile
 ])
 def test_gemv_paths(orc, qlib, M, Din, Dout, dq):
     spec = LinearSpec("g", Din, Dout, 8, 16.0, dq)

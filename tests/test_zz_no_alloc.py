@@ -53,13 +53,19 @@ def test_noalloc_matches_forward(qlib, M, Din, Dout, r, dq, pool):
     x, A, B = dev_bf16(a["x"]), dev_bf16(a["A"]), dev_bf16(a["B"])
     y_ref, T_ref = qlib.forward(x, w, A, B, spec.alpha, pool)
     torch.cuda.synchronize()
-    for _ in range(2):
-        y = torch.full((M, Dout), float("nan"), dtype=torch.bfloat16, device="cuda")
-        T = torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda")
+    ys = [torch.full((M, Dout), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    Ts = [torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda") for _ in range(2)]
+    free = []
+    for y, T in zip(ys, Ts):
+        torch.cuda.synchronize()
+        free.append(torch.cuda.mem_get_info()[0])
         assert _noalloc(lib, qlib, x, w, A, B, r, spec.alpha, pool, y, T) == QLORA_OK
         torch.cuda.synchronize()
         assert_close(host_f64(y), host_f64(y_ref), "y (no-alloc vs workspace forward)")
         assert_close(host_f64(T), host_f64(T_ref), "T (no-alloc vs workspace forward)")
+    # the second call finds the kernels loaded and allocates nothing: the
+    # device's free memory is the same before and after it
+    assert torch.cuda.mem_get_info()[0] == free[1]
 
 
 def test_noalloc_refuses_oversize_request(qlib):
@@ -73,6 +79,23 @@ def test_noalloc_refuses_oversize_request(qlib):
     B = torch.zeros(r, Dout, dtype=torch.bfloat16, device="cuda")
     y = torch.full((M, Dout), 7.0, dtype=torch.bfloat16, device="cuda")
     assert qlib.workspace_size(M, w, r, 1, 0) > (8 << 20)
+    assert _noalloc(lib, qlib, x, w, A, B, r, 16.0, 1, y, None) == QLORA_EWORKSPACE
+    torch.cuda.synchronize()
+    assert bool(torch.all(y == 7.0))
+
+
+def test_noalloc_decode_limits(qlib):
+    """The stated limits: on the 8192 -> 28672 projection (r = 64) M = 1 fits
+    the fixed array and M = 16 does not (refused, output untouched)."""
+    lib = qlib.load()
+    Din, Dout, r = 8192, 28672, 64
+    w = qlib.NF4Weight.empty(Dout, Din, True)
+    A = torch.zeros(Din, r, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(r, Dout, dtype=torch.bfloat16, device="cuda")
+    assert qlib.workspace_size(1, w, r, 1, 0) <= (8 << 20)
+    assert qlib.workspace_size(16, w, r, 1, 0) > (8 << 20)
+    x = torch.zeros(16, Din, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((16, Dout), 7.0, dtype=torch.bfloat16, device="cuda")
     assert _noalloc(lib, qlib, x, w, A, B, r, 16.0, 1, y, None) == QLORA_EWORKSPACE
     torch.cuda.synchronize()
     assert bool(torch.all(y == 7.0))
