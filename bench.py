@@ -196,6 +196,59 @@ def oracle_step_estimate(a, spec, M, rows, quant_rows):
             "step_s_extrapolated": step_s}
 
 
+def oracle_table(budget_s=4.0):
+    """The oracle on every workload of the five configurations: one JSON line
+    per (config, linear, M) with its extrapolated step time on this process's
+    threads (OMP_NUM_THREADS decides how many).  A step is quantize +
+    dequantize of the weight and forward + backward for the training shapes;
+    dequantize + forward for the forward-only decode shapes (the quantized
+    weight is made once, outside the step).  The weight part runs on 512
+    weight rows, the layer part on a token sample grown until it takes about a
+    quarter of `budget_s`; each is scaled to the full shape."""
+    import oracle
+    cb = oracle.nf4_codebook()
+    cores = oracle.num_threads()
+    for cfg, c in synth.CONFIGS.items():
+        train = "bwd" in c["passes"]
+        for lin, spec in enumerate(c["linears"]):
+            a = synth.draw(spec, max(c["M"]), cfg, lin)
+            g = spec.pool_group
+            qr = min(spec.Dout, 512)
+            t0 = time.perf_counter()
+            qs = oracle.quantize(a["W"][:qr], cb, spec.double_quant)
+            tquant = time.perf_counter() - t0
+            t0 = time.perf_counter()
+            oracle.dequantize(qs, cb)
+            tdeq = time.perf_counter() - t0
+            Wt = oracle.dequantize(oracle.quantize(a["W"], cb, spec.double_quant), cb)
+            for M in c["M"]:
+                rows = min(M, 8)
+                while True:
+                    sel = (np.arange(rows) * 131) % M
+                    t0 = time.perf_counter()
+                    oracle.forward(a["x"][sel], Wt, a["A"], a["B"], spec.r, spec.alpha, g)
+                    if train:
+                        oracle.backward(a["x"][sel], a["dY"][sel], Wt, a["A"], a["B"], spec.r,
+                                        spec.alpha, g)
+                    tl = time.perf_counter() - t0
+                    if rows >= M or tl * 4 > budget_s:
+                        break
+                    rows = min(M, rows * 4)
+                tw = (tquant + tdeq) if train else tdeq
+                step = tl * (M / rows) + tw * (spec.Dout / qr)
+                if train:
+                    flops = layer_flops(M, spec.Din, spec.Dout, spec.r)
+                else:
+                    flops = 2 * M * spec.Din * spec.Dout + 2 * M * spec.r * (spec.Din // g + spec.Dout)
+                print(json.dumps({
+                    "config": cfg, "linear": spec.name, "shape": f"{spec.Din}->{spec.Dout}", "M": M,
+                    "passes": "quantize+fwd+bwd" if train else "fwd", "cores": cores,
+                    "step_s": step, "tflops": flops / step / 1e12,
+                    "sample": f"{qr} of {spec.Dout} weight rows, {rows} of {M} token rows"}),
+                    flush=True)
+            del a, Wt
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
@@ -797,7 +850,13 @@ def main():
                          "tokens and exit (a small, fixed launch sequence for ncu captures)")
     ap.add_argument("--oracle-sample", nargs=2, type=int, metavar=("ROWS", "QUANT_ROWS"),
                     help=argparse.SUPPRESS)
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="time the oracle on every workload of the five configurations (CPU "
+                         "only; OMP_NUM_THREADS sets the threads) and exit")
     args = ap.parse_args()
+    if args.oracle_table:
+        oracle_table()
+        return
     if args.oracle_sample:
         spec = synth.CONFIGS[CFG]["linears"][0]
         M = synth.CONFIGS[CFG]["M"][0]
