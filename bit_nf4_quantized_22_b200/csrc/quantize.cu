@@ -300,22 +300,32 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Qua
     const double hk = s_half[j < 15 ? j : 14];
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
-    for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
-        float pre[4][V];
+    // the loads of quarter c + 1 are issued before quarter c is decided
+    float nxt[4][V];
+    auto load_quarter = [&](int c, float (&dst)[4][V]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int bl = 64 * c + 2 * (warp + 8 * i) + half;
             const float *src = W + (b0 + bl) * (16 * V) + V * j;
             if (V == 4) {
-                const float4 v = bl < nblk ? __ldcs(reinterpret_cast<const float4 *>(src))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                pre[i][0] = v.x, pre[i][1] = v.y, pre[i][2] = v.z, pre[i][3] = v.w;
+                const float4 v = (c < 4 && bl < nblk) ? __ldcs(reinterpret_cast<const float4 *>(src))
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                dst[i][0] = v.x, dst[i][1] = v.y, dst[i][2] = v.z, dst[i][3] = v.w;
             } else {
-                const float2 v = bl < nblk ? __ldcs(reinterpret_cast<const float2 *>(src))
-                                           : make_float2(0.f, 0.f);
-                pre[i][0] = v.x, pre[i][1] = v.y;
+                const float2 v = (c < 4 && bl < nblk) ? __ldcs(reinterpret_cast<const float2 *>(src))
+                                                      : make_float2(0.f, 0.f);
+                dst[i][0] = v.x, dst[i][1] = v.y;
             }
         }
+    };
+    load_quarter(0, nxt);
+    for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
+        float pre[4][V];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < V; ++k) pre[i][k] = nxt[i][k];
+        if (c + 1 < 4 && 64 * (c + 1) < nblk) load_quarter(c + 1, nxt);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int bl = 64 * c + 2 * (warp + 8 * i) + half;   // block within the group
@@ -323,10 +333,11 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Qua
             float w[V];
 #pragma unroll
             for (int k = 0; k < V; ++k) w[k] = pre[i][k];
-            // max |w| on the bit patterns: NaN and Inf sort above every finite value
-            uint32_t m = 0;
+            // max |w|, NaN-propagating: a NaN or Inf weight makes a non-finite scale
+            float fm = 0.f;
 #pragma unroll
-            for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[k]) & 0x7fffffffu);
+            for (int k = 0; k < V; ++k) asm("max.NaN.f32 %0, %1, %2;" : "=f"(fm) : "f"(fm), "f"(fabsf(w[k])));
+            const uint32_t m = __float_as_uint(fm);
             const uint32_t m0 = __reduce_max_sync(0xffffffffu, half ? 0u : m);
             const uint32_t m1 = __reduce_max_sync(0xffffffffu, half ? m : 0u);
             const uint32_t ab = half ? m1 : m0;
@@ -360,7 +371,7 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Qua
             if (valid) {
                 // weights V j .. V j + V-1 -> bytes (V/2) j ..; element 2i in the high nibble
                 if (V == 4) {
-                    const uint32_t v = qv[1] | (qv[0] << 4) | (qv[3 % V] << 8) | (qv[2 % V] << 12);
+                    const uint32_t v = (qv[2 % V] * 16u + qv[3 % V]) * 256u + (qv[0] * 16u + qv[1]);
                     *reinterpret_cast<uint16_t *>(packed + (b0 + bl) * 32 + 2 * j) = (uint16_t)v;
                 } else {
                     packed[(b0 + bl) * 16 + j] = (uint8_t)(qv[1] | (qv[0] << 4));

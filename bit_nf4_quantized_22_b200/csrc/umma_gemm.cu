@@ -118,13 +118,18 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *gen_base = smem_raw + (base - raw_addr);
     const uint32_t bar0 = base + kStages * kStageBytes;
-    auto full_a = [&](int s) { return bar0 + 8u * s; };                  // CTA 0: A (+ext) of both
+    // CTA 0's full_a(s): the stage is ready for the MMA -- both CTAs' A (and
+    // extension) bytes landed, CTA 0's 8 dequant warps wrote its B half, and
+    // CTA 1's forwarder reported CTA 1's half (1 + 8 + 1 arrivals).  One wait
+    // per k-tile keeps the single MMA-issuing thread's loop short: it is on
+    // the critical path of every k-tile.
+    auto full_a = [&](int s) { return bar0 + 8u * s; };
     auto full_p = [&](int s) { return bar0 + 8u * (kStages + s); };      // local packed tile
-    auto bready = [&](int s) { return bar0 + 8u * (2 * kStages + s); };  // local B half ready
+    auto bready = [&](int s) { return bar0 + 8u * (2 * kStages + s); };  // CTA 1: its B half written
     auto empty = [&](int s) { return bar0 + 8u * (3 * kStages + s); };   // stage free (both)
-    auto pready = [&](int s) { return bar0 + 8u * (4 * kStages + s); };  // CTA 0: peer's B half ready
     const uint32_t acc_bar = bar0 + 8u * (5 * kStages);
-    // 5 * kStages + 1 barriers (168 B), then the TMEM address and the abort flag
+    // 5 * kStages + 1 barrier slots (168 B; slots 4 kStages .. 5 kStages - 1 unused), then the
+    // TMEM address and the abort flag
     static_assert(8 * (5 * kStages + 1) <= 200, "barrier block overlaps the flags");
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gen_base + kStages * kStageBytes + 208);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gen_base + kStages * kStageBytes + 240);
@@ -139,11 +144,10 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_a(s), 1);
+            mbar_init(full_a(s), 2 + kDqWarps);
             mbar_init(full_p(s), 1);
             mbar_init(bready(s), kDqWarps);
             mbar_init(empty(s), 1);
-            mbar_init(pready(s), 1);
         }
         mbar_init(acc_bar, 1);
         *abort_flag = 0;
@@ -185,7 +189,10 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         tma_load_2d(sp, &tmP, (int)(nc / 2), it * kBK, full_p(s));
                 } else {
                     const int e = it - p.nk;
-                    if (rank == 0) mbar_expect_tx(full_a(s), 2 * (kABytes + kBBytes));
+                    if (rank == 0) {   // no dequantized half: arrive for the warps and the forwarder
+                        mbar_expect_tx(full_a(s), 2 * (kABytes + kBBytes));
+                        mbar_arrive_n(full_a(s), 1 + kDqWarps);
+                    }
                     tma_load_2d_pair(sa, &tmAe, e * 64, y0, fa0);
                     tma_load_2d_pair(sa + kSlabBytes, &tmAe, e * 64, y1, fa0);
                     if (fwd) {
@@ -203,11 +210,11 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         // One cluster-scope arrive per stage tells CTA 0 that this CTA's B
         // half is written (the dequant warps only arrive locally).
         if (lane == 0 && rank == 1) {
-            const uint32_t pready0 = mapa_shared(pready(0), 0);
+            const uint32_t ready0 = mapa_shared(full_a(0), 0);
             for (int it = 0; it < p.nk && ok; ++it) {
                 const int s = it % kStages;
                 ok = mbar_wait(bready(s), (it / kStages) & 1, abort_flag);
-                if (ok) mbar_arrive_cluster(pready0 + 8u * s);
+                if (ok) mbar_arrive_cluster(ready0 + 8u * s);
             }
             if (!ok) *abort_flag = 1;
         }
@@ -215,36 +222,45 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         if (lane == 0 && rank == 0) {
             const uint32_t id_k = p.f16 ? idesc_as_fp16(idesc_bf16(256, 256, 0)) : idesc_bf16(256, 256, 0);
             const uint32_t id_mn = p.f16 ? idesc_as_fp16(idesc_bf16(256, 256, 1)) : idesc_bf16(256, 256, 1);
+            // Descriptors of stage 0's operands; a shared-memory offset o (a
+            // multiple of 16 B, the address staying below 256 KB) adds o >> 4
+            // to the start-address field.  B operand: forward main and
+            // backward extension are K-major (rows of 64 k, 128 B, 8-row groups
+            // 1 KB apart, +32 B per 16 k); backward main and forward extension
+            // are MN-major (2 atoms of 64 columns 8 KB apart, x 64 k rows of
+            // 128 B, +2 KB per 16 k).
+            const uint64_t dA = sdesc(base, 16, 1024);
+            const uint64_t dBk = sdesc(base + kABytes + kPBytes, 16, 1024);
+            const uint64_t dBm = sdesc(base + kABytes + kPBytes, 8192, 1024);
+            constexpr uint32_t kStageD = kStageBytes >> 4, kSlabD = kSlabBytes >> 4;
             for (int it = 0; it < total && ok; ++it) {
-                const int s = it % kStages;
-                const uint32_t par = (it / kStages) & 1;
-                const bool main = it < p.nk;
-                ok = mbar_wait_cluster(full_a(s), par, abort_flag);
-                if (ok && main) ok = mbar_wait(bready(s), par, abort_flag);
-                if (ok && main) ok = mbar_wait_cluster(pready(s), par, abort_flag);
+                const uint32_t s = it & (kStages - 1);
+                ok = mbar_wait_cluster(full_a(s), (it / kStages) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t sa = base + s * kStageBytes;
-                const uint32_t sb = sa + kABytes + kPBytes;
-                int nsteps = 4;
-                if (!main) {
-                    const int rem = p.r - (it - p.nk) * 64;
-                    nsteps = rem >= 64 ? 4 : (rem + 15) / 16;
-                }
-                // B operand: forward main and backward extension are K-major
-                // (rows of 64 k, 128 B, 8-row groups 1 KB apart); backward main
-                // and forward extension are MN-major (2 atoms of 64 columns,
-                // 8 KB apart, x 64 k rows of 128 B).
-                const bool b_kmajor = (fwd == main);
-                const uint32_t idesc = b_kmajor ? id_k : id_mn;
-                for (int kk = 0; kk < nsteps; ++kk) {
-                    const uint64_t bd = b_kmajor ? sdesc(sb + kk * 32, 16, 1024)
-                                                 : sdesc(sb + kk * 2048, 8192, 1024);
+                const uint64_t so = (uint64_t)(s * kStageD);
+                const uint32_t acc0 = it > 0 ? 1u : 0u;
+                if (it < p.nk) {
+                    const uint64_t db = (fwd ? dBk : dBm) + so;
+                    const uint32_t idesc = fwd ? id_k : id_mn;
+                    const uint32_t bstep = fwd ? 2u : 128u;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint64_t ad = sdesc(sa + h * kSlabBytes + kk * 32, 16, 1024);
-                        umma_bf16_pair(tmem + h * 256, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            umma_bf16_pair(tmem + h * 256, dA + so + h * kSlabD + kk * 2, db + kk * bstep, idesc,
+                                           kk > 0 ? 1u : acc0);
+                } else {
+                    const int rem = p.r - (it - p.nk) * 64;
+                    const int nsteps = rem >= 64 ? 4 : (rem + 15) / 16;
+                    const uint64_t db = (fwd ? dBm : dBk) + so;
+                    const uint32_t idesc = fwd ? id_mn : id_k;
+                    const uint32_t bstep = fwd ? 128u : 2u;
+                    for (int kk = 0; kk < nsteps; ++kk)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            umma_bf16_pair(tmem + h * 256, dA + so + h * kSlabD + kk * 2, db + kk * bstep, idesc,
+                                           kk > 0 ? 1u : acc0);
                 }
                 umma_commit_pair(empty(s), 0x3);
             }
@@ -292,7 +308,7 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             }
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bready(s));
+            if (lane == 0) mbar_arrive(rank == 0 ? full_a(s) : bready(s));   // CTA 1: via the forwarder
             return true;
         };
         // scales are fetched three k-tiles ahead of use
