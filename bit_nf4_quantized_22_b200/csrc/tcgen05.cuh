@@ -234,6 +234,28 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
+// The 8 pair MMAs of one 64-deep k-tile of a 512 x 256 tile: MMA halves
+// h = 0, 1 (accumulators d0, d1) x 4 steps of 16 k; a0/a1: the halves' A
+// descriptors per step, b: the B descriptor per step.  acc0 = 0 starts the
+// accumulators at the first step; later steps always accumulate.
+__device__ __forceinline__ void umma_ktile_pair(uint32_t d0, uint32_t d1, const uint64_t (&a0)[4],
+                                                const uint64_t (&a1)[4], const uint64_t (&b)[4],
+                                                uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %14, 0;\n\t"
+        "setp.eq.b32 q, %14, %14;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %2, %10, %15, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], %6, %10, %15, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %3, %11, %15, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], %7, %11, %15, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %4, %12, %15, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], %8, %12, %15, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %13, %15, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], %9, %13, %15, q;\n\t}\n" ::"r"(d0),
+        "r"(d1), "l"(a0[0]), "l"(a0[1]), "l"(a0[2]), "l"(a0[3]), "l"(a1[0]), "l"(a1[1]), "l"(a1[2]),
+        "l"(a1[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(acc0), "r"(idesc));
+}
 // Arrive (once) on the mbarrier at offset `bar` in every CTA of `mask` when
 // all previously issued pair MMAs have completed.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {

@@ -233,35 +233,51 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             const uint64_t dBk = sdesc(base + kABytes + kPBytes, 16, 1024);
             const uint64_t dBm = sdesc(base + kABytes + kPBytes, 8192, 1024);
             constexpr uint32_t kStageD = kStageBytes >> 4, kSlabD = kSlabBytes >> 4;
-            for (int it = 0; it < total && ok; ++it) {
+            // main k-tiles, unrolled over the stages (constant stage addresses)
+            {
+                const uint64_t db0 = fwd ? dBk : dBm;
+                const uint32_t idesc = fwd ? id_k : id_mn;
+                const uint32_t bstep = fwd ? 2u : 128u;
+                for (int it0 = 0; it0 < p.nk && ok; it0 += kStages) {
+                    const uint32_t par = (it0 / kStages) & 1;
+#pragma unroll
+                    for (int j = 0; j < kStages; ++j) {
+                        const int it = it0 + j;
+                        if (it >= p.nk || !ok) break;
+                        ok = mbar_wait_cluster(full_a(j), par, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t so = (uint64_t)(j * kStageD);
+                        uint64_t a0[4], a1[4], bd[4];
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            a0[kk] = dA + so + kk * 2;
+                            a1[kk] = dA + so + kSlabD + kk * 2;
+                            bd[kk] = db0 + so + kk * bstep;
+                        }
+                        umma_ktile_pair(tmem, tmem + 256, a0, a1, bd, idesc, it > 0 ? 1u : 0u);
+                        umma_commit_pair(empty(j), 0x3);
+                    }
+                }
+            }
+            // extension k-tiles (the adapter product)
+            for (int it = p.nk; it < total && ok; ++it) {
                 const uint32_t s = it & (kStages - 1);
                 ok = mbar_wait_cluster(full_a(s), (it / kStages) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint64_t so = (uint64_t)(s * kStageD);
                 const uint32_t acc0 = it > 0 ? 1u : 0u;
-                if (it < p.nk) {
-                    const uint64_t db = (fwd ? dBk : dBm) + so;
-                    const uint32_t idesc = fwd ? id_k : id_mn;
-                    const uint32_t bstep = fwd ? 2u : 128u;
+                const int rem = p.r - (it - p.nk) * 64;
+                const int nsteps = rem >= 64 ? 4 : (rem + 15) / 16;
+                const uint64_t db = (fwd ? dBm : dBk) + so;
+                const uint32_t idesc = fwd ? id_mn : id_k;
+                const uint32_t bstep = fwd ? 128u : 2u;
+                for (int kk = 0; kk < nsteps; ++kk)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            umma_bf16_pair(tmem + h * 256, dA + so + h * kSlabD + kk * 2, db + kk * bstep, idesc,
-                                           kk > 0 ? 1u : acc0);
-                } else {
-                    const int rem = p.r - (it - p.nk) * 64;
-                    const int nsteps = rem >= 64 ? 4 : (rem + 15) / 16;
-                    const uint64_t db = (fwd ? dBm : dBk) + so;
-                    const uint32_t idesc = fwd ? id_mn : id_k;
-                    const uint32_t bstep = fwd ? 128u : 2u;
-                    for (int kk = 0; kk < nsteps; ++kk)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            umma_bf16_pair(tmem + h * 256, dA + so + h * kSlabD + kk * 2, db + kk * bstep, idesc,
-                                           kk > 0 ? 1u : acc0);
-                }
+                    for (int h = 0; h < 2; ++h)
+                        umma_bf16_pair(tmem + h * 256, dA + so + h * kSlabD + kk * 2, db + kk * bstep, idesc,
+                                       kk > 0 ? 1u : acc0);
                 umma_commit_pair(empty(s), 0x3);
             }
             if (ok) umma_commit_pair(acc_bar, 0x3);
