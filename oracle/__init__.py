@@ -59,6 +59,10 @@ def _L():
         lib.orc_nf4_codebook.argtypes = [ctypes.c_double, P]
         lib.orc_fp4_codebook.restype = None
         lib.orc_fp4_codebook.argtypes = [P]
+        lib.orc_e4m3_value.restype = ctypes.c_double
+        lib.orc_e4m3_value.argtypes = [ctypes.c_int]
+        lib.orc_e4m3_encode.restype = ctypes.c_int
+        lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
         lib.orc_quantize.restype = ctypes.c_int
         lib.orc_quantize.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P, P, P,
                                      P]
@@ -127,10 +131,21 @@ def fp4_codebook() -> np.ndarray:
     return out
 
 
+def e4m3_value(code: int) -> float:
+    """The value of an E4M3 code with the sign bit clear (0 .. 0x7E)."""
+    return float(_L().orc_e4m3_value(int(code)))
+
+
+def e4m3_encode(x: float) -> int:
+    """The E4M3 code nearest to x >= 0 (ties to the even mantissa; >= 448 -> 448)."""
+    return int(_L().orc_e4m3_encode(float(x)))
+
+
 # Double-quantization codes of the first-level scales: the unsigned 8-bit
-# code (step = max / 255), the signed INT8 absmax code (step = max / 127), and
-# the signed INT8 code of the scales minus their group mean.
-DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3}
+# code (step = max / 255), the signed INT8 absmax code (step = max / 127), the
+# signed INT8 code of the scales minus their group mean, and the 8-bit float
+# (E4M3) code (step = max / 448).
+DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3, "f8": 4}
 
 
 @dataclass

@@ -38,6 +38,7 @@
 #define ORC_DQ_U8 1     /* unsigned, step = max / 255, codes 0..255 */
 #define ORC_DQ_S8 2     /* signed INT8 absmax code of [CSDN] 4.1: step = max / 127, codes 0..127 */
 #define ORC_DQ_MEAN 3   /* signed INT8 code of a_b minus the group mean; one mean per group */
+#define ORC_DQ_F8 4     /* 8-bit float (E4M3) code of a_b / step, step = max / 448 */
 
 /* ------------------------------------------------------------------------ */
 /* bf16 <-> fp32 helpers (storage format of the inputs and of dequant out)  */
@@ -261,6 +262,32 @@ static void dq_group_mean(const float *a, int64_t n, uint8_t *codes, float *step
     }
 }
 
+/* The 8-bit float code of the scales.  [CSDN] 7.2 stores the first-level
+ * scales in 8 bits without naming the code; an 8-bit float is one of the
+ * readings.  Reading: the E4M3 layout (1 sign bit, 4 exponent bits biased by
+ * 7, 3 mantissa bits, no infinity; exponent field 0 holds the subnormals
+ * m * 2^-9, the largest finite value is 1.75 * 2^8 = 448).  Scales are >= 0,
+ * so the sign bit is clear: codes 0 .. 0x7E. */
+double orc_e4m3_value(int code) {
+    const int e = (code >> 3) & 15, m = code & 7;
+    if (e == 0) return ldexp((double)m, -9);
+    return ldexp(8.0 + (double)m, e - 10);
+}
+
+/* The E4M3 code nearest to x >= 0, ties to the even mantissa; x >= 448
+ * gives 448 (the format has no infinity). */
+int orc_e4m3_encode(double x) {
+    if (!(x > 0.0)) return 0;
+    if (x >= 448.0) return 0x7E;
+    if (x < ldexp(1.0, -6)) return (int)rint(ldexp(x, 9)); /* a rounded-up 8 is the smallest normal */
+    int e2;
+    (void)frexp(x, &e2);
+    const int e = e2 - 1;                                  /* 2^e <= x < 2^(e+1), e in -6..8 */
+    const double m = rint((ldexp(x, -e) - 1.0) * 8.0);     /* exact scaling; rint ties to even */
+    const int code = ((e + 7) << 3) + (int)m;              /* m = 8 carries into the exponent */
+    return code > 0x7E ? 0x7E : code;
+}
+
 /* Quantize Wt:[rows, cols] (fp32, row-major) in blocks of `block` weights
  * (64 by default; 32, 128 or 256 trade scale resolution against metadata,
  * [CSDN] 5.1).  The row-major flattening is cut into consecutive blocks; cols
@@ -316,6 +343,21 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const fl
                 dq_group_mean(a_all + b0, b1 - b0, codes + b0, steps + g, offsets + g);
                 continue;
             }
+            if (dq == ORC_DQ_F8) {
+                /* step f = RN32(max / 448), the largest code's value; each
+                 * scale's quotient is rounded to fp32 first, then to the
+                 * nearest E4M3 value: code = E4M3(RN32(a_b / f)). */
+                float mx = 0.0f;
+                for (int64_t b = b0; b < b1; ++b)
+                    if (a_all[b] > mx) mx = a_all[b];
+                const float f = (float)((double)mx / 448.0);
+                steps[g] = f;
+                for (int64_t b = b0; b < b1; ++b) {
+                    const float qf = f > 0.0f ? (float)((double)a_all[b] / (double)f) : 0.0f;
+                    codes[b] = (uint8_t)orc_e4m3_encode((double)qf);
+                }
+                continue;
+            }
             /* the top code: 255 for the unsigned code, 127 for the signed
              * INT8 code of [CSDN] 4.1 (absmax values are >= 0, so only its
              * codes 0..127 occur) */
@@ -350,7 +392,8 @@ int orc_quantize(const float *W, int64_t rows, int64_t cols, int block, const fl
 /* Decoded first-level scale of block b: a_b itself, or with double
  * quantization RN32(code_b * f_g) -- the product is exact in fp64 and is
  * rounded once to fp32 -- or, for the mean-offset variant with a signed
- * code, RN32(mu_g + RN32(code_b * f_g)). */
+ * code, RN32(mu_g + RN32(code_b * f_g)), or for the 8-bit float code
+ * RN32(E4M3(code_b) * f_g). */
 static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
                          const uint8_t *codes, const float *steps, const float *offsets) {
     if (!dq) return absmax[b];
@@ -359,6 +402,7 @@ static float block_scale(int64_t b, int dq, int dq_group, const float *absmax,
         const float d = (float)((double)(int8_t)codes[b] * (double)steps[g]);
         return (float)((double)offsets[g] + (double)d);
     }
+    if (dq == ORC_DQ_F8) return (float)(orc_e4m3_value(codes[b]) * (double)steps[g]);
     return (float)((double)codes[b] * (double)steps[g]);
 }
 

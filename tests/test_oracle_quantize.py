@@ -456,9 +456,9 @@ def test_dequantize_compute_dtypes(orc, block):
 # ---------------------------------------------------------------- double-quant variants
 # The pages give double quantization's structure (8-bit first-level scales,
 # one fp32 constant per 256; CSDN 7.2) but no 8-bit code.  Besides the
-# unsigned code above, two variants: the signed INT8 absmax code of CSDN 4.1
-# (s = 127 / max|x|) applied to the scales, and a code of the scales minus
-# their group mean.
+# unsigned code above, three variants: the signed INT8 absmax code of CSDN 4.1
+# (s = 127 / max|x|) applied to the scales, a code of the scales minus their
+# group mean, and an 8-bit float (E4M3) code (pinned at the end of the file).
 
 def _rn32(fr):
     return rn32(fr)
@@ -543,3 +543,93 @@ def test_dq_variants_bits_per_parameter(orc):
     q_mean = orc.quantize(W, cb, double_quant=True, dq_variant="mean")
     assert 8 * q_s8.nbytes / n - 4 == 8 / 64 + 32 / (64 * 256)
     assert 8 * q_mean.nbytes / n - 4 == 8 / 64 + 64 / (64 * 256)
+
+
+# --------------------------------------------------------------------------- 8-bit float scale code
+def _e4m3_values_torch():
+    """The 127 non-negative E4M3 values, decoded by torch's own float8_e4m3fn
+    type (an implementation independent of the oracle)."""
+    import torch
+    codes = torch.arange(0, 127, dtype=torch.uint8)
+    return [float(v) for v in codes.view(torch.float8_e4m3fn).float()]
+
+
+def test_e4m3_values_match_torch_float8(orc):
+    """The oracle's E4M3 decode agrees with torch's float8_e4m3fn on every
+    non-negative code, and the values have the format's structure: strictly
+    increasing with the code, 0 and 2^-9 at the bottom, 448 at the top,
+    eight equal steps per binade, the subnormal step equal to the first
+    normal binade's."""
+    want = _e4m3_values_torch()
+    got = [orc.e4m3_value(c) for c in range(127)]
+    assert got == want
+    assert all(b > a for a, b in zip(got, got[1:]))
+    assert got[0] == 0.0 and got[1] == 2.0 ** -9 and got[126] == 448.0
+    for e in range(1, 16):                      # each binade [2^(e-7), 2^(e-6))
+        vals = got[8 * e: 8 * e + 8]
+        steps = {Fr(b) - Fr(a) for a, b in zip(vals, vals[1:])}
+        assert steps == {Fr(vals[0]) / 8}
+    assert {Fr(b) - Fr(a) for a, b in zip(got[:9], got[1:9])} == {Fr(2) ** -9}
+
+
+def test_e4m3_encode_nearest_ties_even(orc):
+    """Encode = the nearest value, ties to the even code, by brute force in
+    exact arithmetic and against torch's float32 -> float8_e4m3fn rounding;
+    every midpoint between neighbours and one float either side of it;
+    quotients just above 448 saturate to 448."""
+    import torch
+    vals = _e4m3_values_torch()
+    fr = [Fr(v) for v in vals]
+
+    def brute(x):
+        X = Fr(float(x))
+        return min(range(127), key=lambda c: (abs(fr[c] - X), c & 1))
+
+    xs = [np.float32(v) for v in vals]
+    for a, b in zip(vals, vals[1:]):
+        mid = np.float32((a + b) / 2)
+        xs += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9))]
+    rng = np.random.default_rng(31)
+    xs += list((rng.random(2000) * 448).astype(np.float32))
+    xs += list((2.0 ** rng.uniform(-12, 8.8, 2000)).astype(np.float32))
+    xs = [x for x in xs if x <= 448]
+    t = torch.tensor(np.array(xs, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).tolist()
+    for x, tc in zip(xs, t):
+        c = orc.e4m3_encode(float(x))
+        assert c == brute(x) == tc, (x, c, brute(x), tc)
+    for x in (448.0, float(np.nextafter(np.float32(448), np.float32(1e9))), 460.0, 1e6):
+        assert orc.e4m3_encode(x) == 0x7E
+
+
+def test_dq_f8_bruteforce(orc):
+    """Step RN32(max / 448); code = the E4M3 value nearest to RN32(a / step)
+    (ties to even), by brute force in exact arithmetic; decode
+    RN32(E4M3(code) * step); bits per parameter as the 8-bit integer codes."""
+    rng = np.random.default_rng(24)
+    cb = orc.nf4_codebook()
+    am = np.abs(rng.standard_normal(256 + 77) * 0.05).astype(np.float32)
+    am[5] = 0.0
+    am[9] = np.float32(1e-7)                       # far below the step: a subnormal code
+    q = orc.quantize(_dq_blocks(am), cb, double_quant=True, dq_variant="f8")
+    vals = [Fr(v) for v in _e4m3_values_torch()]
+    for g0 in (0, 256):
+        grp = am[g0:g0 + 256]
+        f = _rn32(Fr(float(np.max(grp))) / 448)
+        assert q.steps[g0 // 256] == f
+        ff = Fr(float(f))
+        for i, a in enumerate(grp):
+            qf = Fr(float(_rn32(Fr(float(a)) / ff)))
+            want = min(range(127), key=lambda c: (abs(vals[c] - qf), c & 1))
+            assert q.codes[g0 + i] == want
+        assert q.codes[g0 + int(np.argmax(grp))] == 0x7E
+    assert q.codes[5] == 0
+    assert np.array_equal(q.packed, orc.quantize(_dq_blocks(am), cb, double_quant=False).packed)
+    deq = orc.dequantize(q, cb).reshape(-1)
+    idx = unpack(q.packed, deq.size)
+    for e in range(0, deq.size, 11):
+        b = e // BLOCK
+        ah = _rn32(vals[int(q.codes[b])] * Fr(float(q.steps[b // 256])))
+        assert deq[e] == bf16_of_f32(_rn32(Fr(float(ah)) * Fr(float(cb[idx[e]]))))
+    W = (rng.standard_normal((256, 4096)) * 0.02).astype(np.float32)
+    assert 8 * orc.quantize(W, cb, double_quant=True, dq_variant="f8").nbytes / W.size - 4 == \
+        8 / 64 + 32 / (64 * 256)
