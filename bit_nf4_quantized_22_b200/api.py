@@ -18,7 +18,7 @@ from .codebook import nf4_codebook
 BLOCK = 64
 DQ_GROUP = 256
 # double-quantization codes of the block scales (QLORA_DQ_* in qlora.h)
-DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3}
+DQ_VARIANTS = {"u8": 1, "s8": 2, "mean": 3, "f8": 4}
 
 
 def _ptr(t: torch.Tensor | None):
@@ -55,7 +55,7 @@ class NF4Weight:
     codes: torch.Tensor | None = None      # uint8 [nb] (int8 two's complement for "mean")
     steps: torch.Tensor | None = None      # fp32 [ceil(nb/256)]
     block: int = BLOCK                     # weights per first-level scale (32, 64, 128, 256)
-    dq_variant: str = "u8"                 # code of the scales: "u8", "s8" or "mean"
+    dq_variant: str = "u8"                 # code of the scales: "u8", "s8", "mean" or "f8"
     means: torch.Tensor | None = None      # fp32 [ceil(nb/256)] group means ("mean")
     # the layer calls' 16-bit dtype (x, A, B, dY, y, dX, merged weight)
     compute_dtype: torch.dtype = torch.bfloat16
@@ -112,7 +112,7 @@ def quantize(W: torch.Tensor, double_quant: bool = True, codebook: torch.Tensor 
              compute_dtype: torch.dtype = torch.bfloat16) -> NF4Weight:
     """nf4_quantize on W (fp32 [Dout, Din], CUDA) in blocks of `block` weights
     (32, 64, 128 or 256; the layer calls need 64); with double quantization
-    the block scales take the `dq_variant` code ("u8", "s8" or "mean").
+    the block scales take the `dq_variant` code ("u8", "s8", "mean" or "f8").
     `compute_dtype` (bf16 or fp16) is the dtype the layer calls then use."""
     _need(W, torch.float32, "W", 2)
     if compute_dtype not in (torch.bfloat16, torch.float16):

@@ -97,7 +97,7 @@ int check_weight(const nf4_weight_t *q, bool need_rows, bool codec = false) {
         if (q->cols % 64 != 0) return QLORA_EINVAL;
         if (q->block != 64) return QLORA_EUNSUPPORTED;
     }
-    if (q->double_quant < QLORA_DQ_NONE || q->double_quant > QLORA_DQ_MEAN) return QLORA_EINVAL;
+    if (q->double_quant < QLORA_DQ_NONE || q->double_quant > QLORA_DQ_F8) return QLORA_EINVAL;
     if (q->compute_dtype != QLORA_DTYPE_BF16 && q->compute_dtype != QLORA_DTYPE_FP16) return QLORA_EINVAL;
     if (q->rows * q->cols == 0) return QLORA_OK;
     if (!q->packed || !aligned16(q->packed)) return QLORA_EINVAL;

@@ -28,8 +28,16 @@ struct ScaleSrc {
     const float *mean;        // when dq == 3
 };
 
+// The value of an E4M3 code with the sign bit clear (QLORA_DQ_F8): exponent
+// field e, mantissa m; e = 0 holds the subnormals m * 2^-9.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : __fmul_rn((float)m, 0x1p-9f);
+}
+
 __device__ __forceinline__ float dq_decode(uint32_t code, float step, float mean, int dq) {
     if (dq == 3) return __fadd_rn(mean, __fmul_rn((float)(int8_t)(uint8_t)code, step));
+    if (dq == 4) return __fmul_rn(e4m3_value(code), step);
     return __fmul_rn((float)code, step);
 }
 

@@ -106,6 +106,23 @@ __device__ __forceinline__ int dq_code(float d, float f, int top) {
     return (int)fminf(fmaxf(c, -(float)top), (float)top);
 }
 
+// The E4M3 code nearest to x >= 0 (QLORA_DQ_F8): ties to the even code, 448
+// (code 0x7E) for x >= 448.  Below 2^-6 the subnormal code is RNE(x * 2^9)
+// (a power-of-two scaling, exact; 8 is also the smallest normal's code); above,
+// the fp32 mantissa is rounded to 3 bits, the carry of m = 8 moving into the
+// exponent field.
+__device__ __forceinline__ uint32_t e4m3_encode(float x) {
+    if (!(x > 0.f)) return 0u;
+    if (x >= 448.f) return 0x7Eu;
+    if (x < 0x1p-6f) return (uint32_t)rintf(__fmul_rn(x, 512.f));
+    const uint32_t u = __float_as_uint(x);
+    const uint32_t mant = u & 0x7FFFFFu, rem = mant & 0xFFFFFu;
+    uint32_t q = mant >> 20;
+    q += (rem > 0x80000u || (rem == 0x80000u && (q & 1u))) ? 1u : 0u;
+    const uint32_t code = (((u >> 23) - 120u) << 3) + q;
+    return code > 0x7Eu ? 0x7Eu : code;
+}
+
 // Double quantization of one group of first-level scales, one per thread of
 // the CTA (a, valid for the first nvalid threads): writes the step, the
 // codes and, for the mean-offset code, the group mean (the rules of
@@ -138,14 +155,18 @@ __device__ __forceinline__ void dq_group_encode(float a, bool valid, int nvalid,
 #pragma unroll
     for (int i = 1; i < kThreads / 32; ++i) gm = fmaxf(gm, warp_max[i]);
     const int top = dq == QLORA_DQ_U8 ? 255 : 127;
-    const float f = __fdiv_rn(gm, (float)top);
+    const float f = __fdiv_rn(gm, dq == QLORA_DQ_F8 ? 448.f : (float)top);
     if (threadIdx.x == 0) {
         *step_out = f;
         if (dq == QLORA_DQ_MEAN) *mean_out = mu;
     }
     if (valid) {
-        const float d = dq == QLORA_DQ_MEAN ? __fsub_rn(a, mu) : a;
-        *code_out = (uint8_t)(int8_t)dq_code(d, f, top);
+        if (dq == QLORA_DQ_F8) {
+            *code_out = (uint8_t)(f > 0.f ? e4m3_encode(__fdiv_rn(a, f)) : 0u);
+        } else {
+            const float d = dq == QLORA_DQ_MEAN ? __fsub_rn(a, mu) : a;
+            *code_out = (uint8_t)(int8_t)dq_code(d, f, top);
+        }
     }
 }
 

@@ -79,7 +79,13 @@ extern "C" {
  *                  fp64 sum of the group's scales in block order; d = RN32(a - mu);
  *                  f = RN32(max |d| / 127); code = round-half-even(d / f) in
  *                  -127..127 stored as int8; one mu per group in dq_mean
- * Decoded scale: RN32(code * f), or RN32(mu + RN32(code * f)) for QLORA_DQ_MEAN.
+ *   QLORA_DQ_F8    an 8-bit float code: the E4M3 layout (1 sign, 4 exponent
+ *                  bits biased by 7, 3 mantissa bits; no infinity, largest
+ *                  finite value 448, subnormals m * 2^-9); f = RN32(group max /
+ *                  448), code = the E4M3 value nearest to RN32(a / f), ties to
+ *                  the even code, 448 for quotients above it; codes 0..0x7E
+ * Decoded scale: RN32(code * f), RN32(mu + RN32(code * f)) for QLORA_DQ_MEAN,
+ * RN32(E4M3(code) * f) for QLORA_DQ_F8.
  * The weights themselves are encoded with the exact block absmax. */
 /* Compute dtypes (bitsandbytes article (CSDN) 8.3: the dequantized weight
  * and the arithmetic are FP32, BF16 or FP16; 8.5 on FP16's narrower range).
@@ -93,6 +99,7 @@ extern "C" {
 #define QLORA_DQ_U8 1
 #define QLORA_DQ_S8 2
 #define QLORA_DQ_MEAN 3
+#define QLORA_DQ_F8 4
 
 /* One quantized weight Wt:[rows = Dout, cols = Din]; nb = rows*cols/block.
  *   packed      [rows*cols/2] uint8   two 4-bit codebook indices per byte;
@@ -106,7 +113,7 @@ typedef struct {
     int64_t rows;
     int64_t cols;
     int32_t block;          /* 64; the codec calls also take 32, 128, 256 */
-    int32_t double_quant;   /* QLORA_DQ_NONE, _U8, _S8 or _MEAN */
+    int32_t double_quant;   /* QLORA_DQ_NONE, _U8, _S8, _MEAN or _F8 */
     int32_t dq_group;       /* must be 256 when double_quant != 0 */
     int32_t compute_dtype;  /* QLORA_DTYPE_BF16 or _FP16: the layer calls' 16-bit arrays */
     uint8_t *packed;

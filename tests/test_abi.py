@@ -64,10 +64,10 @@ def _wc(rows=64, cols=128, dq=1, block=64, group=256, ptrs=True):
 
 
 def test_dq_variant_validation(lib):
-    """double_quant is a code kind 0..3; the mean-offset kind needs dq_mean."""
+    """double_quant is a code kind 0..4; the mean-offset kind needs dq_mean."""
     cb = _cb(q.nf4_codebook().tolist())
     W = ctypes.c_void_p(1 << 20)
-    for bad in (-1, 4):
+    for bad in (-1, 5):
         assert lib.nf4_quantize(W, ctypes.byref(_wc(dq=bad)), cb, None, None) == _lib.QLORA_EINVAL
     wc = _wc(dq=3)
     wc.dq_mean = None

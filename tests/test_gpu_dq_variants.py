@@ -1,7 +1,8 @@
 """Double-quantization variants on the GPU against the oracle (bitsandbytes
 article (CSDN) 7.2 gives the structure, not the 8-bit code; 4.1 gives the
-symmetric INT8 absmax code): the signed INT8 code (step = group max / 127)
-and the code of the scales minus their group mean.  Quantize and dequantize
+symmetric INT8 absmax code): the signed INT8 code (step = group max / 127),
+the code of the scales minus their group mean, and the 8-bit float (E4M3)
+code (step = group max / 448).  Quantize and dequantize
 are bit-exact (packed indices, codes, steps, means, bf16 weights); the layer
 and the merge are within the parity tolerance."""
 import numpy as np
@@ -14,7 +15,7 @@ from bit_nf4_quantized_22_b200.synth import LinearSpec
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ["s8", "mean"]
+VARIANTS = ["s8", "mean", "f8"]
 
 
 def _check(orc, qlib, W, variant, block=64, cb=None):
@@ -83,3 +84,24 @@ def test_dq_variant_layer(orc, qlib, variant, M):
     register GEMVs); M = 260: the tcgen05 GEMM."""
     _layer(orc, qlib, LinearSpec("dqv", 2048, 1032, 16, 32.0, True), M, 41, variant)
     _layer(orc, qlib, LinearSpec("dqr", 1088, 264, 8, 16.0, True), M, 42, variant)
+
+
+def test_dq_f8_ties_and_subnormals(orc, qlib):
+    """The E4M3 scale code on quotients that sit exactly on midpoints between
+    neighbouring values (ties to the even code), one float either side of
+    them, in the subnormal range and at the top: group max 448 makes the
+    step exactly 1, so each quotient is the block absmax itself."""
+    import torch
+    vals = [float(v) for v in torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).float()]
+    a = [448.0]
+    for lo, hi in zip(vals, vals[1:]):
+        mid = np.float32((lo + hi) / 2)
+        a += [float(mid), float(np.nextafter(mid, np.float32(0))), float(np.nextafter(mid, np.float32(1e9)))]
+    rng = np.random.default_rng(3)
+    a += list(rng.uniform(0, 448, 384 - len(a)))          # 384 blocks: 24 rows of 16
+    a = np.array(a, np.float32)
+    blocks = (rng.uniform(-1, 1, (a.size, 64)) * a[:, None] * 0.9).astype(np.float32)
+    blocks[:, 11] = -a                                   # the block absmax is a
+    for g in range(0, a.size, 256):                      # every group's max is 448: step 1
+        blocks[g, 7] = 448.0
+    _check(orc, qlib, blocks.reshape(-1, 64 * 16), "f8")
