@@ -8,8 +8,10 @@ workload (Din=4096, Dout=11008, M=4096 tokens, r=64, alpha=128, W ~ t5*0.02).
 With N > 1 ranks each rank runs its own batch (weak scaling) and the adapter
 gradients dA, dB are summed over ranks with NCCL (the data-parallel exchange).
 
-Prints ONE JSON line on rank 0.  `--impl reference` times the CPU oracle
-(the only reference there is) on a bounded sample of the same workload.
+On one GPU each timed step is one replay of the step captured in a CUDA
+graph (`--eager` times eager calls).  Prints ONE JSON line on rank 0.
+`--impl reference` times the CPU oracle (the only reference there is) on a
+bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -351,6 +353,34 @@ def run_ours(args, rank, world, dist):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    import ctypes
+
+    # One GPU: the step is captured once in a CUDA graph (the library's
+    # per-kernel timing events become nodes of the graph) and each timed step
+    # is one replay of it -- the same kernels on the same buffers, without the
+    # host's launch gaps.  Several GPUs: eager steps (the NCCL exchange stays
+    # outside graph capture).
+    use_graph = world == 1 and not args.eager
+    graph, per_step_launches = None, 0
+    if use_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        lib.qlora_profile_reset()
+        lib.qlora_profile_enable(1)
+        step()                       # creates the library's timing events outside the capture
+        torch.cuda.synchronize()
+        lib.qlora_profile_reset()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        lib.qlora_profile_enable(0)
+        per_step_launches = lib.qlora_launch_count()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
 
     # ---------------- timed region: K steps, L2 flushed between steps
     uuid = None
@@ -360,30 +390,71 @@ def run_ours(args, rank, world, dist):
         pass
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    lib.qlora_profile_reset()
-    lib.qlora_profile_enable(1)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(uuid) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record()
-            step()
-            ends[i].record()
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    lib.qlora_profile_enable(0)
-    launches = lib.qlora_launch_count()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    import ctypes
     umma_n, umma_ms = ctypes.c_int64(), ctypes.c_double()
     quant_n, quant_ms = ctypes.c_int64(), ctypes.c_double()
-    lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
-    lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+    acc = {"umma_n": 0, "umma_ms": 0.0, "quant_n": 0, "quant_ms": 0.0}
+    if not use_graph:
+        lib.qlora_profile_reset()
+        lib.qlora_profile_enable(1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    def read_replay_events():
+        # the last replay's kernel events (the graph re-records the same events)
+        rc0 = lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
+        rc2 = lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+        if rc0 or rc2:
+            acc["failed"] = True
+        acc["umma_n"] += umma_n.value
+        acc["umma_ms"] += umma_ms.value
+        acc["quant_n"] += quant_n.value
+        acc["quant_ms"] += quant_ms.value
+
+    with ClockSampler(uuid) as clk:
+        for i in range(args.steps):
+            if use_graph and i > 0:
+                torch.cuda.synchronize()          # the previous replay has finished
+            flush.zero_()
+            if use_graph and i > 0:
+                read_replay_events()              # while the GPU flushes L2, outside the events
+            starts[i].record()
+            if use_graph:
+                graph.replay()
+            else:
+                step()
+            ends[i].record()
+        torch.cuda.synchronize()
+        if use_graph:
+            read_replay_events()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    kernel_timing = "library events inside the timed region"
+    if use_graph:
+        launches = per_step_launches * args.steps
+        umma_n.value, umma_ms.value = acc["umma_n"], acc["umma_ms"]
+        quant_n.value, quant_ms.value = acc["quant_n"], acc["quant_ms"]
+        del graph
+        if acc.get("failed"):
+            # the graph's timing events could not be read: the kernels' times
+            # come from the same number of eager steps right after
+            kernel_timing = "library events over an eager pass of the same steps"
+            lib.qlora_profile_reset()
+            lib.qlora_profile_enable(1)
+            for _ in range(args.steps):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
+            lib.qlora_profile_enable(0)
+            lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
+            lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+    else:
+        lib.qlora_profile_enable(0)
+        launches = lib.qlora_launch_count()
+        lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
+        lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -408,7 +479,7 @@ def run_ours(args, rank, world, dist):
             "traffic": traffic,
             "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'} ({peak_src})",
             "frac_of_sustained": (umma_tf / tf_sus) if umma_tf else None,
-            "launches": int(umma_n.value),
+            "launches": int(umma_n.value), "timing": kernel_timing,
             "share_of_step": umma_ms.value / sum(step_ms) if step_ms else None}
     qbytes = Din * Dout * 4 + weight_bytes(Din, Dout)
     quant = {"kernel": "k_nf4_quantize_fast", "bound": "hbm",
@@ -509,7 +580,9 @@ def run_ours(args, rank, world, dist):
         "data": "synthetic (seeded numpy PCG64; W~t5*0.02, x,dY~N(0,1), A~N(0,1/r), B~N(0,1e-4))",
         "config": {"workload": WORKLOAD, "M": M, "Din": Din, "Dout": Dout, "r": r, "alpha": alpha,
                    "double_quant": True, "parallelism": f"dp{world}",
-                   "l2": "flushed between timed steps (256 MB write, outside the step events)"},
+                   "l2": "flushed between timed steps (256 MB write, outside the step events)",
+                   "timing": ("each timed step one replay of the step captured in a CUDA graph"
+                              if use_graph else "eager steps")},
         "roofline": roof,
         "quantize_roofline": quant,
         "e2e": e2e,
@@ -877,11 +950,13 @@ def profile_case(cfg, lin, M):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager steps instead of replays of the captured step")
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--graph-replays", type=int, default=50)

@@ -49,6 +49,17 @@ cudaError_t set_max_smem(const void *fn, int bytes) {
     return e;
 }
 
+// Inside a stream capture a plain event record becomes a dependency inside the
+// graph, not a timestamp: record as an external event node, which each replay
+// of the graph records like cudaEventRecord would.
+static void record_timing_event(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, st);
+}
+
 void prof_begin(int kind, cudaStream_t st) {
     if (!g_on.load(std::memory_order_relaxed)) return;
     std::lock_guard<std::mutex> lk(g_mu);
@@ -60,7 +71,7 @@ void prof_begin(int kind, cudaStream_t st) {
         p.start.push_back(a);
         p.stop.push_back(b);
     }
-    cudaEventRecord(p.start[p.used], st);
+    record_timing_event(p.start[p.used], st);
 }
 
 void prof_end(int kind, cudaStream_t st) {
@@ -68,7 +79,7 @@ void prof_end(int kind, cudaStream_t st) {
     std::lock_guard<std::mutex> lk(g_mu);
     Pairs &p = g_pairs[kind];
     if (p.used < p.start.size()) {
-        cudaEventRecord(p.stop[p.used], st);
+        record_timing_event(p.stop[p.used], st);
         ++p.used;
     }
 }
@@ -93,9 +104,12 @@ int qlora_profile_read(int32_t kind, int64_t *launches, double *total_ms) {
     auto &p = qlora::g_pairs[kind];
     double t = 0.0;
     for (size_t i = 0; i < p.used; ++i) {
-        if (cudaEventSynchronize(p.stop[i]) != cudaSuccess) return QLORA_ECUDA;
         float ms = 0.f;
-        if (cudaEventElapsedTime(&ms, p.start[i], p.stop[i]) != cudaSuccess) return QLORA_ECUDA;
+        if (cudaEventSynchronize(p.stop[i]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, p.start[i], p.stop[i]) != cudaSuccess) {
+            (void)cudaGetLastError();   // a failed readout must not fail the next launch check
+            return QLORA_ECUDA;
+        }
         t += ms;
     }
     *launches = (int64_t)p.used;
