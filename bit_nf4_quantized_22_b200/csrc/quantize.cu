@@ -286,6 +286,11 @@ k_nf4_quantize(const __grid_constant__ CUtensorMap tW, int64_t nb, ThreshPairs t
 // threshold; only then is this kernel used, and the one compare is exact.
 // Blocks with a = 0, a tiny or huge a, or a non-finite weight take the
 // branch-free search (warp-uniform branch).
+// Every lane addresses its weights and packed bytes from two base pointers
+// with constant offsets, and a full group (256 blocks, all but the last one)
+// runs a copy of the loop without the per-block range tests: about 10% fewer
+// issued instructions on this issue-bound kernel.
+template <bool B> struct BoolTag { static constexpr bool value = B; };
 constexpr float kBinK = 15.49f;
 constexpr float kBinC = 12582928.0f;   // 1.5 * 2^23 + 16: the low 5 bits of the sum are the bin
 constexpr int kQfThreads = 256;
@@ -321,90 +326,101 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Qua
     const double hk = s_half[j < 15 ? j : 14];
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
-    // the loads of quarter c + 1 are issued before quarter c is decided
-    float nxt[4][V];
-    auto load_quarter = [&](int c, float (&dst)[4][V]) {
+    // this lane's weights and packed bytes of block bl = 64 c + 16 i + 2 warp + half
+    // are at constant offsets (c, i) from these
+    const float *wlane = W + (b0 + 2 * warp + half) * (16 * V) + V * j;
+    uint8_t *plane = packed + (b0 + 2 * warp + half) * (8 * V) + (V / 2) * j;
+    auto run = [&](auto tag) {
+        constexpr bool FULL = decltype(tag)::value;
+        float nxt[4][V];
+        auto load_quarter = [&](int c, float (&dst)[4][V]) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int bl = 64 * c + 2 * (warp + 8 * i) + half;
-            const float *src = W + (b0 + bl) * (16 * V) + V * j;
-            if (V == 4) {
-                const float4 v = (c < 4 && bl < nblk) ? __ldcs(reinterpret_cast<const float4 *>(src))
-                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                dst[i][0] = v.x, dst[i][1] = v.y, dst[i][2] = v.z, dst[i][3] = v.w;
-            } else {
-                const float2 v = (c < 4 && bl < nblk) ? __ldcs(reinterpret_cast<const float2 *>(src))
-                                                      : make_float2(0.f, 0.f);
-                dst[i][0] = v.x, dst[i][1] = v.y;
+            for (int i = 0; i < 4; ++i) {
+                const int bl = 64 * c + 16 * i + 2 * warp + half;
+                const float *src = wlane + (64 * c + 16 * i) * (16 * V);
+                const bool ld = FULL || bl < nblk;
+                if (V == 4) {
+                    const float4 v = ld ? __ldcs(reinterpret_cast<const float4 *>(src))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    dst[i][0] = v.x, dst[i][1] = v.y, dst[i][2] = v.z, dst[i][3] = v.w;
+                } else {
+                    const float2 v = ld ? __ldcs(reinterpret_cast<const float2 *>(src)) : make_float2(0.f, 0.f);
+                    dst[i][0] = v.x, dst[i][1] = v.y;
+                }
+            }
+        };
+        load_quarter(0, nxt);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            if (!FULL && 64 * c >= nblk) break;
+            float pre[4][V];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < V; ++k) pre[i][k] = nxt[i][k];
+            if (c + 1 < 4 && (FULL || 64 * (c + 1) < nblk)) load_quarter(c + 1, nxt);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int bl = 64 * c + 16 * i + 2 * warp + half;   // block within the group
+                const bool valid = FULL || bl < nblk;
+                float w[V];
+#pragma unroll
+                for (int k = 0; k < V; ++k) w[k] = pre[i][k];
+                // max |w|, NaN-propagating: a NaN or Inf weight makes a non-finite scale
+                float fm = 0.f;
+#pragma unroll
+                for (int k = 0; k < V; ++k) asm("max.NaN.f32 %0, %1, %2;" : "=f"(fm) : "f"(fm), "f"(fabsf(w[k])));
+                const uint32_t m = __float_as_uint(fm);
+                const uint32_t m0 = __reduce_max_sync(0xffffffffu, half ? 0u : m);
+                const uint32_t m1 = __reduce_max_sync(0xffffffffu, half ? m : 0u);
+                const uint32_t ab = half ? m1 : m0;
+                const float a = __uint_as_float(ab);
+                const bool bad = ab >= 0x7f800000u;
+                // tau_j: the smallest fp32 above the exact midpoint h_j * a
+                float tau;
+                if (kExactHalf)
+                    tau = next_up(__double2float_rd(__dmul_rn(hk, (double)a)));
+                else
+                    tau = exact_threshold(c_lo, c_hi, a);
+                if (j == 15) tau = __uint_as_float(0x7f800000u);
+                const bool fast = ab >= 0x0d800000u && ab <= 0x71800000u;   // 2^-100 <= a <= 2^100
+                uint32_t qv[V];
+                if (__all_sync(0xffffffffu, fast || !valid)) {
+                    const float kr = __fmul_rn(kBinK, rcp_approx(a));   // K / a, relative error < 2^-22
+#pragma unroll
+                    for (int k = 0; k < V; ++k) {
+                        const float y = fmaf(w[k], kr, kBinC);
+                        const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
+                        const float t = __shfl_sync(0xffffffffu, tau, (int)jt, 16);
+                        qv[k] = jt + (w[k] >= t ? 1u : 0u);
+                    }
+                } else {
+                    float t[15];
+#pragma unroll
+                    for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k, 16);
+#pragma unroll
+                    for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[k], t);
+                }
+                if (valid) {
+                    // weights V j .. V j + V-1 -> bytes (V/2) j ..; element 2i in the high nibble
+                    uint8_t *dstp = plane + (64 * c + 16 * i) * (8 * V);
+                    if (V == 4) {
+                        const uint32_t v = (qv[2 % V] * 16u + qv[3 % V]) * 256u + (qv[0] * 16u + qv[1]);
+                        *reinterpret_cast<uint16_t *>(dstp) = (uint16_t)v;
+                    } else {
+                        *dstp = (uint8_t)(qv[1] | (qv[0] << 4));
+                    }
+                    if (j == 0) {
+                        s_a[bl] = a;
+                        if (!dq) absmax[b0 + bl] = a;
+                        bad_any |= bad;
+                    }
+                }
             }
         }
     };
-    load_quarter(0, nxt);
-    for (int c = 0; c < 4 && 64 * c < nblk; ++c) {
-        float pre[4][V];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int k = 0; k < V; ++k) pre[i][k] = nxt[i][k];
-        if (c + 1 < 4 && 64 * (c + 1) < nblk) load_quarter(c + 1, nxt);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int bl = 64 * c + 2 * (warp + 8 * i) + half;   // block within the group
-            const bool valid = bl < nblk;
-            float w[V];
-#pragma unroll
-            for (int k = 0; k < V; ++k) w[k] = pre[i][k];
-            // max |w|, NaN-propagating: a NaN or Inf weight makes a non-finite scale
-            float fm = 0.f;
-#pragma unroll
-            for (int k = 0; k < V; ++k) asm("max.NaN.f32 %0, %1, %2;" : "=f"(fm) : "f"(fm), "f"(fabsf(w[k])));
-            const uint32_t m = __float_as_uint(fm);
-            const uint32_t m0 = __reduce_max_sync(0xffffffffu, half ? 0u : m);
-            const uint32_t m1 = __reduce_max_sync(0xffffffffu, half ? m : 0u);
-            const uint32_t ab = half ? m1 : m0;
-            const float a = __uint_as_float(ab);
-            const bool bad = ab >= 0x7f800000u;
-            // tau_j: the smallest fp32 above the exact midpoint h_j * a
-            float tau;
-            if (kExactHalf)
-                tau = next_up(__double2float_rd(__dmul_rn(hk, (double)a)));
-            else
-                tau = exact_threshold(c_lo, c_hi, a);
-            if (j == 15) tau = __uint_as_float(0x7f800000u);
-            const bool fast = ab >= 0x0d800000u && ab <= 0x71800000u;   // 2^-100 <= a <= 2^100
-            uint32_t qv[V];
-            if (__all_sync(0xffffffffu, fast || !valid)) {
-                const float kr = __fmul_rn(kBinK, rcp_approx(a));   // K / a, relative error < 2^-22
-#pragma unroll
-                for (int k = 0; k < V; ++k) {
-                    const float y = fmaf(w[k], kr, kBinC);
-                    const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
-                    const float t = __shfl_sync(0xffffffffu, tau, (int)jt, 16);
-                    qv[k] = jt + (w[k] >= t ? 1u : 0u);
-                }
-            } else {
-                float t[15];
-#pragma unroll
-                for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k, 16);
-#pragma unroll
-                for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[k], t);
-            }
-            if (valid) {
-                // weights V j .. V j + V-1 -> bytes (V/2) j ..; element 2i in the high nibble
-                if (V == 4) {
-                    const uint32_t v = (qv[2 % V] * 16u + qv[3 % V]) * 256u + (qv[0] * 16u + qv[1]);
-                    *reinterpret_cast<uint16_t *>(packed + (b0 + bl) * 32 + 2 * j) = (uint16_t)v;
-                } else {
-                    packed[(b0 + bl) * 16 + j] = (uint8_t)(qv[1] | (qv[0] << 4));
-                }
-                if (j == 0) {
-                    s_a[bl] = a;
-                    if (!dq) absmax[b0 + bl] = a;
-                    bad_any |= bad;
-                }
-            }
-        }
-    }
+    if (nblk == 256) run(BoolTag<true>{});
+    else run(BoolTag<false>{});
     if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
     if (dq) {
         __shared__ float s_mu;
@@ -424,7 +440,9 @@ k_nf4_quantize_fast(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Qua
 // article's section 5.1 trade of scale resolution against metadata).  One
 // CTA per double-quant group of 256 blocks; warp w takes blocks w, w + 8, ...
 // of the group, one whole block per warp with V weights per lane, four
-// blocks' loads issued together.  The decision per weight is the fast
+// blocks' loads issued together (for V <= 4 the next four blocks' loads are
+// issued before these four are decided; a full group runs a copy of the loop
+// without range tests).  The decision per weight is the fast
 // kernel's (bin table, one exact compare against tau_j held by lane j) when
 // the table is usable and a lies in [2^-100, 2^100], else the branch-free
 // search; packing, absmax and double quantization as in the other kernels.
@@ -463,81 +481,180 @@ k_nf4_quantize_blk(const float *__restrict__ W, int64_t nb, ThreshPairs tp, Quan
     const double hk = s_half[j];
     const uint32_t lut = s_lut[lane];
     uint32_t bad_any = 0;
-    for (int c = 0; 8 * kQbUnroll * c < nblk; ++c) {
-        float w[kQbUnroll][V];
+    auto run = [&](auto tag) {
+        constexpr bool FULL = decltype(tag)::value;
+        constexpr int NC = 256 / (8 * kQbUnroll);
+        float nxt[kQbUnroll][V];
+        auto load_chunk = [&](int c, float (&w)[kQbUnroll][V]) {
 #pragma unroll
-        for (int i = 0; i < kQbUnroll; ++i) {
-            const int bl = 8 * (kQbUnroll * c + i) + warp;
-            const float *src = W + (b0 + bl) * B;
-            if (bl < nblk) {
+            for (int i = 0; i < kQbUnroll; ++i) {
+                const int bl = 8 * (kQbUnroll * c + i) + warp;
+                const float *src = W + (b0 + bl) * B;
+                if (FULL || bl < nblk) {
+                    if (V == 1) {
+                        w[i][0] = __ldcs(src + lane);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < V / 4; ++h) {
+                            const float4 v = __ldcs(reinterpret_cast<const float4 *>(src + 128 * h) + lane);
+                            w[i][4 * h] = v.x, w[i][4 * h + 1] = v.y, w[i][4 * h + 2] = v.z, w[i][4 * h + 3] = v.w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < V; ++k) w[i][k] = 0.f;
+                }
+            }
+        };
+        load_chunk(0, nxt);
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            if (!FULL && 8 * kQbUnroll * c >= nblk) break;
+            float w[kQbUnroll][V];
+#pragma unroll
+            for (int i = 0; i < kQbUnroll; ++i)
+#pragma unroll
+                for (int k = 0; k < V; ++k) w[i][k] = nxt[i][k];
+            if (c + 1 < NC && (FULL || 8 * kQbUnroll * (c + 1) < nblk)) load_chunk(c + 1, nxt);
+#pragma unroll
+            for (int i = 0; i < kQbUnroll; ++i) {
+                const int bl = 8 * (kQbUnroll * c + i) + warp;
+                if (!FULL && bl >= nblk) break;                  // warp-uniform
+                // max |w| on the bit patterns: NaN and Inf sort above every finite value
+                uint32_t m = 0;
+#pragma unroll
+                for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[i][k]) & 0x7fffffffu);
+                const uint32_t ab = __reduce_max_sync(0xffffffffu, m);
+                const float a = __uint_as_float(ab);
+                float tau = kExactHalf ? next_up(__double2float_rd(__dmul_rn(hk, (double)a)))
+                                       : exact_threshold(c_lo, c_hi, a);
+                if (lane >= 15) tau = __uint_as_float(0x7f800000u);
+                const bool fast = use_bins && ab >= 0x0d800000u && ab <= 0x71800000u;   // warp-uniform
+                uint32_t qv[V];
+                if (fast) {
+                    const float kr = __fmul_rn(kBinK, rcp_approx(a));
+#pragma unroll
+                    for (int k = 0; k < V; ++k) {
+                        const float y = fmaf(w[i][k], kr, kBinC);
+                        const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
+                        const float t = __shfl_sync(0xffffffffu, tau, (int)jt);
+                        qv[k] = jt + (w[i][k] >= t ? 1u : 0u);
+                    }
+                } else {
+                    float t[15];
+#pragma unroll
+                    for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k);
+#pragma unroll
+                    for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[i][k], t);
+                }
+                uint8_t *dst = packed + (b0 + bl) * (B / 2);
                 if (V == 1) {
-                    w[i][0] = __ldcs(src + lane);
+                    // even lane 2i: byte i = (q_2i << 4) | q_2i+1; lane 8k gathers bytes 4k .. 4k+3
+                    const uint32_t nx = __shfl_down_sync(0xffffffffu, qv[0], 1);
+                    const uint32_t byte = ((qv[0] << 4) | nx) & 0xffu;
+                    const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 2);
+                    const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 4);
+                    const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 6);
+                    if ((lane & 7) == 0)
+                        *reinterpret_cast<uint32_t *>(dst + lane / 2) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
                 } else {
 #pragma unroll
                     for (int h = 0; h < V / 4; ++h) {
-                        const float4 v = __ldcs(reinterpret_cast<const float4 *>(src + 128 * h) + lane);
-                        w[i][4 * h] = v.x, w[i][4 * h + 1] = v.y, w[i][4 * h + 2] = v.z, w[i][4 * h + 3] = v.w;
+                        const uint32_t v = qv[4 * h + 1] | (qv[4 * h] << 4) | (qv[4 * h + 3] << 8) | (qv[4 * h + 2] << 12);
+                        *reinterpret_cast<uint16_t *>(dst + 64 * h + 2 * lane) = (uint16_t)v;
                     }
                 }
-            } else {
-#pragma unroll
-                for (int k = 0; k < V; ++k) w[i][k] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kQbUnroll; ++i) {
-            const int bl = 8 * (kQbUnroll * c + i) + warp;
-            if (bl >= nblk) break;                           // warp-uniform
-            // max |w| on the bit patterns: NaN and Inf sort above every finite value
-            uint32_t m = 0;
-#pragma unroll
-            for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[i][k]) & 0x7fffffffu);
-            const uint32_t ab = __reduce_max_sync(0xffffffffu, m);
-            const float a = __uint_as_float(ab);
-            float tau = kExactHalf ? next_up(__double2float_rd(__dmul_rn(hk, (double)a)))
-                                   : exact_threshold(c_lo, c_hi, a);
-            if (lane >= 15) tau = __uint_as_float(0x7f800000u);
-            const bool fast = use_bins && ab >= 0x0d800000u && ab <= 0x71800000u;   // warp-uniform
-            uint32_t qv[V];
-            if (fast) {
-                const float kr = __fmul_rn(kBinK, rcp_approx(a));
-#pragma unroll
-                for (int k = 0; k < V; ++k) {
-                    const float y = fmaf(w[i][k], kr, kBinC);
-                    const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
-                    const float t = __shfl_sync(0xffffffffu, tau, (int)jt);
-                    qv[k] = jt + (w[i][k] >= t ? 1u : 0u);
-                }
-            } else {
-                float t[15];
-#pragma unroll
-                for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k);
-#pragma unroll
-                for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[i][k], t);
-            }
-            uint8_t *dst = packed + (b0 + bl) * (B / 2);
-            if (V == 1) {
-                // even lane 2i: byte i = (q_2i << 4) | q_2i+1; lane 8k gathers bytes 4k .. 4k+3
-                const uint32_t nx = __shfl_down_sync(0xffffffffu, qv[0], 1);
-                const uint32_t byte = ((qv[0] << 4) | nx) & 0xffu;
-                const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 2);
-                const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 4);
-                const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 6);
-                if ((lane & 7) == 0)
-                    *reinterpret_cast<uint32_t *>(dst + lane / 2) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
-            } else {
-#pragma unroll
-                for (int h = 0; h < V / 4; ++h) {
-                    const uint32_t v = qv[4 * h + 1] | (qv[4 * h] << 4) | (qv[4 * h + 3] << 8) | (qv[4 * h + 2] << 12);
-                    *reinterpret_cast<uint16_t *>(dst + 64 * h + 2 * lane) = (uint16_t)v;
+                if (lane == 0) {
+                    s_a[bl] = a;
+                    if (!dq) absmax[b0 + bl] = a;
+                    bad_any |= ab >= 0x7f800000u;
                 }
             }
-            if (lane == 0) {
-                s_a[bl] = a;
-                if (!dq) absmax[b0 + bl] = a;
-                bad_any |= ab >= 0x7f800000u;
+        }
+    };
+    // blocks of 256: four blocks' loads (8 per lane) already keep enough bytes in
+    // flight; loading the next four ahead measured slower
+    if (V == 8) {
+        for (int c = 0; 8 * kQbUnroll * c < nblk; ++c) {
+            float w[kQbUnroll][V];
+#pragma unroll
+            for (int i = 0; i < kQbUnroll; ++i) {
+                const int bl = 8 * (kQbUnroll * c + i) + warp;
+                const float *src = W + (b0 + bl) * B;
+                if (bl < nblk) {
+                    if (V == 1) {
+                        w[i][0] = __ldcs(src + lane);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < V / 4; ++h) {
+                            const float4 v = __ldcs(reinterpret_cast<const float4 *>(src + 128 * h) + lane);
+                            w[i][4 * h] = v.x, w[i][4 * h + 1] = v.y, w[i][4 * h + 2] = v.z, w[i][4 * h + 3] = v.w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < V; ++k) w[i][k] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kQbUnroll; ++i) {
+                const int bl = 8 * (kQbUnroll * c + i) + warp;
+                if (bl >= nblk) break;                           // warp-uniform
+                // max |w| on the bit patterns: NaN and Inf sort above every finite value
+                uint32_t m = 0;
+#pragma unroll
+                for (int k = 0; k < V; ++k) m = max(m, __float_as_uint(w[i][k]) & 0x7fffffffu);
+                const uint32_t ab = __reduce_max_sync(0xffffffffu, m);
+                const float a = __uint_as_float(ab);
+                float tau = kExactHalf ? next_up(__double2float_rd(__dmul_rn(hk, (double)a)))
+                                       : exact_threshold(c_lo, c_hi, a);
+                if (lane >= 15) tau = __uint_as_float(0x7f800000u);
+                const bool fast = use_bins && ab >= 0x0d800000u && ab <= 0x71800000u;   // warp-uniform
+                uint32_t qv[V];
+                if (fast) {
+                    const float kr = __fmul_rn(kBinK, rcp_approx(a));
+#pragma unroll
+                    for (int k = 0; k < V; ++k) {
+                        const float y = fmaf(w[i][k], kr, kBinC);
+                        const uint32_t jt = __shfl_sync(0xffffffffu, lut, (int)__float_as_uint(y));
+                        const float t = __shfl_sync(0xffffffffu, tau, (int)jt);
+                        qv[k] = jt + (w[i][k] >= t ? 1u : 0u);
+                    }
+                } else {
+                    float t[15];
+#pragma unroll
+                    for (int k = 0; k < 15; ++k) t[k] = __shfl_sync(0xffffffffu, tau, k);
+#pragma unroll
+                    for (int k = 0; k < V; ++k) qv[k] = ab == 0u ? (uint32_t)zero_idx : level_index(w[i][k], t);
+                }
+                uint8_t *dst = packed + (b0 + bl) * (B / 2);
+                if (V == 1) {
+                    // even lane 2i: byte i = (q_2i << 4) | q_2i+1; lane 8k gathers bytes 4k .. 4k+3
+                    const uint32_t nx = __shfl_down_sync(0xffffffffu, qv[0], 1);
+                    const uint32_t byte = ((qv[0] << 4) | nx) & 0xffu;
+                    const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 2);
+                    const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 4);
+                    const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 6);
+                    if ((lane & 7) == 0)
+                        *reinterpret_cast<uint32_t *>(dst + lane / 2) = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < V / 4; ++h) {
+                        const uint32_t v = qv[4 * h + 1] | (qv[4 * h] << 4) | (qv[4 * h + 3] << 8) | (qv[4 * h + 2] << 12);
+                        *reinterpret_cast<uint16_t *>(dst + 64 * h + 2 * lane) = (uint16_t)v;
+                    }
+                }
+                if (lane == 0) {
+                    s_a[bl] = a;
+                    if (!dq) absmax[b0 + bl] = a;
+                    bad_any |= ab >= 0x7f800000u;
+                }
             }
         }
+    } else if (nblk == 256) {
+        run(BoolTag<true>{});
+    } else {
+        run(BoolTag<false>{});
     }
     if (bad_any && status) atomicOr(status, QLORA_STATUS_NONFINITE);
     if (dq) {
