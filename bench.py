@@ -786,7 +786,27 @@ def decode_lines(args, q, lib, torch, dev, hbm, flush):
         del w
     res["merge"] = merge_line(q, lib, torch, dev, hbm, flush)
     res["block_sizes"] = block_size_lines(q, lib, torch, dev, hbm, flush)
+    res["write_only"] = write_only_line(torch, dev, hbm)
     return res
+
+
+def write_only_line(torch, dev, hbm):
+    """Context for the write-dominated dequantize kernels: a 1 GiB memset
+    (torch's fill, no reads) timed with events, in GB/s and as a fraction of
+    the measured copy bandwidth."""
+    buf = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        buf.zero_()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a, b in ev:
+        a.record()
+        buf.zero_()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    gbps = buf.numel() / (ms / 1e3) / 1e9
+    del buf
+    return {"bytes": 1 << 30, "ms": ms, "GBps": gbps, "frac_of_copy_peak": gbps / hbm}
 
 
 def block_size_lines(q, lib, torch, dev, hbm, flush):
