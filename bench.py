@@ -341,6 +341,7 @@ def run_ours(args, rank, world, dist):
     ws_b = torch.empty(q.workspace_size(M, w, r, 1, 1), dtype=torch.uint8, device=dev)
     y = torch.empty(M, Dout, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    FLUSH_REPEAT = 4
 
     def step():
         q.quantize(W, double_quant=True, out=w)
@@ -362,6 +363,10 @@ def run_ours(args, rank, world, dist):
     # outside graph capture).
     use_graph = world == 1 and not args.eager
     graph, per_step_launches = None, 0
+    # Inside the graph only the tensor-core GEMM's launches carry timing events:
+    # each event record is a graph node of its own and costs about 4 us of step
+    # time, so the graph holds the four the roofline needs and the quantize
+    # kernel is timed alone right after the timed region.
     if use_graph:
         side = torch.cuda.Stream(dev)
         side.wait_stream(torch.cuda.current_stream(dev))
@@ -369,6 +374,7 @@ def run_ours(args, rank, world, dist):
             step()
         torch.cuda.current_stream(dev).wait_stream(side)
         lib.qlora_profile_reset()
+        lib.qlora_profile_kinds(1 << 0)
         lib.qlora_profile_enable(1)
         step()                       # creates the library's timing events outside the capture
         torch.cuda.synchronize()
@@ -377,6 +383,7 @@ def run_ours(args, rank, world, dist):
         with torch.cuda.graph(graph):
             step()
         lib.qlora_profile_enable(0)
+        lib.qlora_profile_kinds(0xFFFFFFFF)
         per_step_launches = lib.qlora_launch_count()
         for _ in range(args.warmup):
             graph.replay()
@@ -390,33 +397,35 @@ def run_ours(args, rank, world, dist):
         pass
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    umma_n, umma_ms = ctypes.c_int64(), ctypes.c_double()
+    gemm_each = []    # GEMM launch durations (ms) in launch order: forward, dX of each step
     quant_n, quant_ms = ctypes.c_int64(), ctypes.c_double()
-    acc = {"umma_n": 0, "umma_ms": 0.0, "quant_n": 0, "quant_ms": 0.0}
+    acc = {"failed": False}
+
+    def read_gemm_events(cap):
+        arr = (ctypes.c_double * cap)()
+        n = ctypes.c_int64()
+        if lib.qlora_profile_read_each(0, cap, arr, ctypes.byref(n)) != 0 or n.value > cap:
+            acc["failed"] = True
+            return []
+        return list(arr[:n.value])
+
     if not use_graph:
         lib.qlora_profile_reset()
         lib.qlora_profile_enable(1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    def read_replay_events():
-        # the last replay's kernel events (the graph re-records the same events)
-        rc0 = lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
-        rc2 = lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
-        if rc0 or rc2:
-            acc["failed"] = True
-        acc["umma_n"] += umma_n.value
-        acc["umma_ms"] += umma_ms.value
-        acc["quant_n"] += quant_n.value
-        acc["quant_ms"] += quant_ms.value
-
     with ClockSampler(uuid) as clk:
         for i in range(args.steps):
             if use_graph and i > 0:
                 torch.cuda.synchronize()          # the previous replay has finished
-            flush.zero_()
-            if use_graph and i > 0:
-                read_replay_events()              # while the GPU flushes L2, outside the events
+                gemm_each += read_gemm_events(8)  # its events (each replay records them again)
+            # the L2 flush, outside the events; with a graph it is written four times
+            # so that the replay is submitted while the GPU is still flushing (the
+            # step's device time then excludes the host's graph-launch latency, as
+            # for back-to-back replays)
+            for _ in range(FLUSH_REPEAT if use_graph else 1):
+                flush.zero_()
             starts[i].record()
             if use_graph:
                 graph.replay()
@@ -425,34 +434,49 @@ def run_ours(args, rank, world, dist):
             ends[i].record()
         torch.cuda.synchronize()
         if use_graph:
-            read_replay_events()
+            gemm_each += read_gemm_events(8)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     kernel_timing = "library events inside the timed region"
     if use_graph:
         launches = per_step_launches * args.steps
-        umma_n.value, umma_ms.value = acc["umma_n"], acc["umma_ms"]
-        quant_n.value, quant_ms.value = acc["quant_n"], acc["quant_ms"]
         del graph
-        if acc.get("failed"):
+        if acc["failed"] or len(gemm_each) != 2 * args.steps:
             # the graph's timing events could not be read: the kernels' times
             # come from the same number of eager steps right after
             kernel_timing = "library events over an eager pass of the same steps"
+            acc["failed"] = False
             lib.qlora_profile_reset()
+            lib.qlora_profile_kinds(1 << 0)
             lib.qlora_profile_enable(1)
             for _ in range(args.steps):
                 flush.zero_()
                 step()
             torch.cuda.synchronize()
             lib.qlora_profile_enable(0)
-            lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
-            lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+            lib.qlora_profile_kinds(0xFFFFFFFF)
+            gemm_each = read_gemm_events(2 * args.steps + 8)
+        # the quantize kernel alone, L2 flushed before each launch
+        lib.qlora_profile_reset()
+        lib.qlora_profile_kinds(1 << 2)
+        lib.qlora_profile_enable(1)
+        for _ in range(10):
+            flush.zero_()
+            q.quantize(W, double_quant=True, out=w)
+        torch.cuda.synchronize()
+        lib.qlora_profile_enable(0)
+        lib.qlora_profile_kinds(0xFFFFFFFF)
+        lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+        quant_timing = "the kernel alone after the timed region, L2 flushed before each of 10 launches"
     else:
         lib.qlora_profile_enable(0)
         launches = lib.qlora_launch_count()
-        lib.qlora_profile_read(0, ctypes.byref(umma_n), ctypes.byref(umma_ms))
+        gemm_each = read_gemm_events(2 * args.steps + 8)
         lib.qlora_profile_read(2, ctypes.byref(quant_n), ctypes.byref(quant_ms))
+        quant_timing = "library events inside the timed region"
+    umma_n = len(gemm_each)
+    umma_ms = sum(gemm_each)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
     if world > 1:
@@ -465,7 +489,7 @@ def run_ours(args, rank, world, dist):
     # dominant kernel: the tcgen05 GEMM (forward and dX launches)
     umma_flops = args.steps * (2 * M * Din * Dout + 2 * M * Dout * r      # forward + adapter ext
                                + 2 * M * Dout * Din + 2 * M * Din * r)    # dX + adapter ext
-    umma_tf = umma_flops / (umma_ms.value / 1e3) / 1e12 if umma_ms.value > 0 else None
+    umma_tf = umma_flops / (umma_ms / 1e3) / 1e12 if umma_ms > 0 else None
     traffic = stored_traffic("umma_gemm.cu", "k_umma_qgemm_up_proj_4096x11008_M4096.md")
     # Peak: the burst GEMM figure while the SM clock held its maximum with no
     # power cap during the timed region (short steps do not reach the cap),
@@ -479,12 +503,22 @@ def run_ours(args, rank, world, dist):
             "traffic": traffic,
             "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'} ({peak_src})",
             "frac_of_sustained": (umma_tf / tf_sus) if umma_tf else None,
-            "launches": int(umma_n.value), "timing": kernel_timing,
-            "share_of_step": umma_ms.value / sum(step_ms) if step_ms else None}
+            "launches": umma_n, "timing": kernel_timing,
+            "share_of_step": umma_ms / sum(step_ms) if step_ms else None}
+    # the same kernel split by launch: forward (M x Dout outputs, 4.65 waves of
+    # 74 CTA pairs at the headline) and dX (M x Din outputs, 1.73 waves)
+    if umma_n >= 2 and umma_n % 2 == 0:
+        f_ms = sum(gemm_each[0::2]) / (umma_n // 2)
+        d_ms = sum(gemm_each[1::2]) / (umma_n // 2)
+        f_tf = (2 * M * Din * Dout + 2 * M * Dout * r) / (f_ms / 1e3) / 1e12
+        d_tf = (2 * M * Dout * Din + 2 * M * Din * r) / (d_ms / 1e3) / 1e12
+        roof["by_launch"] = {
+            "forward": {"ms_per_launch": f_ms, "achieved": f_tf, "frac": f_tf / tf_peak},
+            "dX": {"ms_per_launch": d_ms, "achieved": d_tf, "frac": d_tf / tf_peak}}
     qbytes = Din * Dout * 4 + weight_bytes(Din, Dout)
     quant = {"kernel": "k_nf4_quantize_fast", "bound": "hbm",
              "achieved": qbytes / (quant_ms.value / quant_n.value / 1e3) / 1e9 if quant_n.value else None,
-             "peak": hbm, "unit": "GB/s"}
+             "peak": hbm, "unit": "GB/s", "timing": quant_timing}
     if quant["achieved"]:
         quant["frac"] = quant["achieved"] / hbm
 
@@ -580,7 +614,8 @@ def run_ours(args, rank, world, dist):
         "data": "synthetic (seeded numpy PCG64; W~t5*0.02, x,dY~N(0,1), A~N(0,1/r), B~N(0,1e-4))",
         "config": {"workload": WORKLOAD, "M": M, "Din": Din, "Dout": Dout, "r": r, "alpha": alpha,
                    "double_quant": True, "parallelism": f"dp{world}",
-                   "l2": "flushed between timed steps (256 MB write, outside the step events)",
+                   "l2": ("flushed between timed steps (256 MB written 4 times, outside the step events)"
+                          if use_graph else "flushed between timed steps (256 MB write, outside the step events)"),
                    "timing": ("each timed step one replay of the step captured in a CUDA graph"
                               if use_graph else "eager steps")},
         "roofline": roof,

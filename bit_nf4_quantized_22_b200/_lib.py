@@ -20,6 +20,7 @@ EXPORTS = (
     "qlora_strerror", "qlora_version", "qlora_check_codebook", "nf4_quantize",
     "nf4_dequantize", "qlora_workspace_size", "qlora_forward", "qlora_backward",
     "qlora_launch_count", "qlora_profile_enable", "qlora_profile_reset", "qlora_profile_read",
+    "qlora_profile_kinds", "qlora_profile_read_each",
     "qlora_forward_noalloc", "qlora_merge", "qlora_selftest_wait_timeout", "nf4_dequantize_dtype",
     "nf4_codebook", "fp4_codebook",
 )
@@ -91,6 +92,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_profile_reset.argtypes = []
     lib.qlora_profile_read.restype = ctypes.c_int
     lib.qlora_profile_read.argtypes = [i32, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
+    lib.qlora_profile_kinds.restype = None
+    lib.qlora_profile_kinds.argtypes = [ctypes.c_uint32]
+    lib.qlora_profile_read_each.restype = ctypes.c_int
+    lib.qlora_profile_read_each.argtypes = [i32, i64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
     lib.qlora_forward_noalloc.restype = ctypes.c_int
     lib.qlora_forward_noalloc.argtypes = [P, i64, W, P, P, P, i32, ctypes.c_float, i32, P, P, P, P]
     lib.qlora_selftest_wait_timeout.restype = ctypes.c_int

@@ -12,6 +12,7 @@ namespace qlora {
 namespace {
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_on{0};
+std::atomic<uint32_t> g_kinds{0xffffffffu};   // kinds that are timed while enabled
 std::mutex g_mu;
 struct Pairs {
     std::vector<cudaEvent_t> start, stop;
@@ -60,8 +61,12 @@ static void record_timing_event(cudaEvent_t ev, cudaStream_t st) {
         cudaEventRecord(ev, st);
 }
 
+static bool timed(int kind) {
+    return g_on.load(std::memory_order_relaxed) && ((g_kinds.load(std::memory_order_relaxed) >> kind) & 1u);
+}
+
 void prof_begin(int kind, cudaStream_t st) {
-    if (!g_on.load(std::memory_order_relaxed)) return;
+    if (!timed(kind)) return;
     std::lock_guard<std::mutex> lk(g_mu);
     Pairs &p = g_pairs[kind];
     if (p.used == p.start.size()) {
@@ -75,7 +80,7 @@ void prof_begin(int kind, cudaStream_t st) {
 }
 
 void prof_end(int kind, cudaStream_t st) {
-    if (!g_on.load(std::memory_order_relaxed)) return;
+    if (!timed(kind)) return;
     std::lock_guard<std::mutex> lk(g_mu);
     Pairs &p = g_pairs[kind];
     if (p.used < p.start.size()) {
@@ -89,6 +94,8 @@ void prof_end(int kind, cudaStream_t st) {
 extern "C" {
 
 void qlora_profile_enable(int on) { qlora::g_on.store(on ? 1 : 0); }
+
+void qlora_profile_kinds(uint32_t mask) { qlora::g_kinds.store(mask); }
 
 void qlora_profile_reset(void) {
     std::lock_guard<std::mutex> lk(qlora::g_mu);
@@ -114,6 +121,25 @@ int qlora_profile_read(int32_t kind, int64_t *launches, double *total_ms) {
     }
     *launches = (int64_t)p.used;
     *total_ms = t;
+    return QLORA_OK;
+}
+
+int qlora_profile_read_each(int32_t kind, int64_t cap, double *ms_each, int64_t *launches) {
+    if (kind < 0 || kind >= qlora::kProfKinds || cap < 0 || !launches || (cap > 0 && !ms_each))
+        return QLORA_EINVAL;
+    std::lock_guard<std::mutex> lk(qlora::g_mu);
+    auto &p = qlora::g_pairs[kind];
+    const size_t n = p.used < (size_t)cap ? p.used : (size_t)cap;
+    for (size_t i = 0; i < n; ++i) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(p.stop[i]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, p.start[i], p.stop[i]) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return QLORA_ECUDA;
+        }
+        ms_each[i] = ms;
+    }
+    *launches = (int64_t)p.used;
     return QLORA_OK;
 }
 

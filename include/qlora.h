@@ -307,12 +307,25 @@ int64_t qlora_launch_count(void);
  * 4 merge kernel. */
 void qlora_profile_enable(int on);
 
+/* Which kinds are timed while profiling is enabled: bit k for kind k (all by
+ * default).  Each timed launch adds an event pair to the stream, and inside a
+ * CUDA graph each event record is a node of its own, so a benchmark times
+ * only the kinds it reads. */
+void qlora_profile_kinds(uint32_t mask);
+
 /* Forget recorded events and zero the launch count (host only). */
 void qlora_profile_reset(void);
 
 /* Number of timed launches of `kind` since the reset and their summed
  * duration in milliseconds; waits for the recorded events to complete. */
 int qlora_profile_read(int32_t kind, int64_t *launches, double *total_ms);
+
+/* The durations (ms) of the first min(cap, launches) timed launches of `kind`
+ * since the reset, in launch order, into ms_each (caller-owned host array of
+ * cap doubles); *launches receives the count of timed launches.  Waits for
+ * the events like qlora_profile_read.  EINVAL for an unknown kind, cap < 0, a
+ * null count, or a null array with cap > 0. */
+int qlora_profile_read_each(int32_t kind, int64_t cap, double *ms_each, int64_t *launches);
 
 #ifdef __cplusplus
 }
