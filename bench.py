@@ -163,11 +163,14 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "source": self.source}
-        reasons = set()
+        reasons, counts = set(), {}
         for _, r, _ in self.samples:
             reasons |= r
+            for n in r:
+                counts[n] = counts.get(n, 0) + 1
         return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "reason_samples": counts,
                 "power_w_max": max(p for _, _, p in self.samples),
                 "samples": len(self.samples), "source": self.source}
 
@@ -491,11 +494,12 @@ def run_ours(args, rank, world, dist):
                                + 2 * M * Dout * Din + 2 * M * Din * r)    # dX + adapter ext
     umma_tf = umma_flops / (umma_ms / 1e3) / 1e12 if umma_ms > 0 else None
     traffic = stored_traffic("umma_gemm.cu", "k_umma_qgemm_up_proj_4096x11008_M4096.md")
-    # Peak: the burst GEMM figure while the SM clock held its maximum with no
-    # power cap during the timed region (short steps do not reach the cap),
-    # else the sustained, power-capped figure.
+    # Peak: the burst GEMM figure while the SM clock held (within 5%) its
+    # maximum during the timed region (short steps do not reach the power cap),
+    # else the sustained, power-capped figure.  A power-cap reason seen while
+    # the clock stays at its maximum is reported in `clocks`, not acted on.
     csum = clk.summary()
-    capped = ("sw_power_cap" in csum.get("reasons", []) or csum.get("sm_mhz") is None
+    capped = (csum.get("sm_mhz") is None
               or (csum.get("sm_max_mhz") and csum["sm_mhz"] < 0.95 * csum["sm_max_mhz"]))
     tf_peak = tf_sus if capped else tf_burst
     roof = {"bound": "tensor", "kernel": "k_umma_qgemm", "achieved": umma_tf, "peak": tf_peak,

@@ -347,45 +347,48 @@ k_umma_qgemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         // ---------------------------------------------------------- epilogue
         // TMEM -> registers -> bf16 -> the idle stage ring, as 128-byte-swizzled
         // [128 rows][64 columns] boxes (half hh at hh * 64 KB, box j at + 16 KB j),
-        // then TMA stores of whole boxes: coalesced, and clipped at M and N.
+        // then TMA stores of whole boxes: coalesced, and clipped at M and N.  A
+        // box is stored as soon as the four warps of its half have written it,
+        // so the stores overlap the remaining TMEM reads.
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(acc_bar, 0, abort_flag));
-        if (ok) {
-            tc_fence_after();
+        if (ok) tc_fence_after();
+        else *abort_flag = 1;
+        {
             const int q = warp & 3;                       // TMEM lane quarter of this warp
             const int hh = (warp - 2) >> 2;               // accumulator (MMA half) of this warp
             const uint32_t L = 32 * q + lane;             // tile row = TMEM lane
             const uint32_t stile = base + hh * 65536 + L * 128;
+            const bool storer = q == 0 && lane == 0;      // one thread per half issues its boxes
+            const int64_t y = m0 + 256 * hh + 128 * rank;
             for (int c = 0; c < 8; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + hh * 256 + c * 32, v);
-                const uint32_t box = stile + (c >> 1) * 16384;
+                if (ok) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + hh * 256 + c * 32, v);
+                    const uint32_t box = stile + (c >> 1) * 16384;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t chunk = 4 * (c & 1) + i;
-                    const bool f16 = p.f16;
-                    sts128(box + ((chunk ^ (L & 7)) << 4),
-                           pack2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), f16),
-                           pack2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), f16),
-                           pack2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), f16),
-                           pack2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), f16));
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t chunk = 4 * (c & 1) + i;
+                        const bool f16 = p.f16;
+                        sts128(box + ((chunk ^ (L & 7)) << 4),
+                               pack2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]), f16),
+                               pack2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]), f16),
+                               pack2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]), f16),
+                               pack2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]), f16));
+                    }
+                }
+                if (c & 1) {
+                    // box c / 2 of this half is complete once its four warps are here
+                    fence_proxy_async();
+                    asm volatile("bar.sync %0, 128;\n" ::"r"(2 + hh) : "memory");
+                    const int64_t x = n0 + 64 * (c >> 1);
+                    if (ok && storer && y < p.M && x < p.N)
+                        tma_store_2d(&tmY, base + hh * 65536 + (c >> 1) * 16384, (int)x, (int)y);
                 }
             }
-            fence_proxy_async();                          // the writes, visible to the TMA engine
-        } else {
-            *abort_flag = 1;
-        }
-        asm volatile("bar.sync 1, %0;\n" ::"n"(kDqThreads));
-        if (ok && threadIdx.x == 64) {
-            for (int hh = 0; hh < 2; ++hh) {
-                const int64_t y = m0 + 256 * hh + 128 * rank;
-                if (y >= p.M) continue;
-                for (int j = 0; j < 4; ++j) {
-                    const int64_t x = n0 + 64 * j;
-                    if (x < p.N) tma_store_2d(&tmY, base + hh * 65536 + j * 16384, (int)x, (int)y);
-                }
+            if (storer) {
+                bulk_commit();
+                bulk_wait_read();
             }
-            bulk_commit();
-            bulk_wait_all();
         }
     }
 
