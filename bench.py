@@ -58,14 +58,22 @@ def peaks():
     return (6650.0, 1590.0, 1400.0, "fallback")
 
 
+def kernel_source_sha(kernel_file):
+    """sha256 over the kernel's source file and the two headers every kernel
+    file includes (common.cuh, tcgen05.cuh), in that order."""
+    h = hashlib.sha256()
+    for f in (kernel_file, "common.cuh", "tcgen05.cuh"):
+        h.update(open(os.path.join(ROOT, "bit_nf4_quantized_22_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
 def stored_traffic(kernel_file, summary):
-    """dram bytes per launch recorded in a profiles/ summary, if the kernel
-    source is unchanged since that capture (sha256 line), else None."""
+    """dram bytes per launch recorded in a profiles/ summary, if the kernel's
+    sources are unchanged since that capture (sha256 line), else None."""
     path = os.path.join(ROOT, "profiles", summary)
-    src = os.path.join(ROOT, "bit_nf4_quantized_22_b200", "csrc", kernel_file)
     if not os.path.exists(path):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = kernel_source_sha(kernel_file)
     vals = {}
     for line in open(path):
         if line.startswith("bench:"):

@@ -95,11 +95,21 @@ struct ProdTable {
     uint32_t hi[4];   // hi[i] byte k = high byte of entry 4i+k
 };
 
+// The products RN32(a_hat c_j) come two at a time from the packed fp32x2
+// multiply (each lane rounded as a scalar multiply would be).
 __device__ __forceinline__ void build_table(float ah, const Codebook &cb, ProdTable &t, bool f16 = false) {
     uint32_t p[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        p[i] = pack2(__fmul_rn(ah, cb.c[2 * i]), __fmul_rn(ah, cb.c[2 * i + 1]), f16);
+    for (int i = 0; i < 8; ++i) {
+        float lo, hi;
+        asm("{\n\t.reg .b64 ra, rc, rd;\n\t"
+            "mov.b64 ra, {%2, %2};\n\t"
+            "mov.b64 rc, {%3, %4};\n\t"
+            "mul.rn.f32x2 rd, ra, rc;\n\t"
+            "mov.b64 {%0, %1}, rd;\n\t}"
+            : "=f"(lo), "=f"(hi) : "f"(ah), "f"(cb.c[2 * i]), "f"(cb.c[2 * i + 1]));
+        p[i] = pack2(lo, hi, f16);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         t.lo[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x6420);
