@@ -90,6 +90,27 @@ __device__ __forceinline__ uint16_t enc16(float v, bool f16) {
 // lookup of four 4-bit indices is two byte-permutes per plane plus a select
 // on the index's top bit: no shared memory, no local memory.
 // ---------------------------------------------------------------------------
+// (r0, r1) = (RN32(a b0), RN32(a b1)) as one packed fp32x2 multiply.
+__device__ __forceinline__ void mul2_rn(float a, float b0, float b1, float &r0, float &r1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r0), "=f"(r1) : "f"(a), "f"(b0), "f"(b1));
+}
+
+// (r0, r1) = (fma(a, b0, c0), fma(a, b1, c1)), each correctly rounded, as one packed fp32x2 fma.
+__device__ __forceinline__ void fma2_rn(float a, float b0, float b1, float c0, float c1, float &r0, float &r1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "mov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r0), "=f"(r1) : "f"(a), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 struct ProdTable {
     uint32_t lo[4];   // lo[i] byte k = low byte of entry 4i+k
     uint32_t hi[4];   // hi[i] byte k = high byte of entry 4i+k
@@ -102,12 +123,7 @@ __device__ __forceinline__ void build_table(float ah, const Codebook &cb, ProdTa
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         float lo, hi;
-        asm("{\n\t.reg .b64 ra, rc, rd;\n\t"
-            "mov.b64 ra, {%2, %2};\n\t"
-            "mov.b64 rc, {%3, %4};\n\t"
-            "mul.rn.f32x2 rd, ra, rc;\n\t"
-            "mov.b64 {%0, %1}, rd;\n\t}"
-            : "=f"(lo), "=f"(hi) : "f"(ah), "f"(cb.c[2 * i]), "f"(cb.c[2 * i + 1]));
+        mul2_rn(ah, cb.c[2 * i], cb.c[2 * i + 1], lo, hi);
         p[i] = pack2(lo, hi, f16);
     }
 #pragma unroll

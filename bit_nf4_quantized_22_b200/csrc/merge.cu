@@ -238,10 +238,13 @@ k_merge(const uint8_t *__restrict__ packed, ScaleSrc sc, Codebook cb,
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const uint32_t byte = ((nt < 4 ? m.p.x : m.p.y) >> (8 * (nt & 3))) & 0xffu;
-                // both weights rounded to the compute dtype by one paired conversion
-                const uint32_t w = pack2(__fmul_rn(ah, cbs[byte >> 4]), __fmul_rn(ah, cbs[byte & 15]), F16);
-                o[nt] = pack2(fmaf(sg, acc[nt][2 * hr], lo16(w, F16)), fmaf(sg, acc[nt][2 * hr + 1], hi16(w, F16)),
-                              F16);
+                // both weights rounded to the compute dtype by one paired conversion; the
+                // products and the adapter fmas as packed fp32x2 pairs
+                float p0, p1, y0, y1;
+                mul2_rn(ah, cbs[byte >> 4], cbs[byte & 15], p0, p1);
+                const uint32_t w = pack2(p0, p1, F16);
+                fma2_rn(sg, acc[nt][2 * hr], acc[nt][2 * hr + 1], lo16(w, F16), hi16(w, F16), y0, y1);
+                o[nt] = pack2(y0, y1, F16);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(W_out + row * Din + kc + 16 * t);
             __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
