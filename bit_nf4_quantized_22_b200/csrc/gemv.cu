@@ -743,13 +743,35 @@ constexpr int kBsRed = 8 * 32 * 32 * 4;                    // odd-parity warps' 
 constexpr int kBsSmem = kStLut + kBsStages * kBsStage + kBsRed + 1024 + 256;
 static_assert(kBsStage % 1024 == 0, "stages keep 1 KB swizzle alignment");
 
+// (r0, r1) = (a0 op b0, a1 op b1) as one packed fp32x2 operation, each lane rounded as
+// the scalar operation would be.
+__device__ __forceinline__ void mul2_pair(float a0, float a1, float b0, float b1, float &r0, float &r1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2_pair(float a0, float a1, float b0, float b1, float &r0, float &r1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // dY pair v (two 16-bit values of the compute dtype) times two scales, as
 // hi + lo pairs of that dtype: hi = RN(d), lo = RN(d - hi), d = RN32(dY * a_hat).
+// The two products and the two differences each take one packed operation.
 template <bool F16>
 __device__ __forceinline__ void split_scaled(uint32_t v, float s0, float s1, uint32_t &hi, uint32_t &lo) {
-    const float d0 = lo16(v, F16) * s0, d1 = hi16(v, F16) * s1;
+    float d0, d1, e0, e1;
+    mul2_pair(lo16(v, F16), hi16(v, F16), s0, s1, d0, d1);
     hi = pack2(d0, d1, F16);
-    lo = pack2(d0 - lo16(hi, F16), d1 - hi16(hi, F16), F16);
+    sub2_pair(d0, d1, lo16(hi, F16), hi16(hi, F16), e0, e1);
+    lo = pack2(e0, e1, F16);
 }
 
 // The CTA (of G, over T units) whose contiguous range holds unit u.
